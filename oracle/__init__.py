@@ -1,0 +1,210 @@
+"""fp64 CPU oracle for the MSA hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library
+(``block_sparse_long_branch_b200``) never imports it and has no CPU fallback.
+
+The arithmetic lives in ``msa_oracle.c`` (plain loops, fp64); this module only
+marshals numpy arrays through ctypes.  Each wrapper names the passage of the
+pages it follows; the C file carries the same citations.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I32 = ctypes.c_int32
+        lib.msa_oracle_pooled_scores.argtypes = [P, P, I64, P, I32, I32, I32, I64, P]
+        lib.msa_oracle_pooled_scores.restype = None
+        lib.msa_oracle_select_blocks.argtypes = [P, P, I64, I32, I64, I32, I32, P]
+        lib.msa_oracle_select_blocks.restype = None
+        lib.msa_oracle_block_attention.argtypes = [P, P, I64, P, P, I32, I32, I32, I32, I32,
+                                                   ctypes.c_double, P, P, P, P]
+        lib.msa_oracle_block_attention.restype = None
+        lib.msa_oracle_block_query_lists.argtypes = [P, I64, I32, I64, I32, P, P]
+        lib.msa_oracle_block_query_lists.restype = I64
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def as_bf16_bits(x) -> np.ndarray:
+    """A bf16 torch tensor (or uint16 array) as a contiguous uint16 array."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch
+    assert x.dtype == torch.bfloat16
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy()
+                                .view(np.uint16))
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def pooled_scores(qi_rows, pos, k_idx, block: int, nb_out: int) -> np.ndarray:
+    """Index Branch scoring + per-block max over visible tokens.
+
+    ai-tool-zukan MiniMax MSA guide, section "2段階構造の中身": visible key
+    tokens are scored, then max-pooled to the block level.
+    qi_rows [n,G,di] bf16, pos [n] int64, k_idx [T,di] bf16 -> [n,G,nb_out] f64.
+    """
+    lib = _load()
+    qi = as_bf16_bits(qi_rows)
+    ki = as_bf16_bits(k_idx)
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int64))
+    n, G, di = qi.shape
+    assert ki.shape[1] == di and pos.shape == (n,)
+    assert n == 0 or ki.shape[0] > int(pos.max())
+    out = np.empty((n, G, nb_out), dtype=np.float64)
+    lib.msa_oracle_pooled_scores(_ptr(qi), _ptr(pos), n, _ptr(ki), G, di, block, nb_out,
+                                 _ptr(out))
+    return out
+
+
+def select_blocks(pooled: np.ndarray, pos, block: int, top_k: int) -> np.ndarray:
+    """Forced-local top-k per (query, group), ids ascending and -1 padded.
+
+    ai-tool-zukan MiniMax MSA guide, sections "2段階構造の中身" (top-k per query
+    and group, local block always included) and
+    "クエリを含むローカルブロックの強制取り込み".
+    """
+    lib = _load()
+    pooled = np.ascontiguousarray(pooled, dtype=np.float64)
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int64))
+    n, G, nb_in = pooled.shape
+    assert n == 0 or int(pos.max()) // block < nb_in
+    ids = np.empty((n, G, top_k), dtype=np.int32)
+    lib.msa_oracle_select_blocks(_ptr(pooled), _ptr(pos), n, G, nb_in, block, top_k,
+                                 _ptr(ids))
+    return ids
+
+
+def block_attention(q_rows, pos, k, v, ids: np.ndarray, scale: float, block: int,
+                    partials: bool = False):
+    """Main Branch: exact softmax over the selected blocks' visible keys.
+
+    ai-tool-zukan MiniMax MSA guide, section "Index BranchとMain Branchの役割分担".
+    q_rows [n,H,d], k/v [T,G,d] bf16, ids [n,G,top_k] -> out [n,H,d] f64
+    (and, with ``partials``, lse [n,H,top_k] and o [n,H,top_k,d]).
+    """
+    lib = _load()
+    qb = as_bf16_bits(q_rows)
+    kb = as_bf16_bits(k)
+    vb = as_bf16_bits(v)
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int64))
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    n, H, d = qb.shape
+    G = kb.shape[1]
+    top_k = ids.shape[2]
+    assert ids.shape == (n, G, top_k) and kb.shape == vb.shape and kb.shape[2] == d
+    assert H % G == 0
+    out = np.empty((n, H, d), dtype=np.float64)
+    lse = np.empty((n, H, top_k), dtype=np.float64) if partials else None
+    po = np.empty((n, H, top_k, d), dtype=np.float64) if partials else None
+    lib.msa_oracle_block_attention(_ptr(qb), _ptr(pos), n, _ptr(kb), _ptr(vb), H, G, d, block,
+                                   top_k, float(scale), _ptr(ids), _ptr(out), _ptr(lse),
+                                   _ptr(po))
+    if partials:
+        return out, lse, po
+    return out
+
+
+def block_query_lists(ids: np.ndarray, nb: int):
+    """Per-(group, key block) lists of (query t, slot r), ascending t.
+
+    tnkblog MiniMax M3 / MSA post, section "MSA の実装": key blocks are the
+    outer loop and the queries that hit a block are gathered.
+    Returns (row_ptr [G*nb+1] int32, entries [nnz] int32 with (t<<5)|r).
+    """
+    lib = _load()
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    N, G, top_k = ids.shape
+    assert top_k <= 32
+    row_ptr = np.empty(G * nb + 1, dtype=np.int32)
+    entries = np.empty(N * G * top_k, dtype=np.int32)
+    total = lib.msa_oracle_block_query_lists(_ptr(ids), N, G, nb, top_k, _ptr(row_ptr),
+                                             _ptr(entries))
+    if total < 0:
+        raise ValueError("block id out of range")
+    return row_ptr, entries[:total].copy()
+
+
+# ---------------------------------------------------------------------------
+# Whole-path helpers (composition of the steps above, nothing more).
+# ---------------------------------------------------------------------------
+
+def prefill(q, k, v, q_idx, k_idx, *, block: int, top_k: int, scale: float, rows=None,
+            partials: bool = False) -> dict:
+    """Index Branch + Main Branch for the query rows ``rows`` (default: all).
+
+    Returns dict(rows, pooled [n,G,nb], ids [n,G,top_k], out [n,H,d] f64, and
+    with ``partials`` also lse/o per slot).
+    """
+    N = q.shape[0]
+    nb = (N + block - 1) // block
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    qi = as_bf16_bits(q_idx)[rows]
+    pooled = pooled_scores(qi, rows, k_idx, block, nb)
+    ids = select_blocks(pooled, rows, block, top_k)
+    qr = as_bf16_bits(q)[rows]
+    res = dict(rows=rows, pooled=pooled, ids=ids)
+    if partials:
+        res["out"], res["lse"], res["o"] = block_attention(qr, rows, k, v, ids, scale, block,
+                                                          partials=True)
+    else:
+        res["out"] = block_attention(qr, rows, k, v, ids, scale, block)
+    return res
+
+
+def decode(q, q_idx, k_cache, v_cache, k_idx_cache, cu_seqlens, *, block: int, top_k: int,
+           scale: float, seqs=None) -> dict:
+    """One decode step: sequence b's query sits at position L_b - 1 of its cache.
+
+    The pages give no separate decode algorithm (zhaixingw M3 review, section
+    "这套注意力到底怎么省的", reports decode speed only); the plainest reading is
+    the same two branches for the single newest query row.
+    Returns dict(ids [B,G,top_k], out [B,H,d], pooled list per sequence).
+    """
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    B = len(cu) - 1
+    seqs = range(B) if seqs is None else seqs
+    qb = as_bf16_bits(q)
+    qib = as_bf16_bits(q_idx)
+    H, d = qb.shape[1], qb.shape[2]
+    G = qib.shape[1]
+    ids = np.full((B, G, top_k), -1, dtype=np.int32)
+    out = np.full((B, H, d), np.nan)
+    pooled = {}
+    for b in seqs:
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        L = s1 - s0
+        pos = np.array([L - 1], dtype=np.int64)
+        nb = (L + block - 1) // block
+        kb = k_idx_cache[s0:s1]
+        p = pooled_scores(qib[b:b + 1], pos, kb, block, nb)
+        sel = select_blocks(p, pos, block, top_k)
+        o = block_attention(qb[b:b + 1], pos, k_cache[s0:s1], v_cache[s0:s1], sel, scale, block)
+        ids[b] = sel[0]
+        out[b] = o[0]
+        pooled[b] = p[0]
+    return dict(ids=ids, out=out, pooled=pooled)
