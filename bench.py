@@ -1,0 +1,587 @@
+#!/usr/bin/env python3
+"""MSA hot-path benchmark on B200: prefill tokens/s and decode tokens/s.
+
+One step = one msa_prefill over the prefill workload (index branch, query
+lists, Main Branch, merge) plus one msa_decode step over the decode workload
+(16 sequences of 256K cached tokens and one of 1M).  Inputs are seeded
+synthetic tensors (``synth``) resident in HBM; each is larger than the 126 MB
+L2 (Q at 32K is 512 MiB, the decode caches 21 GiB), so no flush is needed
+between steps.  Kernel times come from CUDA events that the library records
+on its own stream at kernel boundaries (msa_set_phase_events).
+
+Prints exactly one JSON line on rank 0.  ``--impl reference`` times the fp64
+CPU oracle on bounded samples of the same workload instead.
+Launch with torchrun for N > 1 GPUs: every rank runs an independent replica
+(the path has no exchange step), ``value`` sums all ranks' tokens over the
+slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MSA prefill tokens/s & decode tokens/s on 1 B200; % of tensor/HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PREFILL_PHASES = ("index_select", "block_query_lists", "main_branch", "merge")
+DECODE_PHASES = ("decode_index", "decode_topk", "decode_attention", "decode_merge")
+
+
+# --------------------------------------------------------------------------
+# algorithmic work (what each kernel must at least do, independent of design)
+# --------------------------------------------------------------------------
+
+def index_flops(N: int, G: int, d_idx: int, block: int = 128) -> float:
+    """2 * d_idx * G * sum_t (keys of the non-local visible blocks of t)."""
+    t = np.arange(N, dtype=np.int64)
+    return 2.0 * d_idx * G * float(((t // block) * block).sum())
+
+
+def dense_flops(N: int, H: int, d: int) -> float:
+    """Dense causal attention over the same heads: 4 * d * H * N(N+1)/2."""
+    return 4.0 * d * H * N * (N + 1) / 2.0
+
+
+def msa_model_flops(N: int, H: int, G: int, d: int, d_idx: int, top_k: int = 16,
+                    block: int = 128) -> float:
+    """Index scoring over every visible token plus the Main Branch budget, per
+    the pages' O(N) dense vs O(k B_k) description (no kernel detail)."""
+    t = np.arange(N, dtype=np.float64)
+    idx = 2.0 * d_idx * G * (t + 1).sum()
+    main = 4.0 * d * H * np.minimum(t + 1, top_k * block).sum()
+    return float(idx + main)
+
+
+def prefill_work(ids: np.ndarray, H: int, d: int, block: int = 128) -> dict:
+    """Exact Main Branch work of one selection ids [N, G, k]."""
+    N, G, k = ids.shape
+    HG = H // G
+    t = np.arange(N, dtype=np.int64)[:, None, None]
+    valid = ids >= 0
+    keys = np.where(valid, np.minimum(block, t - ids.astype(np.int64) * block + 1), 0)
+    slots = int(valid.sum())
+    pairs = slots * HG
+    main_flops = 4.0 * d * HG * float(keys.sum())
+    # gathered q row (2d) + partial o (2d fp16) + lse (4) per (token, head, block)
+    main_bytes = pairs * (2 * d + 2 * d + 4.0)
+    merge_bytes = pairs * (2 * d + 4.0) + N * H * 2.0 * d + N * G * k * 4.0
+    csr_bytes = 3.0 * N * G * k * 4.0
+    return dict(slots=slots, pairs=pairs, main_flops=main_flops, main_bytes=main_bytes,
+                merge_bytes=merge_bytes, csr_bytes=csr_bytes,
+                selected_keys=float(keys.sum()) / max(1, N * G))
+
+
+def decode_work(seq_lens, H: int, G: int, d: int, d_idx: int, ids: np.ndarray,
+                block: int = 128) -> dict:
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    nb = (lens + block - 1) // block
+    scan_keys = float(((nb - 1) * block).sum())
+    idx_bytes = scan_keys * d_idx * 2.0 + len(lens) * G * d_idx * 2.0
+    idx_flops = 2.0 * d_idx * G * scan_keys
+    keys = 0.0
+    for b, L in enumerate(lens):
+        for j in ids[b].ravel():
+            if j >= 0:
+                keys += min(block, int(L) - int(j) * block)
+    attn_bytes = keys * d * 2.0 * 2.0  # K and V rows of each selected block, per group
+    attn_flops = 4.0 * d * (H // G) * keys
+    return dict(idx_bytes=idx_bytes, idx_flops=idx_flops, attn_bytes=attn_bytes,
+                attn_flops=attn_flops, bytes=idx_bytes + attn_bytes)
+
+
+# --------------------------------------------------------------------------
+# environment helpers
+# --------------------------------------------------------------------------
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", target, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, RuntimeError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        loaded = [c for c in sm if c > 0.5 * (max(sm) if sm else 0)]
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(init_group: bool = True):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and init_group:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def reduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (the baseline arm)
+# --------------------------------------------------------------------------
+
+def oracle_prefill_rate(inp, shape, budget_s: float, max_rows: int = 4096, seed: int = 0):
+    """Tokens/s of the oracle over a uniform sample of query rows."""
+    import oracle
+    rows_done, elapsed, n = 0, 0.0, 16
+    rng_seed = seed
+    while elapsed < budget_s and rows_done < max_rows:
+        rows = synth.sample_rows(shape.N, n, seed=rng_seed)[:n]
+        rng_seed += 1
+        t0 = time.perf_counter()
+        oracle.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                       block=shape.block, top_k=shape.top_k, scale=shape.scale, rows=rows)
+        elapsed += time.perf_counter() - t0
+        rows_done += len(rows)
+        n = min(4 * n, max_rows - rows_done) if elapsed < budget_s / 4 else n
+        if n <= 0:
+            break
+    return rows_done / elapsed, rows_done, elapsed
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def host_inputs(shape):
+    """The same seeded inputs, drawn on the host (the oracle's arrays)."""
+    return synth.make_prefill_inputs(shape, device="cpu")
+
+
+# --------------------------------------------------------------------------
+# arms
+# --------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    os.environ.setdefault("OMP_NUM_THREADS", str(cpu_cores()))
+    shape = synth.PREFILL_CONFIGS[args.workload]
+    inp = host_inputs(shape)
+    import oracle
+    rows_per_step = args.ref_rows
+    step_times = []
+    for i in range(args.warmup + args.steps):
+        rows = synth.sample_rows(shape.N, rows_per_step, seed=1000 + i)[:rows_per_step]
+        t0 = time.perf_counter()
+        oracle.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                       block=shape.block, top_k=shape.top_k, scale=shape.scale, rows=rows)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            step_times.append((dt, len(rows)))
+    total_t = sum(t for t, _ in step_times)
+    total_rows = sum(r for _, r in step_times)
+    value = total_rows / total_t
+    sample = (f"{rows_per_step} query rows per step, uniform over positions of the "
+              f"{shape.name} workload (all heads and groups of each row)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args, shape),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": int(os.environ.get(
+            "OMP_NUM_THREADS", cpu_cores())), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def workload_config(args, shape):
+    cfg = {"workload": f"{shape.name}" + ("" if args.no_decode else
+                                          f"+{synth.DECODE_CONFIG.name}"),
+           "N": shape.N, "H": shape.H, "G": shape.G, "d": shape.d, "d_idx": shape.d_idx,
+           "block": shape.block, "top_k": shape.top_k, "needles": shape.n_needles,
+           "l2": "inputs larger than L2 (no flush)", "parallelism": "replicas"}
+    if not args.no_decode:
+        dc = synth.DECODE_CONFIG
+        cfg["decode"] = {"seq_lens": f"16x{dc.seq_lens[0]}+1x{dc.seq_lens[-1]}", "B": dc.B,
+                         "H": dc.H, "G": dc.G, "d": dc.d, "d_idx": dc.d_idx, "top_k": dc.top_k}
+    return cfg
+
+
+def _phase_ms(evs, n_phases):
+    return [evs[i].elapsed_time(evs[i + 1]) for i in range(n_phases)]
+
+
+def run_ours(args, rank, world, local):
+    import block_sparse_long_branch_b200 as msa
+    dev = torch.device("cuda", local)
+    shape = synth.PREFILL_CONFIGS[args.workload]
+    cfg = msa.config(shape.H, shape.G, shape.d, shape.d_idx, top_k=shape.top_k,
+                     block=shape.block, scale=shape.scale)
+    inp = synth.make_prefill_inputs(shape, device=dev, seed=shape.seed + rank)
+    N = shape.N
+    ws = torch.empty(msa.msa_workspace_size(cfg, msa.OP_PREFILL, N), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((N, shape.H, shape.d), dtype=torch.bfloat16, device=dev)
+    ids = torch.empty((N, shape.G, shape.top_k), dtype=torch.int32, device=dev)
+
+    dc = synth.DECODE_CONFIG
+    dec = None
+    if not args.no_decode:
+        dec = synth.make_decode_inputs(dc, device=dev, seed=dc.seed + rank)
+        dcfg = msa.config(dc.H, dc.G, dc.d, dc.d_idx, top_k=dc.top_k, block=dc.block,
+                          scale=dc.scale)
+        cu_dev = dec["cu_seqlens"].to(dev)
+        dws = torch.empty(msa.msa_workspace_size(dcfg, msa.OP_DECODE, dc.total_len, dc.B),
+                          dtype=torch.uint8, device=dev)
+        dout = torch.empty((dc.B, dc.H, dc.d), dtype=torch.bfloat16, device=dev)
+        dids = torch.empty((dc.B, dc.G, dc.top_k), dtype=torch.int32, device=dev)
+        max_len = max(dc.seq_lens)
+
+    def prefill_once():
+        msa.msa_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                        out=out, ids_out=ids, workspace=ws)
+        return msa.msa_last_launch_count()
+
+    def decode_once():
+        msa.msa_decode(dcfg, dec["q"], dec["q_idx"], dec["k_cache"], dec["v_cache"],
+                       dec["k_idx_cache"], cu_dev, max_len, out=dout, ids_out=dids,
+                       workspace=dws)
+        return msa.msa_last_launch_count()
+
+    def mk_events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    # ---- warm-up ----
+    for _ in range(args.warmup):
+        prefill_once()
+        if dec is not None:
+            decode_once()
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_error(ws) == 0, "device error after prefill warm-up"
+    if dec is not None:
+        assert msa.msa_get_device_error(dws) == 0, "device error after decode warm-up"
+
+    pev = [mk_events(5) for _ in range(args.steps)]
+    dev_ev = [mk_events(5) for _ in range(args.steps)]
+    launches = 0
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(args.steps):
+        msa.msa_set_phase_events(pev[i])
+        launches += prefill_once()
+        if dec is not None:
+            msa.msa_set_phase_events(dev_ev[i])
+            launches += decode_once()
+        msa.msa_set_phase_events(None)
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    total_ms = reduce_max(t_start.elapsed_time(t_end), world)
+
+    pre_ph = np.array([_phase_ms(e, 4) for e in pev])          # [K, 4]
+    pre_ms = reduce_max(float(pre_ph.sum(axis=1).mean()), world)
+    if dec is not None:
+        dec_ph = np.array([_phase_ms(e, 4) for e in dev_ev])
+        dec_ms = reduce_max(float(dec_ph.sum(axis=1).mean()), world)
+    assert msa.msa_get_device_error(ws) == 0, "device error in timed prefill"
+
+    # ---- algorithmic work from the selection actually used ----
+    ids_np = ids.cpu().numpy()
+    pw = prefill_work(ids_np, shape.H, shape.d, shape.block)
+    idx_f = index_flops(N, shape.G, shape.d_idx, shape.block)
+    peaks, peak_src = load_peaks()
+    long_region = total_ms > 5000.0
+    tc_peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
+    tc_name = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+    kernels = {}
+
+    def add(name, ms, bound, work, unit_is_bytes):
+        if unit_is_bytes:
+            ach = work / (ms * 1e-3) / 1e9
+            peak, unit = peaks["hbm_gbs"], "GB/s"
+        else:
+            ach = work / (ms * 1e-3) / 1e12
+            peak, unit = tc_peak, "TFLOP/s"
+        kernels[name] = {"ms": ms, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+                         "frac": ach / peak, "work_per_launch": work}
+
+    pm = pre_ph.mean(axis=0)
+    add("index_select", float(pm[0]), "tensor", idx_f, False)
+    add("block_query_lists", float(pm[1]), "hbm", pw["csr_bytes"], True)
+    add("main_branch", float(pm[2]), "hbm", pw["main_bytes"], True)
+    kernels["main_branch"]["tensor_tflops"] = pw["main_flops"] / (pm[2] * 1e-3) / 1e12
+    kernels["main_branch"]["tensor_frac"] = kernels["main_branch"]["tensor_tflops"] / tc_peak
+    add("merge", float(pm[3]), "hbm", pw["merge_bytes"], True)
+    decode_obj = None
+    if dec is not None:
+        dw = decode_work(dc.seq_lens, dc.H, dc.G, dc.d, dc.d_idx, dids.cpu().numpy(), dc.block)
+        dm = dec_ph.mean(axis=0)
+        add("decode_index", float(dm[0]), "hbm", dw["idx_bytes"], True)
+        add("decode_topk", float(dm[1]), "alu", 0.0, True)
+        add("decode_attention", float(dm[2]), "hbm", dw["attn_bytes"], True)
+        add("decode_merge", float(dm[3]), "hbm",
+            dc.B * dc.H * dc.top_k * (2 * dc.d + 4.0) + dc.B * dc.H * dc.d * 2.0, True)
+        dstep_bytes = dw["bytes"]
+        decode_obj = {"value": world * dc.B / (dec_ms * 1e-3), "unit": "tokens/s",
+                      "ms_per_step": dec_ms,
+                      "hbm_frac": dstep_bytes / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                      "bytes_per_step": dstep_bytes}
+    step_ms = total_ms / args.steps
+    for name, kinfo in kernels.items():
+        kinfo["share"] = kinfo["ms"] / step_ms
+    dominant = max(kernels, key=lambda k: kernels[k]["ms"])
+    dk = kernels[dominant]
+    roofline = {"kernel": dominant, "bound": dk["bound"], "achieved": dk["achieved"],
+                "peak": dk["peak"], "unit": dk["unit"], "frac": dk["frac"],
+                "traffic": traffic_for(dominant), "peak_source": f"{peak_src} "
+                f"({'hbm_gbs' if dk['unit'] == 'GB/s' else tc_name})"}
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = run_e2e(args, msa, cfg, shape, inp, ws, dev, dec, dcfg if dec is not None else None,
+                  dws if dec is not None else None, world)
+
+    value = world * N / (pre_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(args, shape),
+        "prefill": {"value": value, "unit": "tokens/s", "ms_per_step": pre_ms,
+                    "dense_flops": dense_flops(N, shape.H, shape.d),
+                    "msa_flops": idx_f + pw["main_flops"],
+                    "selected_keys_per_query": pw["selected_keys"]},
+        "decode": decode_obj, "roofline": roofline, "kernels": kernels, "e2e": e2e,
+        "gpu_launches": launches, "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        os.environ.setdefault("OMP_NUM_THREADS", str(cpu_cores()))
+        hinp = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
+        rate, rows, el = oracle_prefill_rate(hinp, shape, args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s",
+                                "cores": int(os.environ["OMP_NUM_THREADS"]), "kind": "oracle",
+                                "sample": f"{rows} query rows uniform over the {shape.name} "
+                                          f"positions, {el:.1f} s of oracle time"}
+    return line
+
+
+def traffic_for(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it is current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = table.get(kernel)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "block_sparse_long_branch_b200", "csrc", ent.get("source", ""))
+    try:
+        import hashlib
+        with open(src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return ent.get("bytes_per_launch") if h == ent.get("source_sha") else None
+
+
+def run_e2e(args, msa, cfg, shape, inp, ws, dev, dec, dcfg, dws, world):
+    """Host (pinned) inputs -> device -> msa_prefill -> host output, per step."""
+    keys = ("q", "k", "v", "q_idx", "k_idx")
+    host = {k: torch.empty_like(inp[k], device="cpu").pin_memory() for k in keys}
+    for k in keys:
+        host[k].copy_(inp[k])
+    dbuf = {k: torch.empty_like(inp[k]) for k in keys}
+    out = torch.empty((shape.N, shape.H, shape.d), dtype=torch.bfloat16, device=dev)
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+    d2h = out_h.numel() * out_h.element_size()
+    steps = max(3, args.steps // 2)
+    for _ in range(2):
+        for k in keys:
+            dbuf[k].copy_(host[k], non_blocking=True)
+        msa.msa_prefill(cfg, dbuf["q"], dbuf["k"], dbuf["v"], dbuf["q_idx"], dbuf["k_idx"],
+                        out=out, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        for k in keys:
+            dbuf[k].copy_(host[k], non_blocking=True)
+        msa.msa_prefill(cfg, dbuf["q"], dbuf["k"], dbuf["v"], dbuf["q_idx"], dbuf["k_idx"],
+                        out=out, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+    b.record()
+    torch.cuda.synchronize()
+    ms = reduce_max(a.elapsed_time(b) / steps, world)
+    res = {"value": world * shape.N / (ms * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+    if dec is not None:
+        dc = synth.DECODE_CONFIG
+        # per step: the new token's q / q_idx and its k, v, k_idx cache rows in,
+        # the attention output back
+        last = (dec["cu_seqlens"][1:] - 1).to(dev)
+        hq = dec["q"].cpu().pin_memory()
+        hqi = dec["q_idx"].cpu().pin_memory()
+        hk = dec["k_cache"][last].cpu().pin_memory()
+        hv = dec["v_cache"][last].cpu().pin_memory()
+        hki = dec["k_idx_cache"][last].cpu().pin_memory()
+        dq, dqi = torch.empty_like(dec["q"]), torch.empty_like(dec["q_idx"])
+        drow_k, drow_v, drow_ki = (torch.empty_like(hk, device=dev),
+                                   torch.empty_like(hv, device=dev),
+                                   torch.empty_like(hki, device=dev))
+        dout = torch.empty((dc.B, dc.H, dc.d), dtype=torch.bfloat16, device=dev)
+        dout_h = torch.empty(dout.shape, dtype=dout.dtype).pin_memory()
+        cu_dev = dec["cu_seqlens"].to(dev)
+        dh2d = sum(x.numel() * x.element_size() for x in (hq, hqi, hk, hv, hki))
+
+        def dstep():
+            dq.copy_(hq, non_blocking=True)
+            dqi.copy_(hqi, non_blocking=True)
+            drow_k.copy_(hk, non_blocking=True)
+            drow_v.copy_(hv, non_blocking=True)
+            drow_ki.copy_(hki, non_blocking=True)
+            dec["k_cache"].index_copy_(0, last, drow_k)
+            dec["v_cache"].index_copy_(0, last, drow_v)
+            dec["k_idx_cache"].index_copy_(0, last, drow_ki)
+            msa.msa_decode(dcfg, dq, dqi, dec["k_cache"], dec["v_cache"], dec["k_idx_cache"],
+                           cu_dev, max(dc.seq_lens), out=dout, workspace=dws)
+            dout_h.copy_(dout, non_blocking=True)
+
+        for _ in range(2):
+            dstep()
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(steps):
+            dstep()
+        b.record()
+        torch.cuda.synchronize()
+        dms = reduce_max(a.elapsed_time(b) / steps, world)
+        res["decode"] = {"value": world * dc.B / (dms * 1e-3), "unit": "tokens/s",
+                         "h2d_bytes_per_step": int(dh2d),
+                         "d2h_bytes_per_step": int(dout_h.numel() * dout_h.element_size()),
+                         "ms_per_step": dms}
+    return res
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="prefill_32k", choices=sorted(synth.PREFILL_CONFIGS))
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle time for the cpu_baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=32,
+                    help="query rows per step in the reference arm")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_setup(init_group=args.impl == "ours")
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_ours(args, rank, world, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            if dist.is_available() and dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,293 @@
+"""B200 (sm_100a) MiniMax Sparse Attention hot path -- Python binding.
+
+Thin ctypes marshalling over ``libmsa_b200.so`` (C ABI in ``include/msa.h``).
+PyTorch provides device memory and the current CUDA stream; every step of the
+computation runs in the library's CUDA kernels.  There is no CPU fallback: if
+the library is missing or no CUDA device is present, the calls raise.
+
+Function names mirror the C ABI: ``msa_index_scores``, ``msa_select_topk``,
+``msa_build_block_query_lists``, ``msa_prefill``, ``msa_decode``,
+``msa_workspace_size``, ``msa_get_device_error``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "MsaConfig", "MsaError", "config", "library_path", "load_library",
+    "OP_SELECT_TOPK", "OP_BLOCK_QUERY_LISTS", "OP_PREFILL", "OP_DECODE",
+    "msa_workspace_size", "msa_prefill_min_workspace", "msa_index_scores", "msa_select_topk",
+    "msa_build_block_query_lists", "msa_prefill", "msa_decode", "msa_get_device_error",
+    "msa_status_string", "msa_last_launch_count", "msa_set_phase_events",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libmsa_b200.so")
+
+OP_SELECT_TOPK = 0
+OP_BLOCK_QUERY_LISTS = 1
+OP_PREFILL = 2
+OP_DECODE = 3
+
+STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
+                3: "MSA_ERR_WORKSPACE", 4: "MSA_ERR_CUDA", 5: "MSA_ERR_DEVICE_TIMEOUT",
+                6: "MSA_ERR_DEVICE_INDEX"}
+
+
+class MsaConfig(ctypes.Structure):
+    """Mirror of ``msa_config_t``."""
+
+    _fields_ = [("num_heads", ctypes.c_int32), ("num_groups", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("index_dim", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float)]
+
+    def __repr__(self):
+        return (f"MsaConfig(H={self.num_heads}, G={self.num_groups}, d={self.head_dim}, "
+                f"d_idx={self.index_dim}, block={self.block_size}, k={self.top_k}, "
+                f"scale={self.softmax_scale:.6g})")
+
+
+class MsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+def config(H: int, G: int, d: int, d_idx: int, top_k: int = 16, block: int = 128,
+           scale: Optional[float] = None) -> MsaConfig:
+    return MsaConfig(H, G, d, d_idx, block, top_k, 1.0 / math.sqrt(d) if scale is None else scale)
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load the in-tree library (built by ``build.py``); raise if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"libmsa_b200.so not built ({_LIB_PATH}); run "
+                           "block_sparse_long_branch_b200/build.py")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    C = ctypes.POINTER(MsaConfig)
+    lib.msa_workspace_size.argtypes = [C, ctypes.c_int, I64, I32, ctypes.POINTER(SZ)]
+    lib.msa_prefill_min_workspace.argtypes = [C, I64, ctypes.POINTER(SZ)]
+    lib.msa_index_scores.argtypes = [C, P, P, I64, I64, I64, P, P]
+    lib.msa_select_topk.argtypes = [C, P, P, I64, P, P, SZ, P]
+    lib.msa_build_block_query_lists.argtypes = [C, P, I64, P, P, P, SZ, P]
+    lib.msa_prefill.argtypes = [C, P, P, P, P, P, I64, P, P, P, SZ, P]
+    lib.msa_decode.argtypes = [C, P, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
+    lib.msa_get_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.msa_status_string.argtypes = [ctypes.c_int]
+    lib.msa_status_string.restype = ctypes.c_char_p
+    lib.msa_set_phase_events.argtypes = [P, I32]
+    lib.msa_set_phase_events.restype = ctypes.c_int
+    lib.msa_last_launch_count.argtypes = []
+    lib.msa_last_launch_count.restype = I32
+    for name in ("msa_workspace_size", "msa_prefill_min_workspace", "msa_index_scores",
+                 "msa_select_topk", "msa_build_block_query_lists", "msa_prefill", "msa_decode",
+                 "msa_get_device_error"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise MsaError(status, where)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str, shape=None) -> ctypes.c_void_p:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def msa_status_string(status: int) -> str:
+    return load_library().msa_status_string(status).decode()
+
+
+def msa_last_launch_count() -> int:
+    return int(load_library().msa_last_launch_count())
+
+
+def msa_workspace_size(cfg: MsaConfig, op: int, n_tokens: int, batch: int = 0) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load_library().msa_workspace_size(ctypes.byref(cfg), op, n_tokens, batch,
+                                             ctypes.byref(out)), "msa_workspace_size")
+    return int(out.value)
+
+
+def msa_prefill_min_workspace(cfg: MsaConfig, N: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load_library().msa_prefill_min_workspace(ctypes.byref(cfg), N, ctypes.byref(out)),
+           "msa_prefill_min_workspace")
+    return int(out.value)
+
+
+def _workspace(ws: Optional[torch.Tensor], nbytes: int, device) -> torch.Tensor:
+    if ws is None:
+        return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    if ws.dtype != torch.uint8 or not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 CUDA tensor")
+    return ws
+
+
+def msa_index_scores(cfg: MsaConfig, q_idx: torch.Tensor, k_idx: torch.Tensor,
+                     row_begin: int = 0, row_count: Optional[int] = None,
+                     scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Pooled Index Branch scores [rows, G, nb] (fp32, -inf where invisible)."""
+    lib = load_library()
+    N = q_idx.shape[0]
+    G, di = cfg.num_groups, cfg.index_dim
+    nb = (N + cfg.block_size - 1) // cfg.block_size
+    row_count = N - row_begin if row_count is None else row_count
+    if scores is None:
+        scores = torch.empty((row_count, G, nb), dtype=torch.float32, device=q_idx.device)
+    st = lib.msa_index_scores(ctypes.byref(cfg), _dev(q_idx, torch.bfloat16, "q_idx", (N, G, di)),
+                              _dev(k_idx, torch.bfloat16, "k_idx", (N, di)), N, row_begin,
+                              row_count, _dev(scores, torch.float32, "scores", (row_count, G, nb)),
+                              _stream(stream))
+    _check(st, "msa_index_scores")
+    return scores
+
+
+def msa_select_topk(cfg: MsaConfig, q_idx: torch.Tensor, k_idx: torch.Tensor,
+                    ids: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """Forced-local top-k block ids [N, G, k] (int32, ascending, -1 padded)."""
+    lib = load_library()
+    N = q_idx.shape[0]
+    G, di, k = cfg.num_groups, cfg.index_dim, cfg.top_k
+    if ids is None:
+        ids = torch.empty((N, G, k), dtype=torch.int32, device=q_idx.device)
+    ws = _workspace(workspace, msa_workspace_size(cfg, OP_SELECT_TOPK, N), q_idx.device)
+    st = lib.msa_select_topk(ctypes.byref(cfg), _dev(q_idx, torch.bfloat16, "q_idx", (N, G, di)),
+                             _dev(k_idx, torch.bfloat16, "k_idx", (N, di)), N,
+                             _dev(ids, torch.int32, "ids", (N, G, k)), _dev(ws, torch.uint8, "ws"),
+                             ws.numel(), _stream(stream))
+    _check(st, "msa_select_topk")
+    return ids
+
+
+def msa_build_block_query_lists(cfg: MsaConfig, ids: torch.Tensor,
+                                workspace: Optional[torch.Tensor] = None,
+                                stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-(group, block) query lists: (row_ptr [G*nb+1], entries [N*G*k] capacity)."""
+    lib = load_library()
+    N, G, k = ids.shape
+    nb = (N + cfg.block_size - 1) // cfg.block_size
+    row_ptr = torch.empty(G * nb + 1, dtype=torch.int32, device=ids.device)
+    entries = torch.empty(N * G * k, dtype=torch.int32, device=ids.device)
+    ws = _workspace(workspace, msa_workspace_size(cfg, OP_BLOCK_QUERY_LISTS, N), ids.device)
+    st = lib.msa_build_block_query_lists(ctypes.byref(cfg), _dev(ids, torch.int32, "ids"), N,
+                                         _dev(row_ptr, torch.int32, "row_ptr"),
+                                         _dev(entries, torch.int32, "entries"),
+                                         _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(st, "msa_build_block_query_lists")
+    return row_ptr, entries
+
+
+def msa_prefill(cfg: MsaConfig, q, k, v, q_idx, k_idx, out: Optional[torch.Tensor] = None,
+                ids_out=None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Whole MSA prefill.  ``ids_out``: None, True (allocate) or an int32 tensor.
+
+    Returns ``out`` or ``(out, ids)`` when ids are requested.
+    """
+    lib = load_library()
+    N = q.shape[0]
+    H, G, d, di, kk = cfg.num_heads, cfg.num_groups, cfg.head_dim, cfg.index_dim, cfg.top_k
+    if out is None:
+        out = torch.empty((N, H, d), dtype=torch.bfloat16, device=q.device)
+    if ids_out is True:
+        ids_out = torch.empty((N, G, kk), dtype=torch.int32, device=q.device)
+    ws = _workspace(workspace, msa_workspace_size(cfg, OP_PREFILL, N), q.device)
+    ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (N, G, kk))
+    st = lib.msa_prefill(ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (N, H, d)),
+                         _dev(k, torch.bfloat16, "k", (N, G, d)),
+                         _dev(v, torch.bfloat16, "v", (N, G, d)),
+                         _dev(q_idx, torch.bfloat16, "q_idx", (N, G, di)),
+                         _dev(k_idx, torch.bfloat16, "k_idx", (N, di)), N,
+                         _dev(out, torch.bfloat16, "out", (N, H, d)), ids_ptr,
+                         _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(st, "msa_prefill")
+    return out if ids_out is None else (out, ids_out)
+
+
+def msa_decode(cfg: MsaConfig, q, q_idx, k_cache, v_cache, k_idx_cache, cu_seqlens,
+               max_seqlen: int, out: Optional[torch.Tensor] = None, ids_out=None,
+               workspace: Optional[torch.Tensor] = None, stream=None):
+    """One decode step for B sequences (packed caches, device cu_seqlens int64)."""
+    lib = load_library()
+    B = q.shape[0]
+    H, G, d, di, kk = cfg.num_heads, cfg.num_groups, cfg.head_dim, cfg.index_dim, cfg.top_k
+    total = k_cache.shape[0]
+    if out is None:
+        out = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
+    if ids_out is True:
+        ids_out = torch.empty((B, G, kk), dtype=torch.int32, device=q.device)
+    ws = _workspace(workspace, msa_workspace_size(cfg, OP_DECODE, total, B), q.device)
+    ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (B, G, kk))
+    st = lib.msa_decode(ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (B, H, d)),
+                        _dev(q_idx, torch.bfloat16, "q_idx", (B, G, di)),
+                        _dev(k_cache, torch.bfloat16, "k_cache", (total, G, d)),
+                        _dev(v_cache, torch.bfloat16, "v_cache", (total, G, d)),
+                        _dev(k_idx_cache, torch.bfloat16, "k_idx_cache", (total, di)),
+                        _dev(cu_seqlens, torch.int64, "cu_seqlens", (B + 1,)), B, max_seqlen,
+                        _dev(out, torch.bfloat16, "out", (B, H, d)), ids_ptr,
+                        _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(st, "msa_decode")
+    return out if ids_out is None else (out, ids_out)
+
+
+_phase_keep = None
+
+
+def msa_set_phase_events(events) -> None:
+    """Record ``torch.cuda.Event`` objects at kernel phase boundaries (see msa.h);
+    ``None`` stops recording."""
+    global _phase_keep
+    lib = load_library()
+    if events is None:
+        _check(lib.msa_set_phase_events(None, 0), "msa_set_phase_events")
+        _phase_keep = None
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _phase_keep = (arr, events)
+    _check(lib.msa_set_phase_events(arr, len(events)), "msa_set_phase_events")
+
+
+def msa_get_device_error(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise, read and clear the workspace's device error word."""
+    code = ctypes.c_uint32(0)
+    st = load_library().msa_get_device_error(_dev(workspace, torch.uint8, "workspace"),
+                                             _stream(stream), ctypes.byref(code))
+    if st not in (0, 5, 6):
+        _check(st, "msa_get_device_error")
+    return int(code.value)

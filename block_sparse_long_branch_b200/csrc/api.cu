@@ -1,0 +1,463 @@
+// api.cu -- the C ABI (include/msa.h): argument validation, workspace layout,
+// and the order of launches on the caller's stream.  No device memory is
+// allocated here and the stream is never synchronised (except in
+// msa_get_device_error).
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/msa.h"
+#include "kernels.h"
+
+namespace msa {
+namespace {
+
+constexpr int kBlock = 128;
+constexpr size_t kHeader = 256;  // device error word + reserved
+constexpr int kUnitTiles = 8;    // Main Branch tiles per work unit
+
+thread_local int g_launches = 0;
+thread_local void* const* g_events = nullptr;
+thread_local int g_n_events = 0;
+
+void mark(int i, cudaStream_t s) {
+  if (g_events && i < g_n_events && g_events[i])
+    cudaEventRecord(static_cast<cudaEvent_t>(g_events[i]), s);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+msa_status_t check_cfg(const msa_config_t* c) {
+  if (!c) return MSA_ERR_INVALID_ARG;
+  if (c->num_heads <= 0 || c->num_groups <= 0 || c->head_dim <= 0 || c->index_dim <= 0 ||
+      c->top_k <= 0 || c->block_size <= 0)
+    return MSA_ERR_INVALID_ARG;
+  if (c->num_heads % c->num_groups != 0) return MSA_ERR_INVALID_ARG;
+  if (!(c->softmax_scale > 0.f) || !isfinite(c->softmax_scale)) return MSA_ERR_INVALID_ARG;
+  if (c->block_size != kBlock) return MSA_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return MSA_ERR_UNSUPPORTED;
+  if (c->index_dim != 64 && c->index_dim != 128) return MSA_ERR_UNSUPPORTED;
+  if (c->top_k > 32) return MSA_ERR_UNSUPPORTED;
+  if (!pow2(c->num_groups) || c->num_groups > 128) return MSA_ERR_UNSUPPORTED;
+  const int hg = c->num_heads / c->num_groups;
+  if (!pow2(hg) || hg > 128) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+msa_status_t check_tokens(const msa_config_t* c, int64_t n) {
+  if (n < 1) return MSA_ERR_INVALID_ARG;
+  if (n >= (int64_t(1) << 26)) return MSA_ERR_UNSUPPORTED;
+  if (n * c->num_heads >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  if (n * c->num_groups * c->top_k >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+int64_t n_blocks(int64_t n) { return (n + kBlock - 1) / kBlock; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// ---- prefill workspace for one chunk of `rows` query rows ------------------
+struct PrefillLayout {
+  size_t ids, row_ptr, entries, unit_ptr, unit_list, csr, part_o, part_lse, total;
+};
+
+PrefillLayout prefill_layout(const msa_config_t* c, int64_t rows, int64_t nb, bool own_ids) {
+  const int64_t G = c->num_groups, k = c->top_k, HG = c->num_heads / c->num_groups;
+  const int64_t slots = rows * G * k;
+  const int64_t lists = G * nb;
+  const int64_t per_unit = (int64_t)main_tile_tokens(c->num_heads, c->num_groups) * kUnitTiles;
+  const int64_t max_units = (slots + per_unit - 1) / per_unit + lists;
+  PrefillLayout L;
+  size_t off = kHeader;
+  L.ids = off;
+  off += own_ids ? align256(slots * 4) : 0;
+  L.row_ptr = off;
+  off += align256((lists + 1) * 4);
+  L.entries = off;
+  off += align256(slots * 4);
+  L.unit_ptr = off;
+  off += align256((lists + 1) * 4);
+  L.unit_list = off;
+  off += align256(max_units * 4);
+  L.csr = off;
+  off += csr_scratch_bytes(rows, (int32_t)G, (int32_t)k, nb);
+  L.part_o = off;
+  off += align256(slots * HG * c->head_dim * 2);
+  L.part_lse = off;
+  off += align256(slots * HG * 4);
+  L.total = off;
+  return L;
+}
+
+// decode workspace: header | ids | part_o | part_lse | pooled scores (the rest)
+size_t decode_fixed_bytes(const msa_config_t* c, int32_t B, size_t* off_ids, size_t* off_o,
+                          size_t* off_lse) {
+  const int64_t G = c->num_groups, k = c->top_k, HG = c->num_heads / c->num_groups;
+  size_t off = kHeader;
+  *off_ids = off;
+  off += align256((size_t)B * G * k * 4);
+  *off_o = off;
+  off += align256((size_t)B * G * k * HG * c->head_dim * 2);
+  *off_lse = off;
+  off += align256((size_t)B * G * k * HG * 4);
+  return off;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+
+}  // namespace
+}  // namespace msa
+
+using namespace msa;
+
+extern "C" {
+
+const char* msa_status_string(msa_status_t s) {
+  switch (s) {
+    case MSA_OK: return "ok";
+    case MSA_ERR_INVALID_ARG: return "invalid argument";
+    case MSA_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+    case MSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MSA_ERR_CUDA: return "CUDA runtime or launch error";
+    case MSA_ERR_DEVICE_TIMEOUT: return "a device-side wait ran out";
+    case MSA_ERR_DEVICE_INDEX: return "a device-side index was out of range";
+  }
+  return "unknown status";
+}
+
+int32_t msa_last_launch_count(void) { return g_launches; }
+
+msa_status_t msa_set_phase_events(void* const* events, int32_t count) {
+  if (events && count < 0) return MSA_ERR_INVALID_ARG;
+  g_events = events;
+  g_n_events = events ? count : 0;
+  return MSA_OK;
+}
+
+msa_status_t msa_workspace_size(const msa_config_t* cfg, msa_op_t op, int64_t n_tokens,
+                                int32_t batch, size_t* bytes) {
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if (!bytes) return MSA_ERR_INVALID_ARG;
+  if ((st = check_tokens(cfg, n_tokens)) != MSA_OK) return st;
+  const int64_t nb = n_blocks(n_tokens);
+  switch (op) {
+    case MSA_OP_SELECT_TOPK:
+      *bytes = kHeader;
+      return MSA_OK;
+    case MSA_OP_BLOCK_QUERY_LISTS:
+      *bytes = kHeader + csr_scratch_bytes(n_tokens, cfg->num_groups, cfg->top_k, nb);
+      return MSA_OK;
+    case MSA_OP_PREFILL:
+      *bytes = prefill_layout(cfg, n_tokens, nb, true).total;
+      return MSA_OK;
+    case MSA_OP_DECODE: {
+      if (batch < 1 || batch > n_tokens) return MSA_ERR_INVALID_ARG;
+      size_t a, b, c;
+      *bytes = decode_fixed_bytes(cfg, batch, &a, &b, &c) +
+               decode_pooled_rows(n_tokens, batch) * cfg->num_groups * sizeof(float);
+      return MSA_OK;
+    }
+  }
+  return MSA_ERR_INVALID_ARG;
+}
+
+msa_status_t msa_prefill_min_workspace(const msa_config_t* cfg, int64_t N, size_t* bytes) {
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if (!bytes) return MSA_ERR_INVALID_ARG;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  const int64_t rows = N < kBlock ? N : kBlock;
+  *bytes = prefill_layout(cfg, rows, n_blocks(N), true).total;
+  return MSA_OK;
+}
+
+msa_status_t msa_index_scores(const msa_config_t* cfg, const void* q_idx, const void* k_idx,
+                              int64_t N, int64_t row_begin, int64_t row_count, float* scores,
+                              msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  if (!q_idx || !k_idx || !scores) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(scores)) return MSA_ERR_INVALID_ARG;
+  if (row_begin < 0 || row_count < 1 || row_begin + row_count > N) return MSA_ERR_INVALID_ARG;
+  IndexLaunch p{};
+  p.q_idx = q_idx;
+  p.k_idx = k_idx;
+  p.N = N;
+  p.G = cfg->num_groups;
+  p.d_idx = cfg->index_dim;
+  p.top_k = cfg->top_k;
+  p.row_begin = row_begin;
+  p.row_end = row_begin + row_count;
+  p.scores = scores;
+  p.err = nullptr;
+  p.num_sms = sm_count();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = cuda_status(launch_index_scores(p, s));
+  g_launches = 1;
+  return st;
+}
+
+msa_status_t msa_select_topk(const msa_config_t* cfg, const void* q_idx, const void* k_idx,
+                             int64_t N, int32_t* ids, void* ws, size_t ws_bytes,
+                             msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  if (!q_idx || !k_idx || !ids) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(ids)) return MSA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < kHeader || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  IndexLaunch p{};
+  p.q_idx = q_idx;
+  p.k_idx = k_idx;
+  p.N = N;
+  p.G = cfg->num_groups;
+  p.d_idx = cfg->index_dim;
+  p.top_k = cfg->top_k;
+  p.row_begin = 0;
+  p.row_end = N;
+  p.ids = ids;
+  p.err = at<uint32_t>(ws, 0);
+  p.num_sms = sm_count();
+  st = cuda_status(launch_index_select(p, s));
+  g_launches = 1;
+  return st;
+}
+
+msa_status_t msa_build_block_query_lists(const msa_config_t* cfg, const int32_t* ids, int64_t N,
+                                         int32_t* row_ptr, int32_t* entries, void* ws,
+                                         size_t ws_bytes, msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  if (!ids || !row_ptr || !entries) return MSA_ERR_INVALID_ARG;
+  const int64_t nb = n_blocks(N);
+  const size_t need = kHeader + csr_scratch_bytes(N, cfg->num_groups, cfg->top_k, nb);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  CsrLaunch p{};
+  p.ids = ids;
+  p.row_begin = 0;
+  p.rows = N;
+  p.G = cfg->num_groups;
+  p.top_k = cfg->top_k;
+  p.nb = nb;
+  p.row_ptr = row_ptr;
+  p.entries = entries;
+  p.scratch = at<void>(ws, kHeader);
+  p.err = at<uint32_t>(ws, 0);
+  p.unit_ptr = nullptr;
+  p.unit_list = nullptr;
+  int launches = 0;
+  st = cuda_status(launch_csr(p, s, &launches));
+  g_launches = launches;
+  return st;
+}
+
+msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, const void* v,
+                         const void* q_idx, const void* k_idx, int64_t N, void* out,
+                         int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  if (!q || !k || !v || !q_idx || !k_idx || !out) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_idx) || !aligned16(k_idx) ||
+      !aligned16(out) || (ids_out && !aligned16(ids_out)))
+    return MSA_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  const int64_t nb = n_blocks(N);
+  const bool own_ids = ids_out == nullptr;
+  // largest chunk (a multiple of 128 query rows, or all of N) that fits
+  int64_t chunk = N;
+  if (prefill_layout(cfg, chunk, nb, own_ids).total > ws_bytes) {
+    int64_t lo = 1, hi = nb;  // in blocks
+    if (prefill_layout(cfg, kBlock, nb, own_ids).total > ws_bytes) return MSA_ERR_WORKSPACE;
+    while (lo < hi) {
+      const int64_t mid = (lo + hi + 1) / 2;
+      if (prefill_layout(cfg, mid * kBlock, nb, own_ids).total <= ws_bytes)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    chunk = lo * kBlock;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  const int G = cfg->num_groups, H = cfg->num_heads, d = cfg->head_dim, kk = cfg->top_k;
+  const int sms = sm_count();
+  uint32_t* err = at<uint32_t>(ws, 0);
+  int launches = 0;
+  for (int64_t t0 = 0, c = 0; t0 < N; t0 += chunk, ++c) {
+    const int64_t t1 = t0 + chunk < N ? t0 + chunk : N;
+    const int ev = (int)(5 * c);
+    mark(ev, s);
+    const int64_t rows = t1 - t0;
+    const int64_t nbc = n_blocks(t1);
+    const PrefillLayout L = prefill_layout(cfg, rows, nbc, own_ids);
+    int32_t* ids = own_ids ? at<int32_t>(ws, L.ids) : ids_out + t0 * G * kk;
+
+    IndexLaunch ip{};
+    ip.q_idx = q_idx;
+    ip.k_idx = k_idx;
+    ip.N = N;
+    ip.G = G;
+    ip.d_idx = cfg->index_dim;
+    ip.top_k = kk;
+    ip.row_begin = t0;
+    ip.row_end = t1;
+    ip.ids = ids;
+    ip.err = err;
+    ip.num_sms = sms;
+    if (launch_index_select(ip, s) != cudaSuccess) return MSA_ERR_CUDA;
+    ++launches;
+    mark(ev + 1, s);
+
+    CsrLaunch cp{};
+    cp.ids = ids;
+    cp.row_begin = t0;
+    cp.rows = rows;
+    cp.G = G;
+    cp.top_k = kk;
+    cp.nb = nbc;
+    cp.row_ptr = at<int32_t>(ws, L.row_ptr);
+    cp.entries = at<int32_t>(ws, L.entries);
+    cp.scratch = at<void>(ws, L.csr);
+    cp.err = err;
+    cp.unit_ptr = at<int32_t>(ws, L.unit_ptr);
+    cp.unit_list = at<int32_t>(ws, L.unit_list);
+    cp.tile_tokens = main_tile_tokens(H, G);
+    cp.unit_tiles = kUnitTiles;
+    if (launch_csr(cp, s, &launches) != cudaSuccess) return MSA_ERR_CUDA;
+    mark(ev + 2, s);
+
+    MainLaunch mp{};
+    mp.q = q;
+    mp.k = k;
+    mp.v = v;
+    mp.N = N;
+    mp.H = H;
+    mp.G = G;
+    mp.d = d;
+    mp.top_k = kk;
+    mp.scale = cfg->softmax_scale;
+    mp.row_begin = t0;
+    mp.rows = rows;
+    mp.nb = nbc;
+    mp.row_ptr = cp.row_ptr;
+    mp.entries = cp.entries;
+    mp.unit_ptr = cp.unit_ptr;
+    mp.unit_list = cp.unit_list;
+    mp.unit_tiles = kUnitTiles;
+    mp.part_o = at<__half>(ws, L.part_o);
+    mp.part_lse = at<float>(ws, L.part_lse);
+    mp.err = err;
+    mp.grid = sms;
+    if (launch_main(mp, s) != cudaSuccess) return MSA_ERR_CUDA;
+    ++launches;
+    mark(ev + 3, s);
+
+    MergeLaunch gp{};
+    gp.part_o = mp.part_o;
+    gp.part_lse = mp.part_lse;
+    gp.ids = ids;
+    gp.rows = rows;
+    gp.H = H;
+    gp.G = G;
+    gp.d = d;
+    gp.top_k = kk;
+    gp.out = static_cast<uint8_t*>(out) + (size_t)t0 * H * d * 2;
+    if (launch_merge(gp, s) != cudaSuccess) return MSA_ERR_CUDA;
+    ++launches;
+    mark(ev + 4, s);
+  }
+  g_launches = launches;
+  return MSA_OK;
+}
+
+msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_idx,
+                        const void* k_cache, const void* v_cache, const void* k_idx_cache,
+                        const int64_t* cu_seqlens, int32_t B, int64_t max_seqlen, void* out,
+                        int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if (!q || !q_idx || !k_cache || !v_cache || !k_idx_cache || !cu_seqlens || !out)
+    return MSA_ERR_INVALID_ARG;
+  if (B < 1 || max_seqlen < 1) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(q_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(k_idx_cache) || !aligned16(out) || (ids_out && !aligned16(ids_out)))
+    return MSA_ERR_INVALID_ARG;
+  if ((st = check_tokens(cfg, max_seqlen)) != MSA_OK) return st;
+  if (!ws || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  size_t off_ids, off_o, off_lse;
+  const size_t fixed = decode_fixed_bytes(cfg, B, &off_ids, &off_o, &off_lse);
+  const size_t row_bytes = (size_t)cfg->num_groups * sizeof(float);
+  if (ws_bytes < fixed + row_bytes * (size_t)(B + 1)) return MSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  DecodeLaunch p{};
+  p.q = q;
+  p.q_idx = q_idx;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.k_idx_cache = k_idx_cache;
+  p.cu_seqlens = cu_seqlens;
+  p.B = B;
+  p.H = cfg->num_heads;
+  p.G = cfg->num_groups;
+  p.d = cfg->head_dim;
+  p.d_idx = cfg->index_dim;
+  p.top_k = cfg->top_k;
+  p.max_seqlen = max_seqlen;
+  p.scale = cfg->softmax_scale;
+  p.out = out;
+  p.ids = ids_out ? ids_out : at<int32_t>(ws, off_ids);
+  p.part_o = at<__half>(ws, off_o);
+  p.part_lse = at<float>(ws, off_lse);
+  p.pooled = at<float>(ws, fixed);
+  p.pooled_cap = (int64_t)((ws_bytes - fixed) / row_bytes);
+  p.err = at<uint32_t>(ws, 0);
+  p.num_sms = sm_count();
+  p.events = g_events;
+  p.n_events = g_n_events;
+  int launches = 0;
+  st = cuda_status(launch_decode(p, s, &launches));
+  g_launches = launches;
+  return st;
+}
+
+msa_status_t msa_get_device_error(void* ws, msa_stream_t stream, uint32_t* code) {
+  if (!ws || !code) return MSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MSA_ERR_CUDA;
+  uint32_t c = 0;
+  if (cudaMemcpy(&c, ws, sizeof c, cudaMemcpyDeviceToHost) != cudaSuccess) return MSA_ERR_CUDA;
+  if (cudaMemset(ws, 0, sizeof c) != cudaSuccess) return MSA_ERR_CUDA;
+  *code = c;
+  if (c == 0) return MSA_OK;
+  if ((c & 0xF00u) == 0x100u) return MSA_ERR_DEVICE_TIMEOUT;
+  return MSA_ERR_DEVICE_INDEX;
+}
+
+}  // extern "C"

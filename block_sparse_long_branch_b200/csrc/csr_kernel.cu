@@ -1,0 +1,267 @@
+// csr_kernel.cu -- inversion of the block selection into per-(group, key block)
+// query lists: the schedule of the KV-block-outer Main Branch (tnkblog MiniMax
+// M3 / MSA post, section "MSA の実装": key blocks are the outer loop and the
+// queries that hit a block are gathered; CSDN M3 write-up, section "MiniMax
+// Sparse Attention（MSA）").
+//
+// Deterministic stable counting sort on the key (g, j), in t order:
+//   1. hist    : per tile of kTileTok query rows and per group, a shared-memory
+//                histogram over the key blocks -> cnt[(g*nb + j)*ntiles + tile]
+//   2. scan    : exclusive prefix over that table (flattened g, j, tile), so
+//                the entry gives where tile `tile`'s hits on (g, j) start
+//   3. row_ptr : row_ptr[g*nb+j] = scanned[(g*nb+j)*ntiles]
+//   4. scatter : one warp per (tile, group) walks its hits in (t, slot) order;
+//                equal keys inside a 32-hit batch are ranked with match.any,
+//                a shared-memory running count carries the rank across batches
+//   5. units   : per list, number of Main Branch work units; exclusive prefix
+// HBM-bound integer work: each id is read twice, each entry written once.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kTileTok = 256;      // query rows per histogram tile
+constexpr int kBinSlice = 16384;   // shared-memory bins per pass (64 KiB)
+constexpr int kScanThreads = 1024;
+constexpr int kScanPer = 4;
+constexpr int kScanChunk = kScanThreads * kScanPer;
+
+__global__ void __launch_bounds__(256) csr_hist_kernel(const int32_t* __restrict__ ids, int64_t rows,
+                                                       int32_t G, int32_t top_k, int64_t nb,
+                                                       int32_t ntiles, int32_t* __restrict__ cnt,
+                                                       uint32_t* err) {
+  extern __shared__ int32_t bins[];
+  const int tile = blockIdx.x, g = blockIdx.y;
+  const int64_t r0 = (int64_t)tile * kTileTok;
+  const int64_t r1 = min(rows, r0 + kTileTok);
+  const int64_t n_el = (r1 - r0) * top_k;
+  for (int64_t s0 = 0; s0 < nb; s0 += kBinSlice) {
+    const int width = (int)min64(kBinSlice, nb - s0);
+    for (int i = threadIdx.x; i < width; i += blockDim.x) bins[i] = 0;
+    __syncthreads();
+    for (int64_t e = threadIdx.x; e < n_el; e += blockDim.x) {
+      const int64_t row = r0 + e / top_k;
+      const int r = (int)(e % top_k);
+      const int32_t j = ids[(row * G + g) * top_k + r];
+      if (j < -1 || j >= nb) {
+        if (s0 == 0) record_error(err, kDevBadIndex);
+        continue;
+      }
+      if (j >= s0 && j < s0 + width) atomicAdd(&bins[j - s0], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < width; i += blockDim.x)
+      cnt[((int64_t)g * nb + s0 + i) * ntiles + tile] = bins[i];
+    __syncthreads();
+  }
+}
+
+// ---- exclusive scan (int32), chunk of 4096 per CTA --------------------------
+__device__ __forceinline__ int32_t warp_incl_scan(int32_t x) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if ((threadIdx.x & 31) >= o) x += y;
+  }
+  return x;
+}
+
+__global__ void __launch_bounds__(kScanThreads) scan_chunks_kernel(int32_t* __restrict__ data,
+                                                                   int64_t n,
+                                                                   int32_t* __restrict__ sums) {
+  __shared__ int32_t warp_tot[32];
+  const int64_t base = (int64_t)blockIdx.x * kScanChunk + (int64_t)threadIdx.x * kScanPer;
+  int32_t v[kScanPer];
+  int32_t local = 0;
+#pragma unroll
+  for (int i = 0; i < kScanPer; ++i) {
+    v[i] = (base + i < n) ? data[base + i] : 0;
+    local += v[i];
+  }
+  const int32_t incl = warp_incl_scan(local);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int32_t t = warp_tot[l];
+    const int32_t ti = warp_incl_scan(t);
+    warp_tot[l] = ti - t;
+    if (l == 31 && sums) sums[blockIdx.x] = ti;
+  }
+  __syncthreads();
+  int32_t run = warp_tot[w] + incl - local;
+#pragma unroll
+  for (int i = 0; i < kScanPer; ++i) {
+    if (base + i < n) data[base + i] = run;
+    run += v[i];
+  }
+}
+
+__global__ void add_offsets_kernel(int32_t* __restrict__ data, int64_t n,
+                                   const int32_t* __restrict__ offs) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) data[i] += offs[i / kScanChunk];
+}
+
+// total = last exclusive value + last count (read before the scan)
+__global__ void store_total_kernel(const int32_t* scanned, const int32_t* last_count, int64_t n,
+                                   int32_t* total) {
+  *total = scanned[n - 1] + *last_count;
+}
+
+size_t scan_scratch_elems(int64_t n) {
+  size_t s = 0;
+  while (n > kScanChunk) {
+    n = (n + kScanChunk - 1) / kScanChunk;
+    s += (size_t)n;
+  }
+  return s + 1;
+}
+
+// In-place exclusive scan of data[0..n); `tmp` holds scan_scratch_elems(n).
+cudaError_t exclusive_scan(int32_t* data, int64_t n, int32_t* tmp, cudaStream_t s, int* launches) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t nch = (n + kScanChunk - 1) / kScanChunk;
+  scan_chunks_kernel<<<(unsigned)nch, kScanThreads, 0, s>>>(data, n, nch > 1 ? tmp : nullptr);
+  ++*launches;
+  if (nch > 1) {
+    cudaError_t e = exclusive_scan(tmp, nch, tmp + nch, s, launches);
+    if (e != cudaSuccess) return e;
+    add_offsets_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(data, n, tmp);
+    ++*launches;
+  }
+  return cudaGetLastError();
+}
+
+__global__ void csr_rowptr_kernel(const int32_t* __restrict__ scanned, int64_t n_lists,
+                                  int32_t ntiles, const int32_t* __restrict__ total,
+                                  int32_t* __restrict__ row_ptr) {
+  const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x < n_lists) row_ptr[x] = scanned[x * ntiles];
+  if (x == n_lists) row_ptr[x] = *total;
+}
+
+__global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restrict__ ids,
+                                                         int64_t row_begin, int64_t rows,
+                                                         int32_t G, int32_t top_k, int64_t nb,
+                                                         int32_t ntiles,
+                                                         const int32_t* __restrict__ scanned,
+                                                         int32_t* __restrict__ entries) {
+  extern __shared__ int32_t run[];
+  const int tile = blockIdx.x, g = blockIdx.y;
+  const int lane = threadIdx.x;
+  const int64_t r0 = (int64_t)tile * kTileTok;
+  const int64_t r1 = min(rows, r0 + kTileTok);
+  const int64_t n_el = (r1 - r0) * top_k;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int64_t s0 = 0; s0 < nb; s0 += kBinSlice) {
+    const int width = (int)min64(kBinSlice, nb - s0);
+    for (int i = lane; i < width; i += 32) run[i] = 0;
+    __syncwarp();
+    for (int64_t e0 = 0; e0 < n_el; e0 += 32) {
+      const int64_t e = e0 + lane;
+      int32_t j = -1;
+      int64_t row = 0;
+      int r = 0;
+      if (e < n_el) {
+        row = r0 + e / top_k;
+        r = (int)(e % top_k);
+        j = ids[(row * G + g) * top_k + r];
+      }
+      const bool mine = j >= s0 && j < s0 + width;
+      const int key = mine ? (int)(j - s0) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, key);
+      int32_t base = 0;
+      if (mine) {
+        base = run[key];
+        const int rank = __popc(peers & lt_mask);
+        const int64_t pos = (int64_t)scanned[((int64_t)g * nb + j) * ntiles + tile] + base + rank;
+        entries[pos] = (int32_t)(((row_begin + row) << 5) | r);
+      }
+      __syncwarp();
+      if (mine && (peers & lt_mask) == 0) run[key] = base + __popc(peers);
+      __syncwarp();
+    }
+  }
+}
+
+__global__ void unit_fill_kernel(const int32_t* __restrict__ unit_ptr, int64_t n_lists,
+                                 int32_t* __restrict__ unit_list) {
+  const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x < n_lists)
+    for (int32_t u = unit_ptr[x]; u < unit_ptr[x + 1]; ++u) unit_list[u] = (int32_t)x;
+}
+
+__global__ void unit_count_kernel(const int32_t* __restrict__ row_ptr, int64_t n_lists,
+                                  int32_t per_unit, int32_t* __restrict__ units) {
+  const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x < n_lists) {
+    const int32_t len = row_ptr[x + 1] - row_ptr[x];
+    units[x] = (len + per_unit - 1) / per_unit;
+  }
+}
+
+}  // namespace
+
+size_t csr_scratch_bytes(int64_t rows, int32_t G, int32_t top_k, int64_t nb) {
+  (void)top_k;
+  const int64_t ntiles = (rows + kTileTok - 1) / kTileTok;
+  const int64_t table = (int64_t)G * nb * ntiles;
+  const int64_t lists = (int64_t)G * nb + 1;
+  size_t elems = (size_t)table + scan_scratch_elems(table) + 2 + scan_scratch_elems(lists) + 2;
+  return (elems * sizeof(int32_t) + 255) & ~(size_t)255;
+}
+
+cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
+  const int64_t ntiles = (p.rows + kTileTok - 1) / kTileTok;
+  const int64_t n_lists = (int64_t)p.G * p.nb;
+  const int64_t table = n_lists * ntiles;
+  int32_t* cnt = static_cast<int32_t*>(p.scratch);
+  int32_t* scan_tmp = cnt + table;
+  int32_t* total = scan_tmp + scan_scratch_elems(table);
+  int32_t* last = total + 1;
+  int32_t* tmp2 = last + 1;
+  const int bins = (int)(p.nb < kBinSlice ? p.nb : kBinSlice);
+  cudaError_t e;
+
+  dim3 grid((unsigned)ntiles, (unsigned)p.G);
+  const size_t bin_bytes = (size_t)bins * sizeof(int32_t);
+  if (bin_bytes > 48 * 1024) {
+    if ((e = cudaFuncSetAttribute(csr_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)bin_bytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(csr_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)bin_bytes)) != cudaSuccess)
+      return e;
+  }
+  csr_hist_kernel<<<grid, 256, bins * sizeof(int32_t), s>>>(p.ids, p.rows, p.G, p.top_k, p.nb,
+                                                           (int32_t)ntiles, cnt, p.err);
+  ++*launches;
+  if ((e = cudaMemcpyAsync(last, cnt + table - 1, sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) !=
+      cudaSuccess)
+    return e;
+  if ((e = exclusive_scan(cnt, table, scan_tmp, s, launches)) != cudaSuccess) return e;
+  store_total_kernel<<<1, 1, 0, s>>>(cnt, last, table, total);
+  ++*launches;
+  csr_rowptr_kernel<<<(unsigned)((n_lists + 1 + 255) / 256), 256, 0, s>>>(
+      cnt, n_lists, (int32_t)ntiles, total, p.row_ptr);
+  ++*launches;
+  csr_scatter_kernel<<<grid, 32, bins * sizeof(int32_t), s>>>(p.ids, p.row_begin, p.rows, p.G,
+                                                             p.top_k, p.nb, (int32_t)ntiles, cnt,
+                                                             p.entries);
+  ++*launches;
+  if (p.unit_ptr) {
+    unit_count_kernel<<<(unsigned)((n_lists + 255) / 256), 256, 0, s>>>(
+        p.row_ptr, n_lists, p.tile_tokens * p.unit_tiles, p.unit_ptr);
+    ++*launches;
+    // unit_ptr[n_lists] = total units: scan n_lists+1 values with a trailing 0
+    if ((e = cudaMemsetAsync(p.unit_ptr + n_lists, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
+    if ((e = exclusive_scan(p.unit_ptr, n_lists + 1, tmp2, s, launches)) != cudaSuccess) return e;
+    unit_fill_kernel<<<(unsigned)((n_lists + 255) / 256), 256, 0, s>>>(p.unit_ptr, n_lists,
+                                                                      p.unit_list);
+    ++*launches;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace msa

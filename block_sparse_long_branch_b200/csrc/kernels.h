@@ -1,0 +1,106 @@
+// kernels.h -- launchers shared between the kernel translation units and the
+// C-ABI layer.  Host-side declarations only.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace msa {
+
+// ---- Index Branch (index_kernel.cu) ---------------------------------------
+struct IndexLaunch {
+  const void* q_idx;  // [N][G][d_idx] bf16
+  const void* k_idx;  // [N][d_idx] bf16
+  int64_t N;
+  int32_t G, d_idx, top_k;
+  int64_t row_begin, row_end;  // query rows processed: [row_begin, row_end)
+  int32_t* ids;                // selection mode: [row_end-row_begin][G][top_k]
+  float* scores;               // scores mode: [row_end-row_begin][G][nb]
+  uint32_t* err;
+  int num_sms;
+};
+cudaError_t launch_index_select(const IndexLaunch& p, cudaStream_t s);
+cudaError_t launch_index_scores(const IndexLaunch& p, cudaStream_t s);
+
+// ---- query-list inversion (csr_kernel.cu) ---------------------------------
+struct CsrLaunch {
+  const int32_t* ids;  // [rows][G][top_k], query t = row_begin + row
+  int64_t row_begin, rows;
+  int32_t G, top_k;
+  int64_t nb;          // key blocks (lists per group)
+  int32_t* row_ptr;    // [G*nb+1]
+  int32_t* entries;    // [rows*G*top_k]
+  void* scratch;       // csr_scratch_bytes()
+  uint32_t* err;
+  // optional: main-branch work units (tiles of `tile_tokens` queries, at most
+  // `unit_tiles` tiles per unit) per list, exclusive prefix in unit_ptr[G*nb+1]
+  int32_t* unit_ptr;
+  int32_t* unit_list;  // [max units]: list index of every unit
+  int32_t tile_tokens, unit_tiles;
+};
+size_t csr_scratch_bytes(int64_t rows, int32_t G, int32_t top_k, int64_t nb);
+cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches);
+
+// ---- Main Branch (main_kernel.cu) -----------------------------------------
+struct MainLaunch {
+  const void* q;  // [N][H][d] bf16
+  const void* k;  // [N][G][d] bf16
+  const void* v;  // [N][G][d] bf16
+  int64_t N;
+  int32_t H, G, d, top_k;
+  float scale;
+  int64_t row_begin, rows;  // query rows covered by the lists
+  int64_t nb;
+  const int32_t* row_ptr;   // [G*nb+1]
+  const int32_t* entries;
+  const int32_t* unit_ptr;   // [G*nb+1]
+  const int32_t* unit_list;  // [units]
+  int32_t unit_tiles;
+  __half* part_o;   // [rows][G][top_k][H/G][d] fp16
+  float* part_lse;  // [rows][G][top_k][H/G] fp32
+  uint32_t* err;
+  int grid;
+};
+// query tokens per 128-row Main Branch tile
+int main_tile_tokens(int H, int G);
+cudaError_t launch_main(const MainLaunch& p, cudaStream_t s);
+
+// ---- merge (merge_kernel.cu) ----------------------------------------------
+struct MergeLaunch {
+  const __half* part_o;
+  const float* part_lse;
+  const int32_t* ids;  // [rows][G][top_k]
+  int64_t rows;
+  int32_t H, G, d, top_k;
+  void* out;  // [rows][H][d] bf16 (already offset to row_begin)
+};
+cudaError_t launch_merge(const MergeLaunch& p, cudaStream_t s);
+
+// ---- decode (decode_kernel.cu) --------------------------------------------
+struct DecodeLaunch {
+  const void* q;            // [B][H][d]
+  const void* q_idx;        // [B][G][d_idx]
+  const void* k_cache;      // [sumL][G][d]
+  const void* v_cache;      // [sumL][G][d]
+  const void* k_idx_cache;  // [sumL][d_idx]
+  const int64_t* cu_seqlens;
+  int32_t B, H, G, d, d_idx, top_k;
+  int64_t max_seqlen;
+  float scale;
+  void* out;       // [B][H][d] bf16
+  int32_t* ids;    // [B][G][top_k]
+  float* pooled;   // [pooled_cap][G]
+  int64_t pooled_cap;
+  __half* part_o;  // [B][G][top_k][H/G][d]
+  float* part_lse; // [B][G][top_k][H/G]
+  uint32_t* err;
+  int num_sms;
+  void* const* events;  // optional phase events (msa_set_phase_events)
+  int n_events;
+};
+size_t decode_pooled_rows(int64_t total_len, int32_t B);
+cudaError_t launch_decode(const DecodeLaunch& p, cudaStream_t s, int* launches);
+
+}  // namespace msa

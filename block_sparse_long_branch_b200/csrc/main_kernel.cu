@@ -1,0 +1,530 @@
+// main_kernel.cu -- Main Branch prefill, key-block outer loop, gathered queries.
+//
+// Exact softmax attention over the selected blocks only (ai-tool-zukan "MiniMax
+// MSA guide", section "Index BranchとMain Branchの役割分担"), computed with the
+// key/value block as the outer loop: each work unit is one (group g, key block
+// j) and a run of the queries that selected it; K_j and V_j are loaded once per
+// unit and the hitting queries' heads are gathered into 128-row tiles
+// (tnkblog MiniMax M3 / MSA post, section "MSA の実装"; CSDN M3 write-up,
+// section "MiniMax Sparse Attention（MSA）": KV outer, gather Q, each KV block
+// read once).
+//
+// Per tile (128 rows = TT tokens x the H/G heads of group g):
+//   S = Q_tile K_j^T            tcgen05.mma M=128 N=128 K=d   (TMEM, fp32)
+//   P = exp(scale*(S - rowmax)) softmax warps, causal mask on the local block
+//   O = P V_j                   tcgen05.mma M=128 N=d  K=128  (V is MN-major)
+// and the row's partial (o = O / rowsum in fp16, lse = scale*rowmax +
+// ln rowsum) goes to slot (t, g, r, head); the merge kernel combines the <= k
+// slots of a query with log-sum-exp weights.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over units):
+//   warp 0     producer: TMA of K_j / V_j (3-D map: one group's rows), and a
+//              TMA gather of each hitting token's H/G contiguous query rows;
+//   warp 1     MMA issuer (one thread), S of tile i+1 issued before P V of
+//              tile i so the tensor core never waits on the softmax;
+//   warps 2-5  softmax + epilogue, thread <-> TMEM lane <-> tile row; the
+//              epilogue of tile i runs after the softmax of tile i+1.
+// TMEM: two S buffers (2 x 128 columns) and two O buffers (2 x 128 columns).
+#include "kernels.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace msa {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kRows = 128;
+constexpr int kKeys = 128;
+constexpr int kQStages = 3;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct MainCfg {
+  static constexpr int kRegions = D / 64;
+  static constexpr int kQBytes = kRows * D * 2;
+  static constexpr int kKVBytes = kKeys * D * 2;
+  static constexpr int kPBytes = kRows * kKeys * 2;
+  static constexpr int kOffK = kQStages * kQBytes;
+  static constexpr int kOffV = kOffK + kKVBytes;
+  static constexpr int kOffP = kOffV + kKVBytes;
+  static constexpr int kSmem = kOffP + 2 * kPBytes + 1024;
+};
+
+struct MainArgs {
+  int64_t N, row_begin, rows;
+  int32_t H, G, HG, log2slot, TT, top_k;
+  float scale, scale_log2;
+  int64_t nb;
+  const int32_t* row_ptr;
+  const int32_t* entries;
+  const int32_t* unit_ptr;
+  const int32_t* unit_list;
+  int32_t per_unit;
+  __half* part_o;
+  float* part_lse;
+  uint32_t* err;
+};
+
+struct MUnit {
+  int32_t g, j, e0, e1, ntiles;
+};
+
+__device__ __forceinline__ MUnit decode_unit(const MainArgs& a, int u) {
+  MUnit m;
+  const int x = __ldg(a.unit_list + u);
+  const int c = u - __ldg(a.unit_ptr + x);
+  m.g = (int)(x / a.nb);
+  m.j = (int)(x - (int64_t)m.g * a.nb);
+  const int beg = __ldg(a.row_ptr + x), end = __ldg(a.row_ptr + x + 1);
+  m.e0 = beg + c * a.per_unit;
+  m.e1 = min(end, m.e0 + a.per_unit);
+  m.ntiles = (m.e1 - m.e0 + a.TT - 1) / a.TT;
+  return m;
+}
+
+// decoded list entry, validated against the lists' query range
+__device__ __forceinline__ bool read_entry(const MainArgs& a, int e, int64_t& t, int& r) {
+  const int32_t ent = __ldg(a.entries + e);
+  t = (int64_t)(ent >> 5);
+  r = ent & 31;
+  const bool ok = ent >= 0 && t >= a.row_begin && t < a.row_begin + a.rows && t < a.N &&
+                  r < a.top_k;
+  if (!ok) {
+    record_error(a.err, kDevBadIndex);
+    t = a.row_begin;
+    r = 0;
+  }
+  return ok;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    main_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                const __grid_constant__ CUtensorMap map_v, const MainArgs a) {
+  using Cfg = MainCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + Cfg::kOffK;
+  uint8_t* sV = smem + Cfg::kOffV;
+  uint8_t* sP = smem + Cfg::kOffP;
+
+  __shared__ uint64_t bar_q_full[kQStages], bar_q_empty[kQStages];
+  __shared__ uint64_t bar_k_full, bar_k_empty, bar_v_full, bar_v_empty;
+  __shared__ uint64_t bar_s_full[2], bar_s_empty[2];
+  __shared__ uint64_t bar_p_full[2], bar_p_empty[2];
+  __shared__ uint64_t bar_o_full[2], bar_o_empty[2];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+
+  const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&bar_q_full[s], 1);
+      mbar_init(&bar_q_empty[s], 1);
+    }
+    mbar_init(&bar_k_full, 1);
+    mbar_init(&bar_k_empty, 1);
+    mbar_init(&bar_v_full, 1);
+    mbar_init(&bar_v_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_s_full[i], 1);
+      mbar_init(&bar_s_empty[i], 128);
+      mbar_init(&bar_p_full[i], 128);
+      mbar_init(&bar_p_empty[i], 1);
+      mbar_init(&bar_o_full[i], 1);
+      mbar_init(&bar_o_empty[i], 128);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_s, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* abort_flag = &abort_s;
+  const int n_units = __ldg(a.unit_ptr + a.G * a.nb);
+  const int slot = 1 << a.log2slot;
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+    }
+    int qs = 0;
+    uint32_t qph = 0, kph = 0, vph = 0;
+    // last issued phase per barrier, for draining after an abort
+    int q_issued = 0;
+    uint32_t q_last[kQStages] = {0, 0, 0};
+    bool q_any[kQStages] = {false, false, false};
+    bool k_any = false, v_any = false;
+    uint32_t k_last = 0, v_last = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const MUnit m = decode_unit(a, u);
+      if (lane == 0) {
+        ok = mbar_wait(&bar_k_empty, kph ^ 1, abort_flag, a.err, kDevTimeoutMma);
+        if (ok) {
+          mbar_arrive_expect_tx(&bar_k_full, Cfg::kKVBytes);
+#pragma unroll
+          for (int ri = 0; ri < Cfg::kRegions; ++ri)
+            tma_load_3d(sK + ri * kKeys * 128, &map_k, &bar_k_full, ri * 64, m.g, m.j * kKeys);
+          k_any = true;
+          k_last = kph;
+        }
+      }
+      kph ^= 1;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      for (int i = 0; i < m.ntiles && ok; ++i) {
+        const int eb = m.e0 + i * a.TT;
+        const int nt = min(a.TT, m.e1 - eb);
+        if (lane == 0) {
+          ok = mbar_wait(&bar_q_empty[qs], qph ^ 1, abort_flag, a.err, kDevTimeoutMma);
+          if (ok) {
+            mbar_arrive_expect_tx(&bar_q_full[qs], (uint32_t)nt * a.HG * D * 2);
+            q_any[qs] = true;
+            q_last[qs] = qph;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane < nt) {
+          int64_t t;
+          int r;
+          read_entry(a, eb + lane, t, r);
+          const int32_t qrow = (int32_t)(t * a.H + (int64_t)m.g * a.HG);
+          uint8_t* dst = sQ + qs * Cfg::kQBytes + lane * slot * 128;
+#pragma unroll
+          for (int ri = 0; ri < Cfg::kRegions; ++ri)
+            tma_load_2d(dst + ri * kRows * 128, &map_q, &bar_q_full[qs], ri * 64, qrow);
+        }
+        __syncwarp();
+        ++q_issued;
+        if (++qs == kQStages) qs = 0, qph ^= 1;
+        if (i == 0) {
+          if (lane == 0) {
+            ok = mbar_wait(&bar_v_empty, vph ^ 1, abort_flag, a.err, kDevTimeoutMma);
+            if (ok) {
+              mbar_arrive_expect_tx(&bar_v_full, Cfg::kKVBytes);
+#pragma unroll
+              for (int ri = 0; ri < Cfg::kRegions; ++ri)
+                tma_load_3d(sV + ri * kKeys * 128, &map_v, &bar_v_full, ri * 64, m.g, m.j * kKeys);
+              v_any = true;
+              v_last = vph;
+            }
+          }
+          vph ^= 1;
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      volatile int no_abort = 0;
+      for (int s = 0; s < kQStages; ++s)
+        if (q_any[s]) mbar_wait(&bar_q_full[s], q_last[s], &no_abort, nullptr, 0);
+      if (k_any) mbar_wait(&bar_k_full, k_last, &no_abort, nullptr, 0);
+      if (v_any) mbar_wait(&bar_v_full, v_last, &no_abort, nullptr, 0);
+    }
+    (void)q_issued;
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(kRows, kKeys, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16(kRows, D, false, true);
+      int qs = 0, sb = 0, pb = 0, ob = 0;
+      uint32_t qph = 0, kph = 0, vph = 0;
+      uint32_t sph[2] = {0, 0}, pph[2] = {0, 0}, oph[2] = {0, 0};
+      bool ok = true;
+      bool has_prev = false, prev_first = false, prev_last = false;
+      bool committed = false;
+      uint64_t* last_bar = nullptr;
+      uint32_t last_par = 0;
+
+      auto issue_pv = [&](bool first, bool last) -> bool {
+        if (!mbar_wait(&bar_p_full[pb], pph[pb], abort_flag, a.err, kDevTimeoutConsumer)) return false;
+        if (!mbar_wait(&bar_o_empty[ob], oph[ob] ^ 1, abort_flag, a.err, kDevTimeoutConsumer))
+          return false;
+        if (first) {
+          if (!mbar_wait(&bar_v_full, vph, abort_flag, a.err, kDevTimeoutLoad)) return false;
+          vph ^= 1;
+        }
+        tc_fence_after();
+        const uint32_t p_base = smem_u32(sP + pb * Cfg::kPBytes);
+        const uint32_t v_base = smem_u32(sV);
+        const uint32_t d_tm = tmem + 256 + ob * 128;
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          const uint64_t ad =
+              smem_desc_sw128(p_base + (kk >> 2) * kRows * 128 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(v_base + kk * 16 * 128, kKeys * 128, 1024);
+          umma_bf16(d_tm, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar_p_empty[pb]);
+        umma_commit(&bar_o_full[ob]);
+        if (last) umma_commit(&bar_v_empty);
+        committed = true;
+        last_bar = &bar_o_full[ob];
+        last_par = oph[ob];
+        pph[pb] ^= 1;
+        pb ^= 1;
+        oph[ob] ^= 1;
+        ob ^= 1;
+        return true;
+      };
+
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const MUnit m = decode_unit(a, u);
+        for (int i = 0; i < m.ntiles; ++i) {
+          if (i == 0) {
+            if (!mbar_wait(&bar_k_full, kph, abort_flag, a.err, kDevTimeoutLoad)) {
+              ok = false;
+              break;
+            }
+            kph ^= 1;
+          }
+          if (!mbar_wait(&bar_q_full[qs], qph, abort_flag, a.err, kDevTimeoutLoad) ||
+              !mbar_wait(&bar_s_empty[sb], sph[sb] ^ 1, abort_flag, a.err, kDevTimeoutConsumer)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t q_base = smem_u32(sQ + qs * Cfg::kQBytes);
+          const uint32_t k_base = smem_u32(sK);
+          const uint32_t d_tm = tmem + sb * 128;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad =
+                smem_desc_sw128(q_base + (kk >> 2) * kRows * 128 + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd =
+                smem_desc_sw128(k_base + (kk >> 2) * kKeys * 128 + (kk & 3) * 32, 16, 1024);
+            umma_bf16(d_tm, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar_q_empty[qs]);
+          umma_commit(&bar_s_full[sb]);
+          if (i == m.ntiles - 1) umma_commit(&bar_k_empty);
+          committed = true;
+          last_bar = &bar_s_full[sb];
+          last_par = sph[sb];
+          sph[sb] ^= 1;
+          sb ^= 1;
+          if (++qs == kQStages) qs = 0, qph ^= 1;
+          if (has_prev && !issue_pv(prev_first, prev_last)) {
+            ok = false;
+            break;
+          }
+          has_prev = true;
+          prev_first = (i == 0);
+          prev_last = (i == m.ntiles - 1);
+        }
+      }
+      if (ok && has_prev) ok = issue_pv(prev_first, prev_last);
+      if (*abort_flag && committed) {
+        volatile int no_abort = 0;
+        mbar_wait(last_bar, last_par, &no_abort, nullptr, 0);
+      }
+    }
+  } else {
+    // ---------------- softmax + epilogue: warps 2..5 ----------------
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int ts = row >> a.log2slot;
+    const int hh = row & (slot - 1);
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    int sb = 0, pb = 0, ob = 0;
+    uint32_t sph[2] = {0, 0}, pph[2] = {0, 0}, oph[2] = {0, 0};
+    bool ok = true;
+    // the tile whose epilogue is pending
+    bool has_prev = false, prev_valid = false;
+    int64_t prev_t = 0;
+    int prev_r = 0, prev_g = 0;
+    float prev_m = 0.f, prev_l = 1.f;
+
+    auto epilogue = [&]() -> bool {
+      if (!mbar_wait(&bar_o_full[ob], oph[ob], abort_flag, a.err, kDevTimeoutMma)) return false;
+      tc_fence_after();
+      uint32_t o[D / 32][32];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld_32x32b_x32(lane_addr + 256 + ob * 128 + c * 32, o[c]);
+      tmem_wait();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) reg_fence(o[c]);
+      tc_fence_before();
+      mbar_arrive(&bar_o_empty[ob]);
+      oph[ob] ^= 1;
+      ob ^= 1;
+      if (prev_valid) {
+        const float inv = 1.0f / prev_l;
+        const int64_t slot_idx =
+            (((prev_t - a.row_begin) * a.G + prev_g) * a.top_k + prev_r) * a.HG + hh;
+        uint4* dst = reinterpret_cast<uint4*>(a.part_o + slot_idx * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            uint4 w;
+            w.x = pack_half2(__uint_as_float(o[c][q8 * 8 + 0]) * inv,
+                             __uint_as_float(o[c][q8 * 8 + 1]) * inv);
+            w.y = pack_half2(__uint_as_float(o[c][q8 * 8 + 2]) * inv,
+                             __uint_as_float(o[c][q8 * 8 + 3]) * inv);
+            w.z = pack_half2(__uint_as_float(o[c][q8 * 8 + 4]) * inv,
+                             __uint_as_float(o[c][q8 * 8 + 5]) * inv);
+            w.w = pack_half2(__uint_as_float(o[c][q8 * 8 + 6]) * inv,
+                             __uint_as_float(o[c][q8 * 8 + 7]) * inv);
+            dst[c * 4 + q8] = w;
+          }
+        a.part_lse[slot_idx] = prev_m * a.scale + logf(prev_l);
+      }
+      return true;
+    };
+
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const MUnit m = decode_unit(a, u);
+      for (int i = 0; i < m.ntiles; ++i) {
+        const int e = m.e0 + i * a.TT + ts;
+        const bool row_valid = (e < m.e1) && (hh < a.HG);
+        int64_t t = 0;
+        int r = 0;
+        bool good = false;
+        if (row_valid) good = read_entry(a, e, t, r);
+        const int64_t lim64 = t - (int64_t)m.j * kKeys;
+        const int lim = row_valid ? (int)min64(lim64, kKeys - 1) : kKeys - 1;
+
+        // ---- softmax of this tile ----
+        if (!mbar_wait(&bar_s_full[sb], sph[sb], abort_flag, a.err, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t s[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(lane_addr + sb * 128 + c * 32, s[c]);
+        tmem_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_fence(s[c]);
+        tc_fence_before();
+        mbar_arrive(&bar_s_empty[sb]);
+        sph[sb] ^= 1;
+        sb ^= 1;
+
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            if (c * 32 + x <= lim) mx = fmaxf(mx, __uint_as_float(s[c][x]));
+        if (!(row_valid && good) || !(mx > -INFINITY)) mx = 0.f;
+        const float mxs = mx * a.scale_log2;
+
+        if (!mbar_wait(&bar_p_empty[pb], pph[pb] ^ 1, abort_flag, a.err, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        uint8_t* prow = sP + pb * Cfg::kPBytes;
+        float l = 0.f;
+#pragma unroll
+        for (int c8 = 0; c8 < 16; ++c8) {
+          float p[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const int col = c8 * 8 + x;
+            const float sv = __uint_as_float(s[col >> 5][col & 31]);
+            p[x] = (col <= lim) ? fast_exp2(fmaf(sv, a.scale_log2, -mxs)) : 0.f;
+          }
+          uint4 w;
+          w.x = pack_bf16x2(p[0], p[1]);
+          w.y = pack_bf16x2(p[2], p[3]);
+          w.z = pack_bf16x2(p[4], p[5]);
+          w.w = pack_bf16x2(p[6], p[7]);
+          // normalise by the sum of the values the tensor core actually uses
+          l += sum_bf16x2(w.x) + sum_bf16x2(w.y) + sum_bf16x2(w.z) + sum_bf16x2(w.w);
+          *reinterpret_cast<uint4*>(prow + (c8 >> 3) * kRows * 128 + sw128_offset(row, c8 & 7)) = w;
+        }
+        fence_async_smem();
+        mbar_arrive(&bar_p_full[pb]);
+        pph[pb] ^= 1;
+        pb ^= 1;
+
+        // ---- epilogue of the previous tile ----
+        if (has_prev && !epilogue()) {
+          ok = false;
+          break;
+        }
+        has_prev = true;
+        prev_valid = row_valid && good;
+        prev_t = t;
+        prev_r = r;
+        prev_g = m.g;
+        prev_m = mx;
+        prev_l = l;
+      }
+    }
+    if (ok && has_prev) epilogue();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+template <int D>
+cudaError_t launch_main_impl(const MainLaunch& p, cudaStream_t s) {
+  using Cfg = MainCfg<D>;
+  const int HG = p.H / p.G;
+  const int slot = HG < 8 ? 8 : HG;
+  CUtensorMap mq, mk, mv;
+  if (!make_tmap_bf16_2d(&mq, p.q, (uint64_t)p.N * p.H, D, D, (uint32_t)HG, 64,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_bf16_3d(&mk, p.k, D, p.G, p.N, D, (uint64_t)p.G * D, 64, 1, kKeys,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_bf16_3d(&mv, p.v, D, p.G, p.N, D, (uint64_t)p.G * D, 64, 1, kKeys,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  MainArgs a;
+  a.N = p.N;
+  a.row_begin = p.row_begin;
+  a.rows = p.rows;
+  a.H = p.H;
+  a.G = p.G;
+  a.HG = HG;
+  a.log2slot = 31 - __builtin_clz(slot);
+  a.TT = kRows / slot;
+  a.top_k = p.top_k;
+  a.scale = p.scale;
+  a.scale_log2 = p.scale * kLog2e;
+  a.nb = p.nb;
+  a.row_ptr = p.row_ptr;
+  a.entries = p.entries;
+  a.unit_ptr = p.unit_ptr;
+  a.unit_list = p.unit_list;
+  a.per_unit = a.TT * p.unit_tiles;
+  a.part_o = p.part_o;
+  a.part_lse = p.part_lse;
+  a.err = p.err;
+  auto kern = main_kernel<D>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<p.grid, kThreads, Cfg::kSmem, s>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int main_tile_tokens(int H, int G) {
+  const int HG = H / G;
+  return kRows / (HG < 8 ? 8 : HG);
+}
+
+cudaError_t launch_main(const MainLaunch& p, cudaStream_t s) {
+  if (p.d == 128) return launch_main_impl<128>(p, s);
+  return launch_main_impl<64>(p, s);
+}
+
+}  // namespace msa

@@ -1,0 +1,223 @@
+/*
+ * msa.h -- C ABI of the B200 (sm_100a) MiniMax Sparse Attention hot path.
+ *
+ * MSA is two-branch block-sparse attention on top of GQA (ai-tool-zukan
+ * "MiniMax MSA guide", section "MiniMax MSAとは何か"):
+ *   Index Branch: every causally visible key token is scored with one
+ *     index-query head per GQA group against one shared index-key head; the
+ *     token scores are max-pooled per 128-token key block; a top-k operator
+ *     keeps k blocks per (query, group), and the block holding the query is
+ *     always kept (guide, sections "2段階構造の中身——ブロック選択から厳密アテンション
+ *     まで" and "クエリを含むローカルブロックの強制取り込み").  All heads of a group
+ *     share its block set (section "GQAグループ単位の選択共有とは").
+ *   Main Branch: exact causal softmax attention over the selected blocks
+ *     only (section "Index BranchとMain Branchの役割分担"), organised with key
+ *     blocks as the outer loop and the hitting queries gathered per block
+ *     (tnkblog MiniMax M3 / MSA post, section "MSA の実装").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are DEVICE pointers unless stated otherwise, to
+ *    contiguous row-major data, 16-byte aligned.  bf16 tensors are passed as
+ *    `const void*` (IEEE bfloat16 bit patterns).
+ *  - Shapes use N tokens, H query heads, G groups (KV heads; head h belongs to
+ *    group h / (H/G)), d head dim, d_idx index dim, nb = ceil(N/128) blocks,
+ *    k = top_k.
+ *  - Ownership: the caller allocates and owns every buffer, the workspace
+ *    included.  The library never allocates device memory and never
+ *    synchronises the stream (except msa_get_device_error).  Every call is
+ *    asynchronous and ordered on `stream`.
+ *  - Errors: arguments are validated on the host before any launch; an
+ *    invalid call returns a status and launches nothing.  A failed launch
+ *    returns MSA_ERR_CUDA.  Kernels never trap: a wait that runs out or a bad
+ *    index is recorded in a device error word inside the workspace and read
+ *    back with msa_get_device_error.
+ *  - Supported shapes: block_size 128; head_dim and index_dim 64 or 128;
+ *    1 <= top_k <= 32; G divides 128; H/G is a power of two dividing 128;
+ *    1 <= N < 2^26.  Others return MSA_ERR_UNSUPPORTED.
+ *  - Readings where the pages are silent: the token score is the raw dot
+ *    product (no scale); "visible" means key s <= query t; k includes the
+ *    local block; equal pooled scores go to the lower block id; ids are
+ *    written ascending with -1 padding; logits are softmax_scale * <q, k>.
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* msa_stream_t;
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned pointer */
+  MSA_ERR_UNSUPPORTED = 2,    /* shape outside the supported set above */
+  MSA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than required */
+  MSA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  MSA_ERR_DEVICE_TIMEOUT = 5, /* a kernel wait ran out (reported by msa_get_device_error) */
+  MSA_ERR_DEVICE_INDEX = 6    /* a kernel met an out-of-range id (msa_get_device_error) */
+} msa_status_t;
+
+typedef struct {
+  int32_t num_heads;   /* H */
+  int32_t num_groups;  /* G: GQA groups = KV heads = index-query heads */
+  int32_t head_dim;    /* d */
+  int32_t index_dim;   /* d_idx */
+  int32_t block_size;  /* B_k, must be 128 (guide, table "既定ブロックサイズ") */
+  int32_t top_k;       /* k blocks per (query, group), counting the local block */
+  float softmax_scale; /* logits = softmax_scale * <q, k>, usually 1/sqrt(d) */
+} msa_config_t;
+
+typedef enum {
+  MSA_OP_SELECT_TOPK = 0,
+  MSA_OP_BLOCK_QUERY_LISTS = 1,
+  MSA_OP_PREFILL = 2,
+  MSA_OP_DECODE = 3
+} msa_op_t;
+
+/*
+ * Workspace bytes needed by `op`.
+ *   SELECT_TOPK, BLOCK_QUERY_LISTS, PREFILL: n_tokens = N, batch ignored.
+ *     For PREFILL this is the size that processes all N queries in one pass;
+ *     msa_prefill also accepts any workspace of at least
+ *     msa_workspace_size(cfg, PREFILL, 128*ceil(min(N, 16384)/128)...) -- see
+ *     msa_prefill_min_workspace -- and then walks the query axis in chunks.
+ *   DECODE: n_tokens = total cache rows (sum of sequence lengths), batch = B.
+ * Host-only; returns MSA_ERR_INVALID_ARG / MSA_ERR_UNSUPPORTED like the op.
+ */
+MSA_API msa_status_t msa_workspace_size(const msa_config_t* cfg, msa_op_t op, int64_t n_tokens,
+                                int32_t batch, size_t* bytes);
+
+/* Smallest workspace msa_prefill accepts for N tokens (it then processes the
+ * query axis in chunks of at least 128 tokens).  Host-only. */
+MSA_API msa_status_t msa_prefill_min_workspace(const msa_config_t* cfg, int64_t N, size_t* bytes);
+
+/*
+ * Index Branch scores, pooled per block (guide, section "2段階構造の中身": token
+ * scores max-pooled to the block level).
+ *   q_idx  [N][G][d_idx] bf16, k_idx [N][d_idx] bf16.
+ *   scores [row_count][G][nb] fp32 out: for query row t = row_begin + i,
+ *          scores[i][g][j] = max over keys s in block j with s <= t of
+ *          <q_idx[t][g], k_idx[s]> (fp32 accumulation of bf16 products);
+ *          -inf for blocks with no visible key (j > t/128).
+ *   0 <= row_begin, row_begin + row_count <= N, row_count >= 1.
+ * Needs no workspace.  Meant for inspection and tests; msa_select_topk does
+ * not materialise these scores.
+ */
+MSA_API msa_status_t msa_index_scores(const msa_config_t* cfg, const void* q_idx, const void* k_idx,
+                              int64_t N, int64_t row_begin, int64_t row_count, float* scores,
+                              msa_stream_t stream);
+
+/*
+ * Index Branch selection: ids[t][g] = the local block t/128 plus the
+ * min(k-1, t/128) earlier blocks with the highest pooled scores (ties -> lower
+ * block id), ascending, padded with -1 (guide, sections "2段階構造の中身" and
+ * "クエリを含むローカルブロックの強制取り込み"; budget k*128 keys per query,
+ * table in "ブロック単位選択の数値設計").
+ *   q_idx [N][G][d_idx] bf16, k_idx [N][d_idx] bf16 -> ids [N][G][k] int32.
+ *   ws: at least msa_workspace_size(cfg, MSA_OP_SELECT_TOPK, N, 0).
+ * Scores are fp32 on the tensor cores; two blocks whose scores differ by less
+ * than the fp32 rounding of a d_idx-term dot product may rank differently than
+ * in exact arithmetic.
+ */
+MSA_API msa_status_t msa_select_topk(const msa_config_t* cfg, const void* q_idx, const void* k_idx,
+                             int64_t N, int32_t* ids, void* ws, size_t ws_bytes,
+                             msa_stream_t stream);
+
+/*
+ * Inversion of the selection map into per-(group, key block) query lists, the
+ * schedule of the KV-block-outer Main Branch (tnkblog MiniMax M3 / MSA post,
+ * section "MSA の実装"; CSDN M3 write-up, section "MiniMax Sparse Attention
+ * （MSA）": key blocks as the outer loop, the queries that hit a block gathered).
+ *   ids     [N][G][k] int32 (as written by msa_select_topk; -1 = empty)
+ *   row_ptr [G*nb + 1] int32 out: list of (g, j) is entries[row_ptr[g*nb+j] ..
+ *           row_ptr[g*nb+j+1]).
+ *   entries [N*G*k] int32 out (capacity): each entry is (t << 5) | r, the
+ *           query t and the slot r with ids[t][g][r] == j; ascending t.
+ *   ws: at least msa_workspace_size(cfg, MSA_OP_BLOCK_QUERY_LISTS, N, 0).
+ * Deterministic; an id outside [-1, nb) raises MSA_ERR_DEVICE_INDEX in the
+ * device error word and is skipped.
+ */
+MSA_API msa_status_t msa_build_block_query_lists(const msa_config_t* cfg, const int32_t* ids, int64_t N,
+                                         int32_t* row_ptr, int32_t* entries, void* ws,
+                                         size_t ws_bytes, msa_stream_t stream);
+
+/*
+ * Whole prefill: Index Branch selection, query lists, Main Branch over the
+ * selected blocks, merge of the per-block partial softmaxes.
+ *   q [N][H][d], k/v [N][G][d], q_idx [N][G][d_idx], k_idx [N][d_idx] bf16.
+ *   out [N][H][d] bf16 out: softmax over the keys s <= t of the selected
+ *       blocks of softmax_scale*<q[t][h], k[s][g]>, times v[s][g]; fp32
+ *       accumulation, rounded to bf16 (nearest even).
+ *   ids_out [N][G][k] int32 out, nullable: the selection used.
+ *   ws: at least msa_prefill_min_workspace(); with less than
+ *       msa_workspace_size(PREFILL, N) the query axis is processed in chunks.
+ */
+MSA_API msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, const void* v,
+                         const void* q_idx, const void* k_idx, int64_t N, void* out,
+                         int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream);
+
+/*
+ * One decode step for B sequences.  The pages give decode speed-ups only
+ * (zhaixingw M3 review, section "这套注意力到底怎么省的"); the plainest reading,
+ * used here, is the same two branches for the newest query row, which sits at
+ * position L_b - 1 of its sequence (its own key/value rows are already in the
+ * caches).
+ *   q [B][H][d], q_idx [B][G][d_idx] bf16;
+ *   k_cache, v_cache [sum L][G][d], k_idx_cache [sum L][d_idx] bf16, packed:
+ *     sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1;
+ *   cu_seqlens [B+1] int64, DEVICE pointer, cu_seqlens[0] = 0, every L_b >= 1;
+ *   max_seqlen: host value >= every L_b (sizes the grid);
+ *   out [B][H][d] bf16 out; ids_out [B][G][k] int32 out, nullable.
+ *   ws: at least msa_workspace_size(cfg, MSA_OP_DECODE, sum L, B).
+ */
+MSA_API msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_idx,
+                        const void* k_cache, const void* v_cache, const void* k_idx_cache,
+                        const int64_t* cu_seqlens, int32_t B, int64_t max_seqlen, void* out,
+                        int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream);
+
+/*
+ * Reads and clears the device error word of a workspace used by the calls
+ * above.  Synchronises `stream` first.  *code = 0 when no kernel reported a
+ * problem; otherwise the first code recorded (0x1xx: a wait ran out ->
+ * returns MSA_ERR_DEVICE_TIMEOUT; 0x2xx: an out-of-range id ->
+ * MSA_ERR_DEVICE_INDEX).
+ */
+MSA_API msa_status_t msa_get_device_error(void* ws, msa_stream_t stream, uint32_t* code);
+
+/* Static description of a status code. */
+MSA_API const char* msa_status_string(msa_status_t status);
+
+/* Number of kernel launches the last successful call on this host thread
+ * issued (for accounting in benchmarks). */
+MSA_API int32_t msa_last_launch_count(void);
+
+/*
+ * Measurement hook (host thread local).  When `events` is non-NULL, later
+ * msa_prefill and msa_decode calls on this thread record CUDA events (type
+ * cudaEvent_t, created by the caller) on their stream at phase boundaries:
+ *   prefill chunk c: events[5c+0] before the index kernel, [5c+1] after it,
+ *     [5c+2] after the query-list kernels, [5c+3] after the Main Branch
+ *     kernel, [5c+4] after the merge kernel (only while 5c+4 < count);
+ *   decode: [0] before the index scan, [1] after it, [2] after the top-k
+ *     kernel, [3] after the attention kernel, [4] after the merge kernel.
+ * Pass NULL to stop recording.  The events are not owned by the library.
+ */
+MSA_API msa_status_t msa_set_phase_events(void* const* events, int32_t count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H */

@@ -1,0 +1,117 @@
+"""The C-ABI library: it loads, exports every symbol include/msa.h declares, and
+its host-side validation and workspace sizing behave as documented.  No call
+here reaches a kernel, so no GPU is needed."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_long_branch_b200 as msa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "msa.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^MSA_API [^(]*?\b(msa_\w+)\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("msa_index_scores", "msa_select_topk", "msa_build_block_query_lists",
+              "msa_prefill", "msa_decode", "msa_workspace_size", "msa_get_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = msa.load_library()
+    for n in _declared():
+        assert hasattr(lib, n), n
+        assert hasattr(msa, n), n  # the binding keeps the C names
+
+
+def _cfg(**kw):
+    base = dict(H=64, G=8, d=128, d_idx=128, top_k=16)
+    base.update(kw)
+    return msa.config(base["H"], base["G"], base["d"], base["d_idx"], top_k=base["top_k"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(H=6, G=4), 1),            # H % G
+    (dict(d=96), 2),                # head dim
+    (dict(d_idx=32), 2),            # index dim
+    (dict(top_k=33), 2),            # k > 32
+    (dict(top_k=0), 1),
+    (dict(H=24, G=8), 2),           # H/G not a power of two
+    (dict(H=12, G=3), 2),           # G not a power of two
+])
+def test_invalid_configs_are_rejected(kw, status):
+    with pytest.raises(msa.MsaError) as e:
+        msa.msa_workspace_size(_cfg(**kw), msa.OP_PREFILL, 4096)
+    assert e.value.status == status
+
+
+def test_block_size_must_be_128():
+    cfg = _cfg()
+    cfg.block_size = 64
+    with pytest.raises(msa.MsaError) as e:
+        msa.msa_workspace_size(cfg, msa.OP_PREFILL, 4096)
+    assert e.value.status == 2
+
+
+def test_token_limits():
+    with pytest.raises(msa.MsaError):
+        msa.msa_workspace_size(_cfg(), msa.OP_PREFILL, 0)
+    with pytest.raises(msa.MsaError):
+        msa.msa_workspace_size(_cfg(), msa.OP_PREFILL, 1 << 26)
+
+
+def test_workspace_sizes_are_consistent():
+    cfg = _cfg()
+    full = msa.msa_workspace_size(cfg, msa.OP_PREFILL, 32768)
+    small = msa.msa_prefill_min_workspace(cfg, 32768)
+    assert 0 < small < full
+    # partials dominate: rows * G * k * (H/G) * (2d + 4) bytes
+    assert full >= 32768 * 8 * 16 * 8 * (2 * 128 + 4)
+    assert msa.msa_workspace_size(cfg, msa.OP_SELECT_TOPK, 32768) == 256
+    dec = msa.msa_workspace_size(cfg, msa.OP_DECODE, 5242880, 17)
+    assert dec > (5242880 // 128) * 8 * 4
+
+
+def test_null_pointers_rejected_before_any_launch():
+    lib = msa.load_library()
+    cfg = _cfg()
+    st = lib.msa_prefill(ctypes.byref(cfg), None, None, None, None, None, 128, None, None, None,
+                         0, None)
+    assert st == 1
+    st = lib.msa_select_topk(ctypes.byref(cfg), None, None, 128, None, None, 0, None)
+    assert st == 1
+    st = lib.msa_decode(ctypes.byref(cfg), None, None, None, None, None, None, 1, 1, None, None,
+                        None, 0, None)
+    assert st == 1
+
+
+def test_misaligned_pointer_rejected():
+    lib = msa.load_library()
+    cfg = _cfg()
+    p = ctypes.c_void_p(0x1000)
+    bad = ctypes.c_void_p(0x1002)
+    st = lib.msa_select_topk(ctypes.byref(cfg), bad, p, 128, p, p, 4096, None)
+    assert st == 1
+
+
+def test_missing_workspace_rejected():
+    lib = msa.load_library()
+    cfg = _cfg()
+    p = ctypes.c_void_p(0x1000)
+    st = lib.msa_select_topk(ctypes.byref(cfg), p, p, 128, p, None, 0, None)
+    assert st == 3
+    st = lib.msa_build_block_query_lists(ctypes.byref(cfg), p, 1024, p, p, p, 16, None)
+    assert st == 3
+
+
+def test_status_strings():
+    for s in range(7):
+        assert msa.msa_status_string(s)

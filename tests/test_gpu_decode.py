@@ -1,0 +1,115 @@
+"""GPU parity: one decode step against the fp64 oracle, every query checked."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def msa(cuda_device):
+    import block_sparse_long_branch_b200 as m
+    m.load_library()
+    return m
+
+
+def _cfg(msa, s):
+    return msa.config(s.H, s.G, s.d, s.d_idx, top_k=s.top_k, block=s.block, scale=s.scale)
+
+
+def _oracle_one(inp, s, b):
+    """Oracle for sequence b.  Only the selected key blocks' K/V rows are copied
+    to the host: they are stacked in ascending block order, which keeps every
+    selected key's visibility (the local block is the last one)."""
+    cu = inp["cu_seqlens"].tolist()
+    s0, s1 = cu[b], cu[b + 1]
+    L = s1 - s0
+    nb = (L + s.block - 1) // s.block
+    pos = np.array([L - 1], dtype=np.int64)
+    qib = oracle.as_bf16_bits(inp["q_idx"][b:b + 1])
+    pooled = oracle.pooled_scores(qib, pos, inp["k_idx_cache"][s0:s1], s.block, nb)
+    ids = oracle.select_blocks(pooled, pos, s.block, s.top_k)
+    used = sorted({int(j) for j in ids[0].ravel() if j >= 0})
+    remap = {j: c for c, j in enumerate(used)}
+    kc = torch.zeros(len(used) * s.block, s.G, s.d, dtype=torch.bfloat16)
+    vc = torch.zeros_like(kc)
+    for c, j in enumerate(used):
+        r0, r1 = s0 + j * s.block, min(s1, s0 + (j + 1) * s.block)
+        kc[c * s.block:c * s.block + (r1 - r0)] = inp["k_cache"][r0:r1].cpu()
+        vc[c * s.block:c * s.block + (r1 - r0)] = inp["v_cache"][r0:r1].cpu()
+    cids = np.vectorize(lambda j: remap[j] if j >= 0 else -1)(ids).astype(np.int32)
+    cpos = np.array([(len(used) - 1) * s.block + (L - 1) % s.block], dtype=np.int64)
+    out = oracle.block_attention(oracle.as_bf16_bits(inp["q"][b:b + 1]), cpos, kc, vc, cids,
+                                 s.scale, s.block)
+    return ids[0], pooled[0], out[0], (used, remap, kc, vc, cpos)
+
+
+def _run(msa, s, inp):
+    cu = inp["cu_seqlens"].cuda()
+    cfg = _cfg(msa, s)
+    total = inp["k_cache"].shape[0]
+    ws = torch.empty(msa.msa_workspace_size(cfg, msa.OP_DECODE, total, s.B), dtype=torch.uint8,
+                     device="cuda")
+    out, ids = msa.msa_decode(cfg, inp["q"], inp["q_idx"], inp["k_cache"], inp["v_cache"],
+                              inp["k_idx_cache"], cu, max(s.seq_lens), ids_out=True,
+                              workspace=ws)
+    assert msa.msa_get_device_error(ws) == 0
+    return out.float().cpu().numpy(), ids.cpu().numpy()
+
+
+def _check(msa, s, inp):
+    g_out, g_ids = _run(msa, s, inp)
+    n_ties = 0
+    for b in range(s.B):
+        L = s.seq_lens[b]
+        pos = np.array([L - 1])
+        ids, pooled, out, (used, remap, kc, vc, cpos) = _oracle_one(inp, s, b)
+        parity.check_id_rows_valid(g_ids[b:b + 1], pos, s.block, s.top_k)
+        ties = parity.compare_ids(g_ids[b:b + 1], ids[None], pooled[None], pos, s.block, s.top_k)
+        if ties:
+            n_ties += len(ties)
+            # oracle Main Branch on the GPU's blocks (those rows' K/V copied as above)
+            gsel = sorted({int(j) for j in g_ids[b].ravel() if j >= 0})
+            s0 = int(inp["cu_seqlens"][b])
+            kc2 = torch.zeros(len(gsel) * s.block, s.G, s.d, dtype=torch.bfloat16)
+            vc2 = torch.zeros_like(kc2)
+            for c, j in enumerate(gsel):
+                r0, r1 = s0 + j * s.block, min(s0 + L, s0 + (j + 1) * s.block)
+                kc2[c * s.block:c * s.block + (r1 - r0)] = inp["k_cache"][r0:r1].cpu()
+                vc2[c * s.block:c * s.block + (r1 - r0)] = inp["v_cache"][r0:r1].cpu()
+            rm = {j: c for c, j in enumerate(gsel)}
+            cids = np.vectorize(lambda j: rm[j] if j >= 0 else -1)(g_ids[b:b + 1]).astype(np.int32)
+            cpos2 = np.array([(len(gsel) - 1) * s.block + (L - 1) % s.block])
+            out = oracle.block_attention(oracle.as_bf16_bits(inp["q"][b:b + 1]), cpos2, kc2, vc2,
+                                         cids, s.scale, s.block)[0]
+        parity.check_output(g_out[b], out)
+    for (b, j, g) in inp["needles"]:
+        assert j in g_ids[b, g], (b, j, g)
+    return n_ties
+
+
+def test_decode_small_mixed_lengths(msa):
+    s = synth.DecodeShape("ds", seq_lens=(300, 5000, 128 * 20 + 7, 128, 1, 2049), H=16, G=2,
+                          d=128, d_idx=64, top_k=4, needles_per_seq=(1, 2, 2, 0, 0, 1), seed=12)
+    inp = synth.make_decode_inputs(s, device="cuda")
+    _check(msa, s, inp)
+
+
+def test_decode_small_d64_topk32(msa):
+    s = synth.DecodeShape("ds2", seq_lens=(9000, 4096, 700), H=8, G=8, d=64, d_idx=128, top_k=32,
+                          needles_per_seq=(3, 2, 1), seed=13)
+    inp = synth.make_decode_inputs(s, device="cuda")
+    _check(msa, s, inp)
+
+
+@pytest.mark.slow
+def test_decode_full_config_every_query(msa):
+    """16 x 256K + 1 x 1M caches, every one of the 17 queries against the oracle."""
+    s = synth.DECODE_CONFIG
+    inp = synth.make_decode_inputs(s, device="cuda")
+    n_ties = _check(msa, s, inp)
+    assert n_ties <= 8

@@ -1,0 +1,196 @@
+"""GPU parity: the sm_100a prefill path against the fp64 oracle.
+
+Every kernel is reached through the C ABI (ctypes binding).  Inputs come from
+the shared seeded generator; expected values come only from ``oracle/``.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def msa(cuda_device):
+    import block_sparse_long_branch_b200 as m
+    m.load_library()
+    return m
+
+
+def _cfg(msa, s):
+    return msa.config(s.H, s.G, s.d, s.d_idx, top_k=s.top_k, block=s.block, scale=s.scale)
+
+
+def _ref(inp, s, rows=None, partials=False):
+    return oracle.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                          block=s.block, top_k=s.top_k, scale=s.scale, rows=rows,
+                          partials=partials)
+
+
+def _check_prefill(msa, s, inp, rows=None, workspace=None):
+    cfg = _cfg(msa, s)
+    out, ids = msa.msa_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                               ids_out=True, workspace=workspace)
+    torch.cuda.synchronize()
+    ref = _ref(inp, s, rows=rows)
+    rows = ref["rows"]
+    g_ids = ids.cpu().numpy()[rows]
+    parity.check_id_rows_valid(g_ids, rows, s.block, s.top_k)
+    ties = parity.compare_ids(g_ids, ref["ids"], ref["pooled"], rows, s.block, s.top_k)
+    ref_out = ref["out"]
+    if ties:  # re-run the Main Branch of the oracle on the GPU's selection
+        ref_out = oracle.block_attention(oracle.as_bf16_bits(inp["q"])[rows], rows, inp["k"],
+                                         inp["v"], g_ids, s.scale, s.block)
+    g_out = out.float().cpu().numpy()[rows]
+    errs = parity.check_output(g_out, ref_out)
+    return out, ids, ties, errs
+
+
+# ---------------------------------------------------------------- index branch
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_dense"])
+def test_index_scores_match_oracle(msa, name):
+    s = synth.PREFILL_CONFIGS[name]
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    got = msa.msa_index_scores(cfg, inp["q_idx"], inp["k_idx"]).cpu().numpy()
+    rows = np.arange(s.N)
+    want = oracle.pooled_scores(inp["q_idx"], rows, inp["k_idx"], s.block, s.nb)
+    inv = np.isneginf(want)
+    assert np.array_equal(np.isneginf(got), inv)
+    assert np.abs(got[~inv] - want[~inv]).max() < 1e-3
+
+
+def test_index_scores_row_window_ragged(msa):
+    s = synth.PrefillShape("w", N=1000, H=8, G=4, d=128, d_idx=128, top_k=4, n_needles=2,
+                           seed=31)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    got = msa.msa_index_scores(cfg, inp["q_idx"], inp["k_idx"], row_begin=301,
+                               row_count=555).cpu().numpy()
+    rows = np.arange(301, 856)
+    want = oracle.pooled_scores(oracle.as_bf16_bits(inp["q_idx"])[rows], rows, inp["k_idx"],
+                                s.block, s.nb)
+    inv = np.isneginf(want)
+    assert np.array_equal(np.isneginf(got), inv)
+    assert np.abs(got[~inv] - want[~inv]).max() < 1e-3
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_dense"])
+def test_select_topk_matches_oracle(msa, name):
+    s = synth.PREFILL_CONFIGS[name]
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    ids = msa.msa_select_topk(_cfg(msa, s), inp["q_idx"], inp["k_idx"]).cpu().numpy()
+    rows = np.arange(s.N)
+    pooled = oracle.pooled_scores(inp["q_idx"], rows, inp["k_idx"], s.block, s.nb)
+    ref = oracle.select_blocks(pooled, rows, s.block, s.top_k)
+    parity.check_id_rows_valid(ids, rows, s.block, s.top_k)
+    ties = parity.compare_ids(ids, ref, pooled, rows, s.block, s.top_k)
+    assert len(ties) <= 4, ties
+    for (j, g, t) in inp["needles"]:
+        assert j in ids[t, g]
+
+
+def test_select_ties_go_to_lower_block(msa):
+    """Integer-valued index vectors: many exactly equal pooled scores."""
+    s = synth.PrefillShape("ties", N=2048, H=4, G=2, d=64, d_idx=64, top_k=5)
+    g = torch.Generator().manual_seed(3)
+    q_idx = torch.randint(-1, 2, (s.N, s.G, s.d_idx), generator=g).to(torch.bfloat16).cuda()
+    k_idx = torch.randint(-1, 2, (s.N, s.d_idx), generator=g).to(torch.bfloat16).cuda()
+    ids = msa.msa_select_topk(_cfg(msa, s), q_idx, k_idx).cpu().numpy()
+    rows = np.arange(s.N)
+    pooled = oracle.pooled_scores(q_idx, rows, k_idx, s.block, s.nb)
+    ref = oracle.select_blocks(pooled, rows, s.block, s.top_k)
+    np.testing.assert_array_equal(ids, ref)  # integer sums are exact in fp32
+
+
+# ---------------------------------------------------------------- query lists
+
+@pytest.mark.parametrize("N,G,top_k", [(4096, 2, 16), (1000, 4, 4), (5000, 8, 32), (130, 1, 2)])
+def test_block_query_lists_exact(msa, N, G, top_k):
+    s = synth.PrefillShape("c", N=N, H=G, G=G, d=64, d_idx=64, top_k=top_k, n_needles=3,
+                           seed=N + top_k)
+    inp = synth.make_prefill_inputs(s)
+    rows = np.arange(N)
+    ids = oracle.select_blocks(oracle.pooled_scores(inp["q_idx"], rows, inp["k_idx"], s.block,
+                                                    s.nb), rows, s.block, top_k)
+    want_ptr, want_ent = oracle.block_query_lists(ids, s.nb)
+    row_ptr, entries = msa.msa_build_block_query_lists(_cfg(msa, s),
+                                                       torch.from_numpy(ids).cuda())
+    row_ptr = row_ptr.cpu().numpy()
+    np.testing.assert_array_equal(row_ptr, want_ptr)
+    np.testing.assert_array_equal(entries.cpu().numpy()[:row_ptr[-1]], want_ent)
+
+
+# ---------------------------------------------------------------- whole prefill
+
+def test_prefill_tiny_all_rows(msa):
+    s = synth.PREFILL_CONFIGS["tiny"]
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    _, ids, ties, _ = _check_prefill(msa, s, inp)
+    ids = ids.cpu().numpy()
+    for (j, g, t) in inp["needles"]:
+        assert j in ids[t, g]
+
+
+def test_prefill_tiny_topk32_equals_dense(msa):
+    """k >= number of blocks: the GPU result must equal dense causal GQA."""
+    s = synth.PREFILL_CONFIGS["tiny_dense"]
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    out, ids, ties, _ = _check_prefill(msa, s, inp)
+    assert not ties
+    q = inp["q"].float().permute(1, 0, 2)[None]
+    k = inp["k"].float().repeat_interleave(s.H // s.G, dim=1).permute(1, 0, 2)[None]
+    v = inp["v"].float().repeat_interleave(s.H // s.G, dim=1).permute(1, 0, 2)[None]
+    dense = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True,
+                                                             scale=s.scale)
+    dense = dense[0].permute(1, 0, 2)
+    assert (out.float() - dense).abs().max().item() < 1e-2
+
+
+@pytest.mark.parametrize("N,H,G,d,di,k", [(1000, 16, 2, 128, 128, 16), (1333, 8, 8, 64, 128, 3),
+                                         (777, 32, 4, 128, 64, 32), (129, 8, 1, 64, 64, 1)])
+def test_prefill_ragged_shapes(msa, N, H, G, d, di, k):
+    s = synth.PrefillShape("r", N=N, H=H, G=G, d=d, d_idx=di, top_k=k, n_needles=3,
+                           seed=N * 7 + H)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    _check_prefill(msa, s, inp)
+
+
+def test_prefill_chunked_equals_one_shot(msa):
+    s = synth.PrefillShape("ch", N=3000, H=16, G=4, d=128, d_idx=128, top_k=8, n_needles=4,
+                           seed=8)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    out1, ids1 = msa.msa_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                                 ids_out=True)
+    small = msa.msa_prefill_min_workspace(cfg, s.N) * 3
+    ws = torch.empty(small, dtype=torch.uint8, device="cuda")
+    out2, ids2 = msa.msa_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                                 ids_out=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(ids1, ids2)
+    assert torch.equal(out1, out2)
+    assert msa.msa_get_device_error(ws) == 0
+
+
+def test_prefill_32k_sampled_rows(msa):
+    """The 32K workload in the launch configuration the benchmark times."""
+    s = synth.PREFILL_CONFIGS["prefill_32k"]
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    needle_rows = [t for (_, _, t) in inp["needles"]][:16]
+    rows = synth.sample_rows(s.N, 48, seed=5, extra=needle_rows)
+    ws = torch.empty(msa.msa_workspace_size(_cfg(msa, s), msa.OP_PREFILL, s.N),
+                     dtype=torch.uint8, device="cuda")
+    out, ids, ties, errs = _check_prefill(msa, s, inp, rows=rows, workspace=ws)
+    assert msa.msa_get_device_error(ws) == 0
+    ids = ids.cpu().numpy()
+    for (j, g, t) in inp["needles"]:
+        assert j in ids[t, g]
+    # properties that hold at every row: the forced local block and the budget
+    parity.check_id_rows_valid(ids, np.arange(s.N), s.block, s.top_k)
+    assert torch.isfinite(out.float()).all()
