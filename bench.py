@@ -390,12 +390,16 @@ def run_ours(args, rank, world, local):
                          "frac": ach / peak, "work_per_launch": work}
 
     pm = pre_ph.mean(axis=0)
+    pmed = np.median(pre_ph, axis=0)
     add("index_select", float(pm[0]), "tensor", idx_f, False)
     add("block_query_lists", float(pm[1]), "hbm", pw["csr_bytes"], True)
     add("main_branch", float(pm[2]), "hbm", pw["main_bytes"], True)
     kernels["main_branch"]["tensor_tflops"] = pw["main_flops"] / (pm[2] * 1e-3) / 1e12
     kernels["main_branch"]["tensor_frac"] = kernels["main_branch"]["tensor_tflops"] / tc_peak
     add("merge", float(pm[3]), "hbm", pw["merge_bytes"], True)
+    for n, name in enumerate(PREFILL_PHASES):
+        kernels[name]["ms_median"] = float(pmed[n])
+        kernels[name]["ms_min"] = float(pre_ph[:, n].min())
     decode_obj = None
     if dec is not None:
         dw = decode_work(dc.seq_lens, dc.H, dc.G, dc.d, dc.d_idx, dids.cpu().numpy(), dc.block)
@@ -405,6 +409,10 @@ def run_ours(args, rank, world, local):
         add("decode_attention", float(dm[2]), "hbm", dw["attn_bytes"], True)
         add("decode_merge", float(dm[3]), "hbm",
             dc.B * dc.H * dc.top_k * (2 * dc.d + 4.0) + dc.B * dc.H * dc.d * 2.0, True)
+        dmed = np.median(dec_ph, axis=0)
+        for n, name in enumerate(DECODE_PHASES):
+            kernels[name]["ms_median"] = float(dmed[n])
+            kernels[name]["ms_min"] = float(dec_ph[:, n].min())
         dstep_bytes = dw["bytes"]
         decode_obj = {"value": world * dc.B / (dec_ms * 1e-3), "unit": "tokens/s",
                       "ms_per_step": dec_ms,

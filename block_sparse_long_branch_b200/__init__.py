@@ -76,6 +76,10 @@ def load_library():
     global _lib
     if _lib is not None:
         return _lib
+    from . import build as _build
+    if not _build.is_current():
+        # sources changed since the last build: rebuild in-tree (nvcc, sm_100a)
+        _build.build()
     if not os.path.exists(_LIB_PATH):
         raise RuntimeError(f"libmsa_b200.so not built ({_LIB_PATH}); run "
                            "block_sparse_long_branch_b200/build.py")
@@ -278,6 +282,9 @@ def msa_set_phase_events(events) -> None:
         _check(lib.msa_set_phase_events(None, 0), "msa_set_phase_events")
         _phase_keep = None
         return
+    for e in events:  # torch creates the CUDA event lazily, on its first record
+        if not e.cuda_event:
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _phase_keep = (arr, events)
     _check(lib.msa_set_phase_events(arr, len(events)), "msa_set_phase_events")

@@ -37,6 +37,15 @@ def _deps_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def is_current() -> bool:
+    """True when the library exists and was built from the current sources."""
+    stamp = os.path.join(BUILD, "stamp")
+    if not (os.path.exists(LIB) and os.path.exists(stamp)):
+        return False
+    with open(stamp) as f:
+        return f.read().strip() == _deps_hash()
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     tag = _deps_hash()

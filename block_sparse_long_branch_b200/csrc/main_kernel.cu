@@ -22,9 +22,12 @@
 //              TMA gather of each hitting token's H/G contiguous query rows;
 //   warp 1     MMA issuer (one thread), S of tile i+1 issued before P V of
 //              tile i so the tensor core never waits on the softmax;
-//   warps 2-5  softmax + epilogue, thread <-> TMEM lane <-> tile row; the
-//              epilogue of tile i runs after the softmax of tile i+1.
-// TMEM: two S buffers (2 x 128 columns) and two O buffers (2 x 128 columns).
+//   warps 2-9  two softmax + epilogue warpgroups taking alternate tiles;
+//              thread <-> TMEM lane <-> tile row.  The epilogue stages the
+//              fp16 partials in the tile's (consumed) P buffer and writes each
+//              token's heads with one bulk copy (2 KiB for 8 heads of 128).
+// TMEM: two S buffers (2 x 128 columns) and two O buffers (2 x 128 columns),
+// buffer w belonging to warpgroup w.
 #include "kernels.h"
 #include "sm100.cuh"
 #include "tmap.h"
@@ -32,7 +35,7 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA, 2 softmax warpgroups
 constexpr int kRows = 128;
 constexpr int kKeys = 128;
 constexpr int kQStages = 3;
@@ -82,7 +85,52 @@ __device__ __forceinline__ MUnit decode_unit(const MainArgs& a, int u) {
   return m;
 }
 
+struct TilePos {
+  int u, i;
+  MUnit m;
+  bool more;
+};
+
+__device__ __forceinline__ TilePos first_tile(const MainArgs& a, int n_units) {
+  TilePos p;
+  p.u = blockIdx.x;
+  p.i = 0;
+  p.more = p.u < n_units;
+  if (p.more) p.m = decode_unit(a, p.u);
+  return p;
+}
+
+__device__ __forceinline__ void next_tile(TilePos& p, const MainArgs& a, int n_units) {
+  if (!p.more) return;
+  if (++p.i >= p.m.ntiles) {
+    p.i = 0;
+    p.u += gridDim.x;
+    p.more = p.u < n_units;
+    if (p.more) p.m = decode_unit(a, p.u);
+  }
+}
+
+// raw list entry of this thread's row in tile p (-1 for padding rows)
+__device__ __forceinline__ int32_t prefetch_entry(const MainArgs& a, const TilePos& p, int ts,
+                                                  int hh) {
+  const int e = p.m.e0 + p.i * a.TT + ts;
+  return (e < p.m.e1 && hh < a.HG) ? __ldg(a.entries + e) : -1;
+}
+
 // decoded list entry, validated against the lists' query range
+__device__ __forceinline__ bool check_entry(const MainArgs& a, int32_t ent, int64_t& t, int& r) {
+  t = (int64_t)(ent >> 5);
+  r = ent & 31;
+  const bool ok = ent >= 0 && t >= a.row_begin && t < a.row_begin + a.rows && t < a.N &&
+                  r < a.top_k;
+  if (!ok) {
+    record_error(a.err, kDevBadIndex);
+    t = a.row_begin;
+    r = 0;
+  }
+  return ok;
+}
+
 __device__ __forceinline__ bool read_entry(const MainArgs& a, int e, int64_t& t, int& r) {
   const int32_t ent = __ldg(a.entries + e);
   t = (int64_t)(ent >> 5);
@@ -100,7 +148,8 @@ __device__ __forceinline__ bool read_entry(const MainArgs& a, int e, int64_t& t,
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     main_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                const __grid_constant__ CUtensorMap map_v, const MainArgs a) {
+                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
+                const MainArgs a) {
   using Cfg = MainCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -157,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&map_q);
       tma_prefetch_desc(&map_k);
       tma_prefetch_desc(&map_v);
+      tma_prefetch_desc(&map_o);
     }
     int qs = 0;
     uint32_t qph = 0, kph = 0, vph = 0;
@@ -331,111 +381,112 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---------------- softmax + epilogue: warps 2..5 ----------------
+    // ---------------- softmax + epilogue: two warpgroups ----------------
+    // warpgroup w (warps 2+4w .. 5+4w) owns the tiles of parity w, and with
+    // them S buffer w, P buffer w and O buffer w.
+    const int wg = (warp - 2) >> 2;
+    const uint32_t bar_id = 1 + wg;  // named barrier of this warpgroup
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int ts = row >> a.log2slot;
     const int hh = row & (slot - 1);
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    int sb = 0, pb = 0, ob = 0;
-    uint32_t sph[2] = {0, 0}, pph[2] = {0, 0}, oph[2] = {0, 0};
+    const uint32_t s_col = wg * 128, o_col = 256 + wg * 128;
+    uint8_t* pbuf = sP + wg * Cfg::kPBytes;
+    uint32_t sph = 0, pph = 0, oph = 0;
     bool ok = true;
-    // the tile whose epilogue is pending
-    bool has_prev = false, prev_valid = false;
-    int64_t prev_t = 0;
-    int prev_r = 0, prev_g = 0;
-    float prev_m = 0.f, prev_l = 1.f;
+    bool store_pending = false;  // this thread issued bulk stores from pbuf
 
-    auto epilogue = [&]() -> bool {
-      if (!mbar_wait(&bar_o_full[ob], oph[ob], abort_flag, a.err, kDevTimeoutMma)) return false;
-      tc_fence_after();
-      uint32_t o[D / 32][32];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld_32x32b_x32(lane_addr + 256 + ob * 128 + c * 32, o[c]);
-      tmem_wait();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) reg_fence(o[c]);
-      tc_fence_before();
-      mbar_arrive(&bar_o_empty[ob]);
-      oph[ob] ^= 1;
-      ob ^= 1;
-      if (prev_valid) {
-        const float inv = 1.0f / prev_l;
-        const int64_t slot_idx =
-            (((prev_t - a.row_begin) * a.G + prev_g) * a.top_k + prev_r) * a.HG + hh;
-        uint4* dst = reinterpret_cast<uint4*>(a.part_o + slot_idx * D);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c)
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            uint4 w;
-            w.x = pack_half2(__uint_as_float(o[c][q8 * 8 + 0]) * inv,
-                             __uint_as_float(o[c][q8 * 8 + 1]) * inv);
-            w.y = pack_half2(__uint_as_float(o[c][q8 * 8 + 2]) * inv,
-                             __uint_as_float(o[c][q8 * 8 + 3]) * inv);
-            w.z = pack_half2(__uint_as_float(o[c][q8 * 8 + 4]) * inv,
-                             __uint_as_float(o[c][q8 * 8 + 5]) * inv);
-            w.w = pack_half2(__uint_as_float(o[c][q8 * 8 + 6]) * inv,
-                             __uint_as_float(o[c][q8 * 8 + 7]) * inv);
-            dst[c * 4 + q8] = w;
-          }
-        a.part_lse[slot_idx] = prev_m * a.scale + logf(prev_l);
+    // Tile position in this CTA's sequence; this warpgroup takes every other
+    // tile.  The next tile's list entry is loaded one iteration ahead.
+    TilePos cur = first_tile(a, n_units);
+    if (wg == 1) next_tile(cur, a, n_units);
+    int32_t cur_ent = cur.more ? prefetch_entry(a, cur, ts, hh) : -1;
+
+    while (cur.more && ok) {
+      TilePos nxt = cur;
+      next_tile(nxt, a, n_units);
+      next_tile(nxt, a, n_units);
+      const int32_t nxt_ent = nxt.more ? prefetch_entry(a, nxt, ts, hh) : -1;
+      const MUnit& m = cur.m;
+      const int e = m.e0 + cur.i * a.TT + ts;
+      const bool row_valid = (e < m.e1) && (hh < a.HG);
+      int64_t t = 0;
+      int r = 0;
+      bool good = false;
+      if (row_valid) good = check_entry(a, cur_ent, t, r);
+      const int lim = row_valid ? (int)min64(t - (int64_t)m.j * kKeys, kKeys - 1) : kKeys - 1;
+      const bool unmasked = __all_sync(0xffffffffu, lim >= kKeys - 1);
+
+      // ---- softmax ----
+      if (!mbar_wait(&bar_s_full[wg], sph, abort_flag, a.err, kDevTimeoutMma)) {
+        ok = false;
+        break;
       }
-      return true;
-    };
-
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const MUnit m = decode_unit(a, u);
-      for (int i = 0; i < m.ntiles; ++i) {
-        const int e = m.e0 + i * a.TT + ts;
-        const bool row_valid = (e < m.e1) && (hh < a.HG);
-        int64_t t = 0;
-        int r = 0;
-        bool good = false;
-        if (row_valid) good = read_entry(a, e, t, r);
-        const int64_t lim64 = t - (int64_t)m.j * kKeys;
-        const int lim = row_valid ? (int)min64(lim64, kKeys - 1) : kKeys - 1;
-
-        // ---- softmax of this tile ----
-        if (!mbar_wait(&bar_s_full[sb], sph[sb], abort_flag, a.err, kDevTimeoutMma)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t s[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(lane_addr + sb * 128 + c * 32, s[c]);
+      tc_fence_after();
+      // pass 1: row max, streaming S from TMEM in 64-column halves
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t sv[2][32];
+        tmem_ld_32x32b_x32(lane_addr + s_col + hf * 64, sv[0]);
+        tmem_ld_32x32b_x32(lane_addr + s_col + hf * 64 + 32, sv[1]);
         tmem_wait();
+        reg_fence(sv[0]);
+        reg_fence(sv[1]);
+        if (unmasked) {
+          float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence(s[c]);
-        tc_fence_before();
-        mbar_arrive(&bar_s_empty[sb]);
-        sph[sb] ^= 1;
-        sb ^= 1;
-
-        float mx = -INFINITY;
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+            for (int x = 0; x < 32; x += 4) {
+              x0 = fmaxf(x0, __uint_as_float(sv[c][x]));
+              x1 = fmaxf(x1, __uint_as_float(sv[c][x + 1]));
+              x2 = fmaxf(x2, __uint_as_float(sv[c][x + 2]));
+              x3 = fmaxf(x3, __uint_as_float(sv[c][x + 3]));
+            }
+          mx = fmaxf(mx, fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
+        } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if (c * 32 + x <= lim) mx = fmaxf(mx, __uint_as_float(s[c][x]));
-        if (!(row_valid && good) || !(mx > -INFINITY)) mx = 0.f;
-        const float mxs = mx * a.scale_log2;
-
-        if (!mbar_wait(&bar_p_empty[pb], pph[pb] ^ 1, abort_flag, a.err, kDevTimeoutMma)) {
-          ok = false;
-          break;
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              if (hf * 64 + c * 32 + x <= lim) mx = fmaxf(mx, __uint_as_float(sv[c][x]));
         }
-        uint8_t* prow = sP + pb * Cfg::kPBytes;
-        float l = 0.f;
+      }
+      if (!(row_valid && good) || !(mx > -INFINITY)) mx = 0.f;
+      const float mxs = mx * a.scale_log2;
+
+      if (!mbar_wait(&bar_p_empty[wg], pph ^ 1, abort_flag, a.err, kDevTimeoutMma)) {
+        ok = false;
+        break;
+      }
+      // the previous tile's partials are still being copied out of this buffer
+      if (store_pending) {
+        bulk_wait_read<0>();
+        store_pending = false;
+      }
+      named_barrier(bar_id, 128);
+      // pass 2: P = exp2(scale*log2e*(S - max)) in bf16, written in the K-major
+      // 128-byte-swizzled layout the PV MMA reads
+      float l = 0.f;
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t sv[2][32];
+        tmem_ld_32x32b_x32(lane_addr + s_col + hf * 64, sv[0]);
+        tmem_ld_32x32b_x32(lane_addr + s_col + hf * 64 + 32, sv[1]);
+        tmem_wait();
+        reg_fence(sv[0]);
+        reg_fence(sv[1]);
 #pragma unroll
-        for (int c8 = 0; c8 < 16; ++c8) {
+        for (int c8 = 0; c8 < 8; ++c8) {
           float p[8];
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
-            const int col = c8 * 8 + x;
-            const float sv = __uint_as_float(s[col >> 5][col & 31]);
-            p[x] = (col <= lim) ? fast_exp2(fmaf(sv, a.scale_log2, -mxs)) : 0.f;
+            const int cl = c8 * 8 + x;  // column within this half
+            const float v = fast_exp2(
+                fmaf(__uint_as_float(sv[cl >> 5][cl & 31]), a.scale_log2, -mxs));
+            p[x] = (unmasked || hf * 64 + cl <= lim) ? v : 0.f;
           }
           uint4 w;
           w.x = pack_bf16x2(p[0], p[1]);
@@ -444,28 +495,66 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.w = pack_bf16x2(p[6], p[7]);
           // normalise by the sum of the values the tensor core actually uses
           l += sum_bf16x2(w.x) + sum_bf16x2(w.y) + sum_bf16x2(w.z) + sum_bf16x2(w.w);
-          *reinterpret_cast<uint4*>(prow + (c8 >> 3) * kRows * 128 + sw128_offset(row, c8 & 7)) = w;
+          *reinterpret_cast<uint4*>(pbuf + hf * kRows * 128 + sw128_offset(row, c8)) = w;
         }
-        fence_async_smem();
-        mbar_arrive(&bar_p_full[pb]);
-        pph[pb] ^= 1;
-        pb ^= 1;
-
-        // ---- epilogue of the previous tile ----
-        if (has_prev && !epilogue()) {
-          ok = false;
-          break;
-        }
-        has_prev = true;
-        prev_valid = row_valid && good;
-        prev_t = t;
-        prev_r = r;
-        prev_g = m.g;
-        prev_m = mx;
-        prev_l = l;
       }
+      tc_fence_before();
+      mbar_arrive(&bar_s_empty[wg]);
+      sph ^= 1;
+      fence_async_smem();
+      mbar_arrive(&bar_p_full[wg]);
+      pph ^= 1;
+
+      // ---- epilogue: O / l -> fp16 partial, staged in the (now free) P buffer ----
+      if (!mbar_wait(&bar_o_full[wg], oph, abort_flag, a.err, kDevTimeoutMma)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool valid = row_valid && good;
+      const float inv = 1.0f / l;
+      // same 128-byte-swizzled layout as P: conflict-free writes, and the TMA
+      // store below undoes the swizzle on its way to global memory
+#pragma unroll 1
+      for (int hf = 0; hf < D / 64; ++hf) {
+        uint32_t o[2][32];
+        tmem_ld_32x32b_x32(lane_addr + o_col + hf * 64, o[0]);
+        tmem_ld_32x32b_x32(lane_addr + o_col + hf * 64 + 32, o[1]);
+        tmem_wait();
+        reg_fence(o[0]);
+        reg_fence(o[1]);
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint4 w;
+          const uint32_t* src = &o[c8 >> 2][(c8 & 3) * 8];
+          w.x = pack_half2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
+          w.y = pack_half2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
+          w.z = pack_half2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
+          w.w = pack_half2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
+          *reinterpret_cast<uint4*>(pbuf + hf * kRows * 128 + sw128_offset(row, c8)) = w;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar_o_empty[wg]);
+      oph ^= 1;
+      fence_async_smem();
+      named_barrier(bar_id, 128);
+      if (valid) {
+        const int64_t slot0 = (((t - a.row_begin) * a.G + m.g) * a.top_k + r) * a.HG;
+        a.part_lse[slot0 + hh] = mx * a.scale + logf(l);
+        if (hh == 0) {
+#pragma unroll
+          for (int ri = 0; ri < Cfg::kRegions; ++ri)
+            tma_store_2d(&map_o, pbuf + ri * kRows * 128 + (ts << a.log2slot) * 128, ri * 64,
+                         (int32_t)slot0);
+          bulk_commit();
+          store_pending = true;
+        }
+      }
+      cur = nxt;
+      cur_ent = nxt_ent;
     }
-    if (ok && has_prev) epilogue();
+    if (store_pending) bulk_wait<0>();
   }
 
   tc_fence_before();
@@ -478,9 +567,12 @@ cudaError_t launch_main_impl(const MainLaunch& p, cudaStream_t s) {
   using Cfg = MainCfg<D>;
   const int HG = p.H / p.G;
   const int slot = HG < 8 ? 8 : HG;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
+  const uint64_t part_rows = (uint64_t)p.rows * p.G * p.top_k * HG;
   if (!make_tmap_bf16_2d(&mq, p.q, (uint64_t)p.N * p.H, D, D, (uint32_t)HG, 64,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&mo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.part_o, part_rows, D, D,
+                    (uint32_t)HG, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_bf16_3d(&mk, p.k, D, p.G, p.N, D, (uint64_t)p.G * D, 64, 1, kKeys,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_bf16_3d(&mv, p.v, D, p.G, p.N, D, (uint64_t)p.G * D, 64, 1, kKeys,
@@ -511,7 +603,7 @@ cudaError_t launch_main_impl(const MainLaunch& p, cudaStream_t s) {
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<p.grid, kThreads, Cfg::kSmem, s>>>(mq, mk, mv, a);
+  kern<<<p.grid, kThreads, Cfg::kSmem, s>>>(mq, mk, mv, mo, a);
   return cudaGetLastError();
 }
 

@@ -22,21 +22,29 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D bf16 view [rows][cols] (row pitch `pitch_elems`), box [box_rows][box_cols].
-// Returns false if the driver rejects the map (alignment, box or stride rules).
-inline bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                              uint64_t pitch_elems, uint32_t box_rows, uint32_t box_cols,
-                              CUtensorMapSwizzle swizzle) {
+// 2-D view [rows][cols] of 16-bit elements (row pitch `pitch_elems`), box
+// [box_rows][box_cols].  Returns false if the driver rejects the map
+// (alignment, box or stride rules).
+inline bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base,
+                         uint64_t rows, uint64_t cols, uint64_t pitch_elems, uint32_t box_rows,
+                         uint32_t box_cols, CUtensorMapSwizzle swizzle) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {pitch_elems * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+inline bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                              uint64_t pitch_elems, uint32_t box_rows, uint32_t box_cols,
+                              CUtensorMapSwizzle swizzle) {
+  return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rows, cols, pitch_elems,
+                      box_rows, box_cols, swizzle);
 }
 
 // 3-D bf16 view [d2][d1][d0] (element strides: 1, pitch1, pitch2), box

@@ -100,6 +100,8 @@ PREFILL_CONFIGS = {
                          n_needles=8, seed=SEED_BASE + 0),
     "tiny_dense": PrefillShape("tiny_dense", N=4096, H=4, G=2, d=64, d_idx=64,
                                top_k=32, n_needles=8, seed=SEED_BASE + 0),
+    "prefill_8k": PrefillShape("prefill_8k", N=8192, H=64, G=8, d=128, d_idx=128, top_k=16,
+                               n_needles=16, seed=SEED_BASE + 5),
     "prefill_32k": PrefillShape("prefill_32k", N=32768, H=64, G=8, d=128,
                                 d_idx=128, top_k=16, n_needles=64,
                                 seed=SEED_BASE + 1),
