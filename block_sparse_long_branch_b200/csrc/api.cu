@@ -43,6 +43,7 @@ msa_status_t check_cfg(const msa_config_t* c) {
   if (!pow2(c->num_groups) || c->num_groups > 128) return MSA_ERR_UNSUPPORTED;
   const int hg = c->num_heads / c->num_groups;
   if (!pow2(hg) || hg > 128) return MSA_ERR_UNSUPPORTED;
+  if (hg * c->head_dim > 2048) return MSA_ERR_UNSUPPORTED;  // one group's heads: <= 4 KiB bf16
   return MSA_OK;
 }
 

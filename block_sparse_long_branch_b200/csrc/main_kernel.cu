@@ -145,6 +145,38 @@ __device__ __forceinline__ bool read_entry(const MainArgs& a, int e, int64_t& t,
   return ok;
 }
 
+// exp2 of 64 scores (one half of a row), bf16 packing into the swizzled P
+// tile, and the fp32 sum of the rounded values.  MASK: keep columns <= lim.
+template <bool MASK>
+__device__ __forceinline__ void softmax_chunk(const uint32_t (&sv)[2][32], uint64_t k2,
+                                              uint64_t nm2, int lim, uint8_t* pdst, int row,
+                                              uint64_t& acc_a, uint64_t& acc_b) {
+#pragma unroll
+  for (int c8 = 0; c8 < 8; ++c8) {
+    uint32_t w4[4];
+#pragma unroll
+    for (int x2 = 0; x2 < 4; ++x2) {
+      const int col = c8 * 8 + 2 * x2;
+      const uint64_t s2 = f2_pack(__uint_as_float(sv[col >> 5][col & 31]),
+                                  __uint_as_float(sv[col >> 5][(col & 31) + 1]));
+      float a0, a1;
+      f2_unpack(f2_fma(s2, k2, nm2), a0, a1);
+      float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+      if (MASK) {
+        p0 = col <= lim ? p0 : 0.f;
+        p1 = col + 1 <= lim ? p1 : 0.f;
+      }
+      const uint32_t w = pack_bf16x2(p0, p1);
+      if (x2 & 1)
+        acc_b = f2_add(acc_b, bf16x2_as_f2(w));
+      else
+        acc_a = f2_add(acc_a, bf16x2_as_f2(w));
+      w4[x2] = w;
+    }
+    *reinterpret_cast<uint4*>(pdst + sw128_offset(row, c8)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     main_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -435,17 +467,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         reg_fence(sv[0]);
         reg_fence(sv[1]);
         if (unmasked) {
-          float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
+          float x0 = mx, x1 = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int x = 0; x < 32; x += 4) {
-              x0 = fmaxf(x0, __uint_as_float(sv[c][x]));
-              x1 = fmaxf(x1, __uint_as_float(sv[c][x + 1]));
-              x2 = fmaxf(x2, __uint_as_float(sv[c][x + 2]));
-              x3 = fmaxf(x3, __uint_as_float(sv[c][x + 3]));
+              x0 = max3f(x0, __uint_as_float(sv[c][x]), __uint_as_float(sv[c][x + 1]));
+              x1 = max3f(x1, __uint_as_float(sv[c][x + 2]), __uint_as_float(sv[c][x + 3]));
             }
-          mx = fmaxf(mx, fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
+          mx = fmaxf(x0, x1);
         } else {
 #pragma unroll
           for (int c = 0; c < 2; ++c)
@@ -468,8 +498,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       named_barrier(bar_id, 128);
       // pass 2: P = exp2(scale*log2e*(S - max)) in bf16, written in the K-major
-      // 128-byte-swizzled layout the PV MMA reads
-      float l = 0.f;
+      // 128-byte-swizzled layout the PV MMA reads; l sums the rounded values
+      const uint64_t k2 = f2_pack(a.scale_log2, a.scale_log2);
+      const uint64_t nm2 = f2_pack(-mxs, -mxs);
+      uint64_t acc_a = f2_pack(0.f, 0.f), acc_b = acc_a;
 #pragma unroll 1
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t sv[2][32];
@@ -478,26 +510,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait();
         reg_fence(sv[0]);
         reg_fence(sv[1]);
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          float p[8];
-#pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            const int cl = c8 * 8 + x;  // column within this half
-            const float v = fast_exp2(
-                fmaf(__uint_as_float(sv[cl >> 5][cl & 31]), a.scale_log2, -mxs));
-            p[x] = (unmasked || hf * 64 + cl <= lim) ? v : 0.f;
-          }
-          uint4 w;
-          w.x = pack_bf16x2(p[0], p[1]);
-          w.y = pack_bf16x2(p[2], p[3]);
-          w.z = pack_bf16x2(p[4], p[5]);
-          w.w = pack_bf16x2(p[6], p[7]);
-          // normalise by the sum of the values the tensor core actually uses
-          l += sum_bf16x2(w.x) + sum_bf16x2(w.y) + sum_bf16x2(w.z) + sum_bf16x2(w.w);
-          *reinterpret_cast<uint4*>(pbuf + hf * kRows * 128 + sw128_offset(row, c8)) = w;
+        uint8_t* pdst = pbuf + hf * kRows * 128;
+        if (unmasked) {
+          softmax_chunk<false>(sv, k2, nm2, 0, pdst, row, acc_a, acc_b);
+        } else {
+          softmax_chunk<true>(sv, k2, nm2, lim - hf * 64, pdst, row, acc_a, acc_b);
         }
       }
+      float la0, la1, lb0, lb1;
+      f2_unpack(acc_a, la0, la1);
+      f2_unpack(acc_b, lb0, lb1);
+      const float l = (la0 + la1) + (lb0 + lb1);
       tc_fence_before();
       mbar_arrive(&bar_s_empty[wg]);
       sph ^= 1;
@@ -513,6 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool valid = row_valid && good;
       const float inv = 1.0f / l;
+      const uint64_t inv2 = f2_pack(inv, inv);
       // same 128-byte-swizzled layout as P: conflict-free writes, and the TMA
       // store below undoes the swizzle on its way to global memory
 #pragma unroll 1
@@ -527,10 +551,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c8 = 0; c8 < 8; ++c8) {
           uint4 w;
           const uint32_t* src = &o[c8 >> 2][(c8 & 3) * 8];
-          w.x = pack_half2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
-          w.y = pack_half2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
-          w.z = pack_half2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
-          w.w = pack_half2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
+#pragma unroll
+          for (int x2 = 0; x2 < 4; ++x2) {
+            float f0, f1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(src[2 * x2]), __uint_as_float(src[2 * x2 + 1])),
+                             inv2),
+                      f0, f1);
+            (&w.x)[x2] = pack_half2(f0, f1);
+          }
           *reinterpret_cast<uint4*>(pbuf + hf * kRows * 128 + sw128_offset(row, c8)) = w;
         }
       }

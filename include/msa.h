@@ -33,8 +33,9 @@
  *    index is recorded in a device error word inside the workspace and read
  *    back with msa_get_device_error.
  *  - Supported shapes: block_size 128; head_dim and index_dim 64 or 128;
- *    1 <= top_k <= 32; G divides 128; H/G is a power of two dividing 128;
- *    1 <= N < 2^26.  Others return MSA_ERR_UNSUPPORTED.
+ *    1 <= top_k <= 32; G divides 128; H/G is a power of two with
+ *    (H/G) * head_dim <= 2048; 1 <= N < 2^26.  Others return
+ *    MSA_ERR_UNSUPPORTED.
  *  - Readings where the pages are silent: the token score is the raw dot
  *    product (no scale); "visible" means key s <= query t; k includes the
  *    local block; equal pooled scores go to the lower block id; ids are
