@@ -23,7 +23,7 @@ __all__ = [
     "OP_SELECT_TOPK", "OP_BLOCK_QUERY_LISTS", "OP_PREFILL", "OP_DECODE",
     "msa_workspace_size", "msa_prefill_min_workspace", "msa_index_scores", "msa_select_topk",
     "msa_build_block_query_lists", "msa_prefill", "msa_decode", "msa_get_device_error",
-    "msa_status_string", "msa_last_launch_count", "msa_set_phase_events",
+    "msa_status_string", "msa_last_launch_count", "msa_set_phase_events", "msa_decode_static",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -93,6 +93,7 @@ def load_library():
     lib.msa_build_block_query_lists.argtypes = [C, P, I64, P, P, P, SZ, P]
     lib.msa_prefill.argtypes = [C, P, P, P, P, P, I64, P, P, P, SZ, P]
     lib.msa_decode.argtypes = [C, P, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
+    lib.msa_decode_static.argtypes = [C, P, P, P, P, P, P, I32, I64, I64, P, P, I32, P]
     lib.msa_get_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
     lib.msa_status_string.argtypes = [ctypes.c_int]
     lib.msa_status_string.restype = ctypes.c_char_p
@@ -102,7 +103,7 @@ def load_library():
     lib.msa_last_launch_count.restype = I32
     for name in ("msa_workspace_size", "msa_prefill_min_workspace", "msa_index_scores",
                  "msa_select_topk", "msa_build_block_query_lists", "msa_prefill", "msa_decode",
-                 "msa_get_device_error"):
+                 "msa_decode_static", "msa_get_device_error"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -267,6 +268,64 @@ def msa_decode(cfg: MsaConfig, q, q_idx, k_cache, v_cache, k_idx_cache, cu_seqle
                         _dev(out, torch.bfloat16, "out", (B, H, d)), ids_ptr,
                         _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(st, "msa_decode")
+    return out if ids_out is None else (out, ids_out)
+
+
+def msa_decode_static(cfg: MsaConfig, q, q_idx, k_cache, v_cache, k_idx_cache, cu_seqlens,
+                      max_seqlen: int, total_len: int, out: Optional[torch.Tensor] = None,
+                      ids_out=None, check_device_error: bool = False, stream=None):
+    """msa_decode with the library's fixed scratch array instead of a workspace.
+
+    For callers that cannot allocate device memory: the library allocates
+    nothing either.  ``out``/``ids_out`` must then be passed in by the caller.
+    """
+    lib = load_library()
+    B = q.shape[0]
+    H, G, d, di, kk = cfg.num_heads, cfg.num_groups, cfg.head_dim, cfg.index_dim, cfg.top_k
+    total = k_cache.shape[0]
+    if out is None:
+        out = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
+    if ids_out is True:
+        ids_out = torch.empty((B, G, kk), dtype=torch.int32, device=q.device)
+    ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (B, G, kk))
+    st = lib.msa_decode_static(ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (B, H, d)),
+                               _dev(q_idx, torch.bfloat16, "q_idx", (B, G, di)),
+                               _dev(k_cache, torch.bfloat16, "k_cache", (total, G, d)),
+                               _dev(v_cache, torch.bfloat16, "v_cache", (total, G, d)),
+                               _dev(k_idx_cache, torch.bfloat16, "k_idx_cache", (total, di)),
+                               _dev(cu_seqlens, torch.int64, "cu_seqlens", (B + 1,)), B,
+                               max_seqlen, total_len, _dev(out, torch.bfloat16, "out", (B, H, d)),
+                               ids_ptr, 1 if check_device_error else 0, _stream(stream))
+    _check(st, "msa_decode_static")
+    return out if ids_out is None else (out, ids_out)
+
+
+def msa_decode_static(cfg: MsaConfig, q, q_idx, k_cache, v_cache, k_idx_cache, cu_seqlens,
+                      max_seqlen: int, total_len: int, out: Optional[torch.Tensor] = None,
+                      ids_out=None, check_device_error: bool = False, stream=None):
+    """msa_decode with the library's fixed scratch array instead of a workspace.
+
+    For callers that cannot allocate device memory: the library allocates
+    nothing either.  ``out``/``ids_out`` must then be passed in by the caller.
+    """
+    lib = load_library()
+    B = q.shape[0]
+    H, G, d, di, kk = cfg.num_heads, cfg.num_groups, cfg.head_dim, cfg.index_dim, cfg.top_k
+    total = k_cache.shape[0]
+    if out is None:
+        out = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
+    if ids_out is True:
+        ids_out = torch.empty((B, G, kk), dtype=torch.int32, device=q.device)
+    ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (B, G, kk))
+    st = lib.msa_decode_static(ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (B, H, d)),
+                               _dev(q_idx, torch.bfloat16, "q_idx", (B, G, di)),
+                               _dev(k_cache, torch.bfloat16, "k_cache", (total, G, d)),
+                               _dev(v_cache, torch.bfloat16, "v_cache", (total, G, d)),
+                               _dev(k_idx_cache, torch.bfloat16, "k_idx_cache", (total, di)),
+                               _dev(cu_seqlens, torch.int64, "cu_seqlens", (B + 1,)), B,
+                               max_seqlen, total_len, _dev(out, torch.bfloat16, "out", (B, H, d)),
+                               ids_ptr, 1 if check_device_error else 0, _stream(stream))
+    _check(st, "msa_decode_static")
     return out if ids_out is None else (out, ids_out)
 
 

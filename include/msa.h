@@ -189,6 +189,31 @@ MSA_API msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const vo
                         int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream);
 
 /*
+ * msa_decode without a workspace argument, for callers that cannot allocate
+ * device memory (a serving loop whose memory another runtime reserved up
+ * front, a thread that must not enter the allocator, an embedding that only
+ * passes raw input/output pointers).  The pages have no counterpart: this is
+ * a deployment convenience around msa_decode, whose arguments it shares.
+ *   total_len: host value, the sum of the sequence lengths (cu_seqlens[B]).
+ *   check_device_error: non-zero -> synchronise `stream` after the launches
+ *     and return the device error status (as msa_get_device_error would).
+ * Scratch lives in a 16 MiB array compiled into this library, held on every
+ * GPU that loads the library until the process exits.  A call that needs more
+ * (msa_workspace_size(cfg, MSA_OP_DECODE, total_len, B) > 16 MiB; e.g. more
+ * than about 28 sequences at H=64, G=8, d=128, k=16) returns
+ * MSA_ERR_WORKSPACE and launches nothing.  The first call on a device looks
+ * up the array's address (cudaGetSymbolAddress): make it before any stream
+ * capture.  All calls share the array, so calls that overlap on the GPU race;
+ * the caller serialises them.  Allocates nothing: no cudaMalloc / cudaFree.
+ */
+MSA_API msa_status_t msa_decode_static(const msa_config_t* cfg, const void* q, const void* q_idx,
+                                       const void* k_cache, const void* v_cache,
+                                       const void* k_idx_cache, const int64_t* cu_seqlens,
+                                       int32_t B, int64_t max_seqlen, int64_t total_len,
+                                       void* out, int32_t* ids_out, int32_t check_device_error,
+                                       msa_stream_t stream);
+
+/*
  * Reads and clears the device error word of a workspace used by the calls
  * above.  Synchronises `stream` first.  *code = 0 when no kernel reported a
  * problem; otherwise the first code recorded (0x1xx: a wait ran out ->
