@@ -37,7 +37,7 @@ import synth  # noqa: E402
 METRIC = "MSA prefill tokens/s & decode tokens/s on 1 B200; % of tensor/HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_PHASES = ("index_select", "block_query_lists", "main_branch", "merge")
-DECODE_PHASES = ("decode_index", "decode_topk", "decode_attention", "decode_merge")
+DECODE_PHASES = ("decode_index", "decode_select_attend")
 
 
 # --------------------------------------------------------------------------
@@ -272,16 +272,24 @@ def run_reference(args, rank, world):
     return line
 
 
+def decode_shape(args):
+    return synth.DECODE_CONFIG if args.decode_workload == "full" else synth.DECODE_SMALL
+
+
 def workload_config(args, shape):
-    cfg = {"workload": f"{shape.name}" + ("" if args.no_decode else
-                                          f"+{synth.DECODE_CONFIG.name}"),
+    parts = [] if args.no_prefill else [shape.name]
+    if not args.no_decode:
+        parts.append(decode_shape(args).name)
+    cfg = {"workload": "+".join(parts),
            "N": shape.N, "H": shape.H, "G": shape.G, "d": shape.d, "d_idx": shape.d_idx,
            "block": shape.block, "top_k": shape.top_k, "needles": shape.n_needles,
            "l2": "inputs larger than L2 (no flush)", "parallelism": "replicas"}
     if not args.no_decode:
-        dc = synth.DECODE_CONFIG
-        cfg["decode"] = {"seq_lens": f"16x{dc.seq_lens[0]}+1x{dc.seq_lens[-1]}", "B": dc.B,
-                         "H": dc.H, "G": dc.G, "d": dc.d, "d_idx": dc.d_idx, "top_k": dc.top_k}
+        dc = decode_shape(args)
+        lens = sorted(set(dc.seq_lens))
+        desc = "+".join(f"{dc.seq_lens.count(L)}x{L}" for L in lens)
+        cfg["decode"] = {"seq_lens": desc, "B": dc.B, "H": dc.H, "G": dc.G, "d": dc.d,
+                         "d_idx": dc.d_idx, "top_k": dc.top_k}
     return cfg
 
 
@@ -293,16 +301,22 @@ def run_ours(args, rank, world, local):
     import block_sparse_long_branch_b200 as msa
     dev = torch.device("cuda", local)
     shape = synth.PREFILL_CONFIGS[args.workload]
+    do_prefill = not args.no_prefill
+    N = shape.N
     cfg = msa.config(shape.H, shape.G, shape.d, shape.d_idx, top_k=shape.top_k,
                      block=shape.block, scale=shape.scale)
-    inp = synth.make_prefill_inputs(shape, device=dev, seed=shape.seed + rank)
-    N = shape.N
-    ws = torch.empty(msa.msa_workspace_size(cfg, msa.OP_PREFILL, N), dtype=torch.uint8,
-                     device=dev)
-    out = torch.empty((N, shape.H, shape.d), dtype=torch.bfloat16, device=dev)
-    ids = torch.empty((N, shape.G, shape.top_k), dtype=torch.int32, device=dev)
+    if do_prefill:
+        inp = synth.make_prefill_inputs(shape, device=dev, seed=shape.seed + rank)
+        full_ws = msa.msa_workspace_size(cfg, msa.OP_PREFILL, N)
+        cap = int(args.ws_gb * (1 << 30))
+        ws = torch.empty(max(min(full_ws, cap), msa.msa_prefill_min_workspace(cfg, N)),
+                         dtype=torch.uint8, device=dev)
+        out = torch.empty((N, shape.H, shape.d), dtype=torch.bfloat16, device=dev)
+        ids = torch.empty((N, shape.G, shape.top_k), dtype=torch.int32, device=dev)
+        chunk = msa.msa_prefill_chunk_tokens(cfg, N, ws.numel(), ids_returned=True)
+        n_chunks = (N + chunk - 1) // chunk
 
-    dc = synth.DECODE_CONFIG
+    dc = decode_shape(args)
     dec = None
     if not args.no_decode:
         dec = synth.make_decode_inputs(dc, device=dev, seed=dc.seed + rank)
@@ -331,16 +345,19 @@ def run_ours(args, rank, world, local):
 
     # ---- warm-up ----
     for _ in range(args.warmup):
-        prefill_once()
+        if do_prefill:
+            prefill_once()
         if dec is not None:
             decode_once()
     torch.cuda.synchronize()
-    assert msa.msa_get_device_error(ws) == 0, "device error after prefill warm-up"
+    if do_prefill:
+        assert msa.msa_get_device_error(ws) == 0, "device error after prefill warm-up"
     if dec is not None:
         assert msa.msa_get_device_error(dws) == 0, "device error after decode warm-up"
 
-    pev = [mk_events(5) for _ in range(args.steps)]
-    dev_ev = [mk_events(5) for _ in range(args.steps)]
+    # prefill chunks: 5 events per chunk of the query axis
+    pev = [mk_events(5 * n_chunks) for _ in range(args.steps)] if do_prefill else []
+    dev_ev = [mk_events(3) for _ in range(args.steps)]
     launches = 0
     barrier(world)
     torch.cuda.synchronize()
@@ -350,8 +367,9 @@ def run_ours(args, rank, world, local):
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record()
     for i in range(args.steps):
-        msa.msa_set_phase_events(pev[i])
-        launches += prefill_once()
+        if do_prefill:
+            msa.msa_set_phase_events(pev[i])
+            launches += prefill_once()
         if dec is not None:
             msa.msa_set_phase_events(dev_ev[i])
             launches += decode_once()
@@ -361,66 +379,63 @@ def run_ours(args, rank, world, local):
     barrier(world)
     clocks = sampler.stop()
     total_ms = reduce_max(t_start.elapsed_time(t_end), world)
-
-    pre_ph = np.array([_phase_ms(e, 4) for e in pev])          # [K, 4]
-    pre_ms = reduce_max(float(pre_ph.sum(axis=1).mean()), world)
-    if dec is not None:
-        dec_ph = np.array([_phase_ms(e, 4) for e in dev_ev])
-        dec_ms = reduce_max(float(dec_ph.sum(axis=1).mean()), world)
-    assert msa.msa_get_device_error(ws) == 0, "device error in timed prefill"
-
-    # ---- algorithmic work from the selection actually used ----
-    ids_np = ids.cpu().numpy()
-    pw = prefill_work(ids_np, shape.H, shape.d, shape.block)
-    idx_f = index_flops(N, shape.G, shape.d_idx, shape.block)
+    step_ms = total_ms / args.steps
     peaks, peak_src = load_peaks()
     long_region = total_ms > 5000.0
-    tc_peak = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
     tc_name = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+    tc_peak = peaks[tc_name]
     kernels = {}
 
-    def add(name, ms, bound, work, unit_is_bytes):
+    def add(name, ms_arr, bound, work, unit_is_bytes):
+        ms = float(np.mean(ms_arr))
         if unit_is_bytes:
             ach = work / (ms * 1e-3) / 1e9
             peak, unit = peaks["hbm_gbs"], "GB/s"
         else:
             ach = work / (ms * 1e-3) / 1e12
             peak, unit = tc_peak, "TFLOP/s"
-        kernels[name] = {"ms": ms, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
-                         "frac": ach / peak, "work_per_launch": work}
+        kernels[name] = {"ms": ms, "ms_median": float(np.median(ms_arr)),
+                         "ms_min": float(np.min(ms_arr)), "bound": bound, "achieved": ach,
+                         "peak": peak, "unit": unit, "frac": ach / peak,
+                         "work_per_launch": work, "share": ms / step_ms}
 
-    pm = pre_ph.mean(axis=0)
-    pmed = np.median(pre_ph, axis=0)
-    add("index_select", float(pm[0]), "tensor", idx_f, False)
-    add("block_query_lists", float(pm[1]), "hbm", pw["csr_bytes"], True)
-    add("main_branch", float(pm[2]), "hbm", pw["main_bytes"], True)
-    kernels["main_branch"]["tensor_tflops"] = pw["main_flops"] / (pm[2] * 1e-3) / 1e12
-    kernels["main_branch"]["tensor_frac"] = kernels["main_branch"]["tensor_tflops"] / tc_peak
-    add("merge", float(pm[3]), "hbm", pw["merge_bytes"], True)
-    for n, name in enumerate(PREFILL_PHASES):
-        kernels[name]["ms_median"] = float(pmed[n])
-        kernels[name]["ms_min"] = float(pre_ph[:, n].min())
+    prefill_obj, value, pre_ms = None, None, None
+    if do_prefill:
+        assert msa.msa_get_device_error(ws) == 0, "device error in timed prefill"
+        chunks_run = n_chunks
+        # per step, per phase: summed over the chunks of the query axis
+        pre_ph = np.array([[sum(e[5 * c + ph].elapsed_time(e[5 * c + ph + 1])
+                                for c in range(chunks_run)) for ph in range(4)] for e in pev])
+        pre_ms = reduce_max(float(pre_ph.sum(axis=1).mean()), world)
+        ids_np = ids.cpu().numpy()
+        pw = prefill_work(ids_np, shape.H, shape.d, shape.block)
+        idx_f = index_flops(N, shape.G, shape.d_idx, shape.block)
+        add("index_select", pre_ph[:, 0], "tensor", idx_f, False)
+        add("block_query_lists", pre_ph[:, 1], "hbm", pw["csr_bytes"], True)
+        add("main_branch", pre_ph[:, 2], "hbm", pw["main_bytes"], True)
+        kernels["main_branch"]["tensor_tflops"] = (pw["main_flops"] /
+                                                   (kernels["main_branch"]["ms"] * 1e-3) / 1e12)
+        kernels["main_branch"]["tensor_frac"] = kernels["main_branch"]["tensor_tflops"] / tc_peak
+        add("merge", pre_ph[:, 3], "hbm", pw["merge_bytes"], True)
+        value = world * N / (pre_ms * 1e-3)
+        prefill_obj = {"value": value, "unit": "tokens/s", "ms_per_step": pre_ms,
+                       "query_chunks": chunks_run, "dense_flops": dense_flops(N, shape.H, shape.d),
+                       "msa_flops": idx_f + pw["main_flops"],
+                       "selected_keys_per_query": pw["selected_keys"]}
     decode_obj = None
     if dec is not None:
+        dec_ph = np.array([_phase_ms(e, 2) for e in dev_ev])
+        dec_ms = reduce_max(float(dec_ph.sum(axis=1).mean()), world)
         dw = decode_work(dc.seq_lens, dc.H, dc.G, dc.d, dc.d_idx, dids.cpu().numpy(), dc.block)
-        dm = dec_ph.mean(axis=0)
-        add("decode_index", float(dm[0]), "hbm", dw["idx_bytes"], True)
-        add("decode_topk", float(dm[1]), "alu", 0.0, True)
-        add("decode_attention", float(dm[2]), "hbm", dw["attn_bytes"], True)
-        add("decode_merge", float(dm[3]), "hbm",
-            dc.B * dc.H * dc.top_k * (2 * dc.d + 4.0) + dc.B * dc.H * dc.d * 2.0, True)
-        dmed = np.median(dec_ph, axis=0)
-        for n, name in enumerate(DECODE_PHASES):
-            kernels[name]["ms_median"] = float(dmed[n])
-            kernels[name]["ms_min"] = float(dec_ph[:, n].min())
+        add("decode_index", dec_ph[:, 0], "hbm", dw["idx_bytes"], True)
+        add("decode_select_attend", dec_ph[:, 1], "hbm", dw["attn_bytes"], True)
         dstep_bytes = dw["bytes"]
         decode_obj = {"value": world * dc.B / (dec_ms * 1e-3), "unit": "tokens/s",
                       "ms_per_step": dec_ms,
                       "hbm_frac": dstep_bytes / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                       "bytes_per_step": dstep_bytes}
-    step_ms = total_ms / args.steps
-    for name, kinfo in kernels.items():
-        kinfo["share"] = kinfo["ms"] / step_ms
+        if value is None:
+            value = decode_obj["value"]
     dominant = max(kernels, key=lambda k: kernels[k]["ms"])
     dk = kernels[dominant]
     roofline = {"kernel": dominant, "bound": dk["bound"], "achieved": dk["achieved"],
@@ -429,23 +444,19 @@ def run_ours(args, rank, world, local):
                 f"({'hbm_gbs' if dk['unit'] == 'GB/s' else tc_name})"}
 
     # ---- end to end through the public API with host buffers ----
-    e2e = run_e2e(args, msa, cfg, shape, inp, ws, dev, dec, dcfg if dec is not None else None,
+    e2e = run_e2e(args, msa, cfg, shape, inp if do_prefill else None,
+                  ws if do_prefill else None, dev, dec, dcfg if dec is not None else None,
                   dws if dec is not None else None, world)
 
-    value = world * N / (pre_ms * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": workload_config(args, shape),
-        "prefill": {"value": value, "unit": "tokens/s", "ms_per_step": pre_ms,
-                    "dense_flops": dense_flops(N, shape.H, shape.d),
-                    "msa_flops": idx_f + pw["main_flops"],
-                    "selected_keys_per_query": pw["selected_keys"]},
-        "decode": decode_obj, "roofline": roofline, "kernels": kernels, "e2e": e2e,
-        "gpu_launches": launches, "clocks": clocks,
+        "prefill": prefill_obj, "decode": decode_obj, "roofline": roofline, "kernels": kernels,
+        "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
     }
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+    if world == 1 and rank == 0 and do_prefill and not args.no_cpu_baseline:
         os.environ.setdefault("OMP_NUM_THREADS", str(cpu_cores()))
         hinp = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
         rate, rows, el = oracle_prefill_rate(hinp, shape, args.cpu_budget)
@@ -478,84 +489,132 @@ def traffic_for(kernel: str):
 
 
 def run_e2e(args, msa, cfg, shape, inp, ws, dev, dec, dcfg, dws, world):
-    """Host (pinned) inputs -> device -> msa_prefill -> host output, per step."""
+    """Host (pinned) inputs -> device -> msa_prefill -> host output, every step.
+
+    Three streams overlap consecutive steps: step i's kernels run while step
+    i+1's inputs are copied in and step i-1's output is copied out.  Inputs and
+    outputs are double-buffered on both sides; each step still moves its full
+    inputs host->device and its full output device->host inside the timed
+    region.
+    """
+    res = {}
+    if inp is not None:
+        res = _e2e_prefill(args, msa, cfg, shape, inp, ws, dev, world)
+    if dec is not None:
+        res["decode"] = _e2e_decode(args, msa, dec, dcfg, dws, dev, world)
+        if inp is None:
+            res.update({k: v for k, v in res["decode"].items()})
+    return res
+
+
+def _e2e_prefill(args, msa, cfg, shape, inp, ws, dev, world):
     keys = ("q", "k", "v", "q_idx", "k_idx")
-    host = {k: torch.empty_like(inp[k], device="cpu").pin_memory() for k in keys}
-    for k in keys:
-        host[k].copy_(inp[k])
-    dbuf = {k: torch.empty_like(inp[k]) for k in keys}
-    out = torch.empty((shape.N, shape.H, shape.d), dtype=torch.bfloat16, device=dev)
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
-    d2h = out_h.numel() * out_h.element_size()
-    steps = max(3, args.steps // 2)
-    for _ in range(2):
+    host = [{k: torch.empty_like(inp[k], device="cpu").pin_memory() for k in keys}
+            for _ in range(2)]
+    for hb in host:
         for k in keys:
-            dbuf[k].copy_(host[k], non_blocking=True)
-        msa.msa_prefill(cfg, dbuf["q"], dbuf["k"], dbuf["v"], dbuf["q_idx"], dbuf["k_idx"],
-                        out=out, workspace=ws)
-        out_h.copy_(out, non_blocking=True)
+            hb[k].copy_(inp[k])
+    dbuf = [{k: torch.empty_like(inp[k]) for k in keys} for _ in range(2)]
+    outs = [torch.empty((shape.N, shape.H, shape.d), dtype=torch.bfloat16, device=dev)
+            for _ in range(2)]
+    out_h = [torch.empty(outs[0].shape, dtype=outs[0].dtype).pin_memory() for _ in range(2)]
+    h2d = sum(host[0][k].numel() * host[0][k].element_size() for k in keys)
+    d2h = out_h[0].numel() * out_h[0].element_size()
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    steps = max(4, args.steps)
+
+    def run(n, start=None, end=None):
+        used = [False, False]
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if used[b]:
+                    s_in.wait_event(ev_cmp[b])  # buffer b's inputs consumed by step i-2
+                if i == 0 and start is not None:
+                    start.record(s_in)
+                for k in keys:
+                    dbuf[b][k].copy_(host[b][k], non_blocking=True)
+                ev_in[b].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[b])
+                if used[b]:
+                    s_cmp.wait_event(ev_out[b])  # output buffer b copied out by step i-2
+                msa.msa_prefill(cfg, dbuf[b]["q"], dbuf[b]["k"], dbuf[b]["v"], dbuf[b]["q_idx"],
+                                dbuf[b]["k_idx"], out=outs[b], workspace=ws, stream=s_cmp)
+                ev_cmp[b].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[b])
+                out_h[b].copy_(outs[b], non_blocking=True)
+                ev_out[b].record(s_out)
+            used[b] = True
+        if end is not None:
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_in[(n - 1) % 2])
+                end.record(s_out)
+
+    run(2)
     torch.cuda.synchronize()
     barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        for k in keys:
-            dbuf[k].copy_(host[k], non_blocking=True)
-        msa.msa_prefill(cfg, dbuf["q"], dbuf["k"], dbuf["v"], dbuf["q_idx"], dbuf["k_idx"],
-                        out=out, workspace=ws)
-        out_h.copy_(out, non_blocking=True)
-    b.record()
+    run(steps, a, b)
     torch.cuda.synchronize()
     ms = reduce_max(a.elapsed_time(b) / steps, world)
     res = {"value": world * shape.N / (ms * 1e-3), "unit": "tokens/s",
-           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
-    if dec is not None:
-        dc = synth.DECODE_CONFIG
-        # per step: the new token's q / q_idx and its k, v, k_idx cache rows in,
-        # the attention output back
-        last = (dec["cu_seqlens"][1:] - 1).to(dev)
-        hq = dec["q"].cpu().pin_memory()
-        hqi = dec["q_idx"].cpu().pin_memory()
-        hk = dec["k_cache"][last].cpu().pin_memory()
-        hv = dec["v_cache"][last].cpu().pin_memory()
-        hki = dec["k_idx_cache"][last].cpu().pin_memory()
-        dq, dqi = torch.empty_like(dec["q"]), torch.empty_like(dec["q_idx"])
-        drow_k, drow_v, drow_ki = (torch.empty_like(hk, device=dev),
-                                   torch.empty_like(hv, device=dev),
-                                   torch.empty_like(hki, device=dev))
-        dout = torch.empty((dc.B, dc.H, dc.d), dtype=torch.bfloat16, device=dev)
-        dout_h = torch.empty(dout.shape, dtype=dout.dtype).pin_memory()
-        cu_dev = dec["cu_seqlens"].to(dev)
-        dh2d = sum(x.numel() * x.element_size() for x in (hq, hqi, hk, hv, hki))
-
-        def dstep():
-            dq.copy_(hq, non_blocking=True)
-            dqi.copy_(hqi, non_blocking=True)
-            drow_k.copy_(hk, non_blocking=True)
-            drow_v.copy_(hv, non_blocking=True)
-            drow_ki.copy_(hki, non_blocking=True)
-            dec["k_cache"].index_copy_(0, last, drow_k)
-            dec["v_cache"].index_copy_(0, last, drow_v)
-            dec["k_idx_cache"].index_copy_(0, last, drow_ki)
-            msa.msa_decode(dcfg, dq, dqi, dec["k_cache"], dec["v_cache"], dec["k_idx_cache"],
-                           cu_dev, max(dc.seq_lens), out=dout, workspace=dws)
-            dout_h.copy_(dout, non_blocking=True)
-
-        for _ in range(2):
-            dstep()
-        torch.cuda.synchronize()
-        a.record()
-        for _ in range(steps):
-            dstep()
-        b.record()
-        torch.cuda.synchronize()
-        dms = reduce_max(a.elapsed_time(b) / steps, world)
-        res["decode"] = {"value": world * dc.B / (dms * 1e-3), "unit": "tokens/s",
-                         "h2d_bytes_per_step": int(dh2d),
-                         "d2h_bytes_per_step": int(dout_h.numel() * dout_h.element_size()),
-                         "ms_per_step": dms}
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms,
+           "pipelined": "3 streams: copy-in, kernels, copy-out; double-buffered"}
     return res
+
+
+def _e2e_decode(args, msa, dec, dcfg, dws, dev, world):
+    dc = dec["shape"]
+    steps = max(4, args.steps)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # per step: the new token's q / q_idx and its k, v, k_idx cache rows in,
+    # the attention output back
+    last = (dec["cu_seqlens"][1:] - 1).to(dev)
+    hq = dec["q"].cpu().pin_memory()
+    hqi = dec["q_idx"].cpu().pin_memory()
+    hk = dec["k_cache"][last].cpu().pin_memory()
+    hv = dec["v_cache"][last].cpu().pin_memory()
+    hki = dec["k_idx_cache"][last].cpu().pin_memory()
+    dq, dqi = torch.empty_like(dec["q"]), torch.empty_like(dec["q_idx"])
+    drow_k, drow_v, drow_ki = (torch.empty_like(hk, device=dev),
+                               torch.empty_like(hv, device=dev),
+                               torch.empty_like(hki, device=dev))
+    dout = torch.empty((dc.B, dc.H, dc.d), dtype=torch.bfloat16, device=dev)
+    dout_h = torch.empty(dout.shape, dtype=dout.dtype).pin_memory()
+    cu_dev = dec["cu_seqlens"].to(dev)
+    dh2d = sum(x.numel() * x.element_size() for x in (hq, hqi, hk, hv, hki))
+
+    def dstep():
+        dq.copy_(hq, non_blocking=True)
+        dqi.copy_(hqi, non_blocking=True)
+        drow_k.copy_(hk, non_blocking=True)
+        drow_v.copy_(hv, non_blocking=True)
+        drow_ki.copy_(hki, non_blocking=True)
+        dec["k_cache"].index_copy_(0, last, drow_k)
+        dec["v_cache"].index_copy_(0, last, drow_v)
+        dec["k_idx_cache"].index_copy_(0, last, drow_ki)
+        msa.msa_decode(dcfg, dq, dqi, dec["k_cache"], dec["v_cache"], dec["k_idx_cache"],
+                       cu_dev, max(dc.seq_lens), out=dout, workspace=dws)
+        dout_h.copy_(dout, non_blocking=True)
+
+    for _ in range(2):
+        dstep()
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(steps):
+        dstep()
+    b.record()
+    torch.cuda.synchronize()
+    dms = reduce_max(a.elapsed_time(b) / steps, world)
+    return {"value": world * dc.B / (dms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(dh2d),
+            "d2h_bytes_per_step": int(dout_h.numel() * dout_h.element_size()),
+            "ms_per_step": dms}
 
 
 def main(argv=None):
@@ -566,9 +625,14 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="prefill_32k", choices=sorted(synth.PREFILL_CONFIGS))
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="time only the decode step (profiling)")
+    ap.add_argument("--decode-workload", choices=("full", "small"), default="full")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle time for the cpu_baseline sample")
+    ap.add_argument("--ws-gb", type=float, default=96.0,
+                    help="cap on the prefill workspace; above it the query axis is chunked")
     ap.add_argument("--ref-rows", type=int, default=32,
                     help="query rows per step in the reference arm")
     args = ap.parse_args(argv)

@@ -21,7 +21,8 @@ import torch
 __all__ = [
     "MsaConfig", "MsaError", "config", "library_path", "load_library",
     "OP_SELECT_TOPK", "OP_BLOCK_QUERY_LISTS", "OP_PREFILL", "OP_DECODE",
-    "msa_workspace_size", "msa_prefill_min_workspace", "msa_index_scores", "msa_select_topk",
+    "msa_workspace_size", "msa_prefill_min_workspace", "msa_prefill_chunk_tokens",
+    "msa_index_scores", "msa_select_topk",
     "msa_build_block_query_lists", "msa_prefill", "msa_decode", "msa_get_device_error",
     "msa_status_string", "msa_last_launch_count", "msa_set_phase_events", "msa_decode_static",
 ]
@@ -88,6 +89,7 @@ def load_library():
     C = ctypes.POINTER(MsaConfig)
     lib.msa_workspace_size.argtypes = [C, ctypes.c_int, I64, I32, ctypes.POINTER(SZ)]
     lib.msa_prefill_min_workspace.argtypes = [C, I64, ctypes.POINTER(SZ)]
+    lib.msa_prefill_chunk_tokens.argtypes = [C, I64, SZ, I32, ctypes.POINTER(I64)]
     lib.msa_index_scores.argtypes = [C, P, P, I64, I64, I64, P, P]
     lib.msa_select_topk.argtypes = [C, P, P, I64, P, P, SZ, P]
     lib.msa_build_block_query_lists.argtypes = [C, P, I64, P, P, P, SZ, P]
@@ -101,7 +103,8 @@ def load_library():
     lib.msa_set_phase_events.restype = ctypes.c_int
     lib.msa_last_launch_count.argtypes = []
     lib.msa_last_launch_count.restype = I32
-    for name in ("msa_workspace_size", "msa_prefill_min_workspace", "msa_index_scores",
+    for name in ("msa_workspace_size", "msa_prefill_min_workspace", "msa_prefill_chunk_tokens",
+                 "msa_index_scores",
                  "msa_select_topk", "msa_build_block_query_lists", "msa_prefill", "msa_decode",
                  "msa_decode_static", "msa_get_device_error"):
         getattr(lib, name).restype = ctypes.c_int
@@ -153,6 +156,16 @@ def msa_prefill_min_workspace(cfg: MsaConfig, N: int) -> int:
     out = ctypes.c_size_t(0)
     _check(load_library().msa_prefill_min_workspace(ctypes.byref(cfg), N, ctypes.byref(out)),
            "msa_prefill_min_workspace")
+    return int(out.value)
+
+
+def msa_prefill_chunk_tokens(cfg: MsaConfig, N: int, ws_bytes: int,
+                             ids_returned: bool = True) -> int:
+    """Query rows per chunk that msa_prefill uses with ``ws_bytes`` of workspace."""
+    out = ctypes.c_int64(0)
+    _check(load_library().msa_prefill_chunk_tokens(ctypes.byref(cfg), N, ws_bytes,
+                                                   1 if ids_returned else 0, ctypes.byref(out)),
+           "msa_prefill_chunk_tokens")
     return int(out.value)
 
 

@@ -98,17 +98,30 @@ PrefillLayout prefill_layout(const msa_config_t* c, int64_t rows, int64_t nb, bo
   return L;
 }
 
-// decode workspace: header | ids | part_o | part_lse | pooled scores (the rest)
-size_t decode_fixed_bytes(const msa_config_t* c, int32_t B, size_t* off_ids, size_t* off_o,
-                          size_t* off_lse) {
-  const int64_t G = c->num_groups, k = c->top_k, HG = c->num_heads / c->num_groups;
+// Query rows per chunk that msa_prefill processes with `ws_bytes` of workspace:
+// all of N if it fits, else the largest multiple of 128 rows that fits; 0 if
+// not even 128 rows fit.
+int64_t prefill_chunk(const msa_config_t* cfg, int64_t N, size_t ws_bytes, bool own_ids) {
+  const int64_t nb = n_blocks(N);
+  if (prefill_layout(cfg, N, nb, own_ids).total <= ws_bytes) return N;
+  if (prefill_layout(cfg, kBlock, nb, own_ids).total > ws_bytes) return 0;
+  int64_t lo = 1, hi = nb;  // in blocks
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) / 2;
+    if (prefill_layout(cfg, mid * kBlock, nb, own_ids).total <= ws_bytes)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo * kBlock;
+}
+
+// decode workspace: header | ids | pooled block scores (the rest)
+size_t decode_fixed_bytes(const msa_config_t* c, int32_t B, size_t* off_ids) {
+  const int64_t G = c->num_groups, k = c->top_k;
   size_t off = kHeader;
   *off_ids = off;
   off += align256((size_t)B * G * k * 4);
-  *off_o = off;
-  off += align256((size_t)B * G * k * HG * c->head_dim * 2);
-  *off_lse = off;
-  off += align256((size_t)B * G * k * HG * 4);
   return off;
 }
 
@@ -153,6 +166,15 @@ msa_status_t msa_workspace_size(const msa_config_t* cfg, msa_op_t op, int64_t n_
   msa_status_t st = check_cfg(cfg);
   if (st != MSA_OK) return st;
   if (!bytes) return MSA_ERR_INVALID_ARG;
+  if (op == MSA_OP_DECODE) {
+    // total cache rows over all sequences; only per-sequence lengths are bounded
+    if (n_tokens < 1 || batch < 1 || batch > n_tokens || n_tokens >= (int64_t(1) << 40))
+      return MSA_ERR_INVALID_ARG;
+    size_t a;
+    *bytes = decode_fixed_bytes(cfg, batch, &a) +
+             decode_pooled_rows(n_tokens, batch) * cfg->num_groups * sizeof(float);
+    return MSA_OK;
+  }
   if ((st = check_tokens(cfg, n_tokens)) != MSA_OK) return st;
   const int64_t nb = n_blocks(n_tokens);
   switch (op) {
@@ -165,13 +187,8 @@ msa_status_t msa_workspace_size(const msa_config_t* cfg, msa_op_t op, int64_t n_
     case MSA_OP_PREFILL:
       *bytes = prefill_layout(cfg, n_tokens, nb, true).total;
       return MSA_OK;
-    case MSA_OP_DECODE: {
-      if (batch < 1 || batch > n_tokens) return MSA_ERR_INVALID_ARG;
-      size_t a, b, c;
-      *bytes = decode_fixed_bytes(cfg, batch, &a, &b, &c) +
-               decode_pooled_rows(n_tokens, batch) * cfg->num_groups * sizeof(float);
-      return MSA_OK;
-    }
+    case MSA_OP_DECODE:
+      break;
   }
   return MSA_ERR_INVALID_ARG;
 }
@@ -184,6 +201,16 @@ msa_status_t msa_prefill_min_workspace(const msa_config_t* cfg, int64_t N, size_
   const int64_t rows = N < kBlock ? N : kBlock;
   *bytes = prefill_layout(cfg, rows, n_blocks(N), true).total;
   return MSA_OK;
+}
+
+msa_status_t msa_prefill_chunk_tokens(const msa_config_t* cfg, int64_t N, size_t ws_bytes,
+                                      int32_t ids_returned, int64_t* chunk) {
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if (!chunk) return MSA_ERR_INVALID_ARG;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  *chunk = prefill_chunk(cfg, N, ws_bytes, ids_returned == 0);
+  return *chunk == 0 ? MSA_ERR_WORKSPACE : MSA_OK;
 }
 
 msa_status_t msa_index_scores(const msa_config_t* cfg, const void* q_idx, const void* k_idx,
@@ -289,20 +316,8 @@ msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, 
   if (!ws || !aligned16(ws)) return MSA_ERR_WORKSPACE;
   const int64_t nb = n_blocks(N);
   const bool own_ids = ids_out == nullptr;
-  // largest chunk (a multiple of 128 query rows, or all of N) that fits
-  int64_t chunk = N;
-  if (prefill_layout(cfg, chunk, nb, own_ids).total > ws_bytes) {
-    int64_t lo = 1, hi = nb;  // in blocks
-    if (prefill_layout(cfg, kBlock, nb, own_ids).total > ws_bytes) return MSA_ERR_WORKSPACE;
-    while (lo < hi) {
-      const int64_t mid = (lo + hi + 1) / 2;
-      if (prefill_layout(cfg, mid * kBlock, nb, own_ids).total <= ws_bytes)
-        lo = mid;
-      else
-        hi = mid - 1;
-    }
-    chunk = lo * kBlock;
-  }
+  const int64_t chunk = prefill_chunk(cfg, N, ws_bytes, own_ids);
+  if (chunk == 0) return MSA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
   const int G = cfg->num_groups, H = cfg->num_heads, d = cfg->head_dim, kk = cfg->top_k;
@@ -411,8 +426,8 @@ msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_id
     return MSA_ERR_INVALID_ARG;
   if ((st = check_tokens(cfg, max_seqlen)) != MSA_OK) return st;
   if (!ws || !aligned16(ws)) return MSA_ERR_WORKSPACE;
-  size_t off_ids, off_o, off_lse;
-  const size_t fixed = decode_fixed_bytes(cfg, B, &off_ids, &off_o, &off_lse);
+  size_t off_ids;
+  const size_t fixed = decode_fixed_bytes(cfg, B, &off_ids);
   const size_t row_bytes = (size_t)cfg->num_groups * sizeof(float);
   if (ws_bytes < fixed + row_bytes * (size_t)(B + 1)) return MSA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -434,8 +449,6 @@ msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_id
   p.scale = cfg->softmax_scale;
   p.out = out;
   p.ids = ids_out ? ids_out : at<int32_t>(ws, off_ids);
-  p.part_o = at<__half>(ws, off_o);
-  p.part_lse = at<float>(ws, off_lse);
   p.pooled = at<float>(ws, fixed);
   p.pooled_cap = (int64_t)((ws_bytes - fixed) / row_bytes);
   p.err = at<uint32_t>(ws, 0);

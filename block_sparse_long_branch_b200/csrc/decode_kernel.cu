@@ -129,14 +129,14 @@ struct TopList {
 #pragma unroll
     for (int i = 0; i < KSEL; ++i) sc[i] = -INFINITY, id[i] = 0x7FFFFFFF;
   }
-  // candidates must arrive in increasing id order
+  // candidates must arrive in increasing id order: a later equal score loses
   __device__ __forceinline__ void insert(float s, int32_t j) {
     if (!(s > sc[KSEL - 1])) return;
     sc[KSEL - 1] = s;
     id[KSEL - 1] = j;
 #pragma unroll
     for (int i = KSEL - 1; i > 0; --i)
-      if (sc[i] > sc[i - 1] || (sc[i] == sc[i - 1] && id[i] < id[i - 1])) {
+      if (sc[i] > sc[i - 1]) {
         const float ts = sc[i];
         sc[i] = sc[i - 1];
         sc[i - 1] = ts;
@@ -157,163 +157,319 @@ __device__ __forceinline__ bool better(float sa, int32_t ia, float sb, int32_t i
   return sa > sb || (sa == sb && ia < ib);
 }
 
-template <int KSEL>
-__global__ void __launch_bounds__(256)
-    decode_topk_kernel(const float* __restrict__ pooled, const int64_t* __restrict__ cu, int32_t G,
-                       int32_t top_k, int64_t pooled_cap, int32_t* __restrict__ ids) {
-  const int g = blockIdx.x, b = blockIdx.y;
-  const int64_t L = cu[b + 1] - cu[b];
-  const int64_t nb = (L + kBlock - 1) / kBlock;
-  // no scores were written past the workspace: keep only the local block
-  const int64_t n_cand = (pooled_offset(cu, b) + nb > pooled_cap) ? 0 : nb - 1;
-  const float* ps = pooled + pooled_offset(cu, b) * G + g;
-  TopList<KSEL> list;
-  list.init();
-  for (int64_t j = threadIdx.x; j < n_cand; j += blockDim.x) list.insert(ps[j * G], (int32_t)j);
+constexpr int kAttnThreads = 256;
+constexpr int kAttnWarps = kAttnThreads / 32;
 
-  __shared__ float ws_s[8];
-  __shared__ int32_t ws_i[8];
-  __shared__ int32_t chosen[32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int want = (int)min64(top_k - 1, n_cand);
-  for (int round = 0; round < want; ++round) {
-    float s = list.sc[0];
-    int32_t i = list.id[0];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-      const int32_t i2 = __shfl_xor_sync(0xffffffffu, i, o);
-      if (better(s2, i2, s, i)) s = s2, i = i2;
-    }
-    if (lane == 0) ws_s[warp] = s, ws_i[warp] = i;
-    __syncthreads();
-    float bs = ws_s[0];
-    int32_t bi = ws_i[0];
-    for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
-      if (better(ws_s[w], ws_i[w], bs, bi)) bs = ws_s[w], bi = ws_i[w];
-    if (list.id[0] == bi) list.pop();  // ids are unique: exactly one owner pops
-    if (threadIdx.x == 0) chosen[round] = bi;
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
-    int32_t o[33];
-    int n = 0;
-    o[n++] = (int32_t)(nb - 1);
-    for (int r = 0; r < want; ++r) o[n++] = chosen[r];
-    for (int x = 1; x < n; ++x)  // insertion sort, ascending
-      for (int y = x; y > 0 && o[y - 1] > o[y]; --y) {
-        const int32_t t = o[y];
-        o[y] = o[y - 1];
-        o[y - 1] = t;
-      }
-    int32_t* dst = ids + ((int64_t)b * G + g) * top_k;
-    for (int r = 0; r < top_k; ++r) dst[r] = r < n ? o[r] : -1;
-  }
+template <int D, int NT>
+struct AttnSmem {
+  __nv_bfloat16 v[2][kBlock * D];       // V tiles, 16-byte chunks swizzled by key
+  __nv_bfloat16 p[NT * 8][kBlock + 8];  // P (heads x keys), padded rows
+  float red_m[kAttnWarps][NT * 8];
+  float red_l[kAttnWarps][NT * 8];
+  float m_run[NT * 8], l_run[NT * 8], alpha[NT * 8];
+  float o_t[NT * 8][D + 4];             // final O (heads x d) for coalesced stores
+  float ws_s[kAttnWarps];
+  int32_t ws_i[kAttnWarps];
+  int32_t sel[32];
+  int32_t nsel;
+};
+
+// smem offset (elements) of 16-byte chunk c of key row s in a swizzled V tile
+template <int D>
+__device__ __forceinline__ int v_off(int s, int c) {
+  return s * D + ((c ^ (s & 7)) << 3);
 }
 
-// One CTA of 128 threads per (slot r, group g, sequence b).
-template <int D>
-__global__ void __launch_bounds__(128)
-    decode_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
-                       const __nv_bfloat16* __restrict__ vc, const int64_t* __restrict__ cu,
-                       const int32_t* __restrict__ ids, int32_t H, int32_t G, int32_t top_k,
-                       float scale, __half* __restrict__ part_o, float* __restrict__ part_lse,
-                       uint32_t* err) {
-  constexpr int MAXHG = 8;
-  const int r = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int HG = H / G;
-  const int tid = threadIdx.x;
-  const int64_t slot = ((int64_t)b * G + g) * top_k + r;
-  const int32_t j = ids[slot];
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                                  uint32_t& r3, const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p)));
+}
+
+// One CTA per (group g, sequence b):
+//   1. top-k over the pooled scores of the sequence's non-local blocks
+//      (register lists per thread, then k-1 rounds of a block arg-max);
+//   2. attention of the group's H/G heads over the selected blocks with an
+//      online softmax across blocks.  S^T = K Q^T on mma.sync (K rows read
+//      straight from global memory with the permuted reduction axis, Q in
+//      registers), P to shared memory, O^T += V^T P^T on mma.sync with V in a
+//      swizzled shared tile (ldmatrix.trans).  The next block's V is copied in
+//      (cp.async) while the current one is used.
+template <int D, int NT, int KSEL>
+__global__ void __launch_bounds__(kAttnThreads)
+    decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
+                         const __nv_bfloat16* __restrict__ vc, const int64_t* __restrict__ cu,
+                         const float* __restrict__ pooled, int64_t pooled_cap, int32_t G,
+                         int32_t HG, int32_t top_k, float scale_log2,
+                         int32_t* __restrict__ ids_out, __nv_bfloat16* __restrict__ out) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  AttnSmem<D, NT>& sm = *reinterpret_cast<AttnSmem<D, NT>*>(smem_raw);
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t s0 = cu[b];
   const int64_t L = cu[b + 1] - s0;
   const int64_t nb = (L + kBlock - 1) / kBlock;
-  if (j < 0 || j >= nb) {
-    if (j >= nb) record_error(err, kDevBadIndex);
-    for (int h = tid; h < HG; h += blockDim.x) part_lse[slot * HG + h] = -INFINITY;
-    return;
-  }
-  __shared__ float q_s[MAXHG][D];
-  __shared__ float p_s[MAXHG][kBlock];
-  __shared__ __align__(16) __nv_bfloat16 v_s[kBlock][D];
-  __shared__ float red[MAXHG][4];
-  const int nkeys = (int)min64(kBlock, L - (int64_t)j * kBlock);  // keys s <= L-1
 
-  for (int hb = 0; hb < HG; hb += MAXHG) {
-    const int hn = min(MAXHG, HG - hb);
-    for (int x = tid; x < hn * D; x += blockDim.x) {
-      const int h = x / D, c = x % D;
-      q_s[h][c] = __bfloat162float(q[((int64_t)b * H + g * HG + hb + h) * D + c]) * scale;
-    }
-    for (int x = tid; x < kBlock * D / 8; x += blockDim.x) {
-      const int s = x / (D / 8), c8 = x % (D / 8);
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (s < nkeys)
-        val = __ldg(reinterpret_cast<const uint4*>(vc + ((s0 + (int64_t)j * kBlock + s) * G + g) * D) + c8);
-      reinterpret_cast<uint4*>(&v_s[s][0])[c8] = val;
-    }
-    __syncthreads();
-    // logits: thread = key
-    float kreg[D];
-    if (tid < nkeys) {
-      const uint4* kr = reinterpret_cast<const uint4*>(kc + ((s0 + (int64_t)j * kBlock + tid) * G + g) * D);
+  // ---------------- 1. selection ----------------
+  {
+    const int64_t n_cand = (pooled_offset(cu, b) + nb > pooled_cap) ? 0 : nb - 1;
+    const float* ps = pooled + pooled_offset(cu, b) * G + g;
+    TopList<KSEL> list;
+    list.init();
+    for (int64_t j = tid; j < n_cand; j += kAttnThreads) list.insert(ps[j * G], (int32_t)j);
+    const int want = (int)min64(top_k - 1, n_cand);
+    for (int round = 0; round < want; ++round) {
+      float sc = list.sc[0];
+      int32_t id = list.id[0];
 #pragma unroll
-      for (int c8 = 0; c8 < D / 8; ++c8) {
-        const uint4 val = __ldg(kr + c8);
-        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&val);
+      for (int o = 16; o > 0; o >>= 1) {
+        const float s2 = __shfl_xor_sync(0xffffffffu, sc, o);
+        const int32_t i2 = __shfl_xor_sync(0xffffffffu, id, o);
+        if (better(s2, i2, sc, id)) sc = s2, id = i2;
+      }
+      if (lane == 0) sm.ws_s[warp] = sc, sm.ws_i[warp] = id;
+      __syncthreads();
+      float bs = sm.ws_s[0];
+      int32_t bi = sm.ws_i[0];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const float2 f = __bfloat1622float2(hv[x]);
-          kreg[c8 * 8 + 2 * x] = f.x;
-          kreg[c8 * 8 + 2 * x + 1] = f.y;
+      for (int w = 1; w < kAttnWarps; ++w)
+        if (better(sm.ws_s[w], sm.ws_i[w], bs, bi)) bs = sm.ws_s[w], bi = sm.ws_i[w];
+      if (list.id[0] == bi) list.pop();  // ids are unique: exactly one owner pops
+      if (tid == 0) sm.sel[round] = bi;
+      __syncthreads();
+    }
+    if (tid == 0) {
+      // ascending: insertion of the local block (largest id) into sorted picks
+      int n = want;
+      for (int x = 1; x < n; ++x)
+        for (int y = x; y > 0 && sm.sel[y - 1] > sm.sel[y]; --y) {
+          const int32_t t = sm.sel[y];
+          sm.sel[y] = sm.sel[y - 1];
+          sm.sel[y - 1] = t;
         }
-      }
+      sm.sel[n++] = (int32_t)(nb - 1);
+      sm.nsel = n;
+      int32_t* dst = ids_out + ((int64_t)b * G + g) * top_k;
+      for (int r = 0; r < top_k; ++r) dst[r] = r < n ? sm.sel[r] : -1;
     }
-    const int lane = tid & 31, warp = tid >> 5;
-    for (int h = 0; h < hn; ++h) {
-      float sv = -INFINITY;
-      if (tid < nkeys) {
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int c = 0; c < D; c += 2) {
-          a0 = fmaf(q_s[h][c], kreg[c], a0);
-          a1 = fmaf(q_s[h][c + 1], kreg[c + 1], a1);
-        }
-        sv = a0 + a1;
-      }
-      float m = sv;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (lane == 0) red[h][warp] = m;
-      __syncthreads();
-      m = fmaxf(fmaxf(red[h][0], red[h][1]), fmaxf(red[h][2], red[h][3]));
-      const float p = tid < nkeys ? __expf(sv - m) : 0.f;
-      float l = p;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-      __syncthreads();
-      if (lane == 0) red[h][warp] = l;
-      __syncthreads();
-      l = red[h][0] + red[h][1] + red[h][2] + red[h][3];
-      p_s[h][tid] = p / l;
-      if (tid == 0) part_lse[slot * HG + hb + h] = m + logf(l);
-    }
-    __syncthreads();
-    // o[h][c] = sum_s p[h][s] v[s][c]
-    for (int c = tid; c < D; c += blockDim.x) {
-      float acc[MAXHG];
-#pragma unroll
-      for (int h = 0; h < MAXHG; ++h) acc[h] = 0.f;
-      for (int s = 0; s < nkeys; ++s) {
-        const float vv = __bfloat162float(v_s[s][c]);
-#pragma unroll
-        for (int h = 0; h < MAXHG; ++h)
-          if (h < hn) acc[h] = fmaf(p_s[h][s], vv, acc[h]);
-      }
-      for (int h = 0; h < hn; ++h) part_o[(slot * HG + hb + h) * D + c] = __float2half_rn(acc[h]);
-    }
+    if (tid < NT * 8) sm.m_run[tid] = -INFINITY, sm.l_run[tid] = 0.f;
     __syncthreads();
   }
+
+  // ---------------- 2. attention ----------------
+  constexpr int WPR = D / 8;  // 32-bit words per lane per row (permuted reduction axis)
+  const int gq = lane >> 2, tq = lane & 3;
+  const int nsel = sm.nsel;
+  const __nv_bfloat16* kbase = kc + (s0 * G + g) * (int64_t)D;
+  const __nv_bfloat16* vbase = vc + (s0 * G + g) * (int64_t)D;
+  const int64_t row_pitch = (int64_t)G * D;
+
+  // Q^T fragments: head nt*8+gq of this group, this lane's dims
+  uint32_t qw[NT][WPR];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int h = nt * 8 + gq;
+    if (h < HG) {
+      const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)b * G * HG + g * HG + h) * D +
+                                                        tq * (D / 4));
+#pragma unroll
+      for (int i = 0; i < WPR / 4; ++i) {
+        const uint4 v = __ldg(src + i);
+        qw[nt][4 * i] = v.x, qw[nt][4 * i + 1] = v.y, qw[nt][4 * i + 2] = v.z,
+        qw[nt][4 * i + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < WPR; ++i) qw[nt][i] = 0;
+    }
+  }
+
+  auto load_v = [&](int bi, int buf) {
+    const int64_t j = sm.sel[bi];
+    const int nk = (int)min64(kBlock, L - j * kBlock);
+    for (int x = tid; x < kBlock * (D / 8); x += kAttnThreads) {
+      const int s = x / (D / 8), c = x % (D / 8);
+      const __nv_bfloat16* src = vbase + (j * kBlock + (s < nk ? s : 0)) * row_pitch + c * 8;
+      cp_async_16_zfill(&sm.v[buf][v_off<D>(s, c)], src, s < nk);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  float oacc[NT][4];  // O^T fragment: d rows 16*warp + gq (+8), heads nt*8 + 2tq (+1)
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
+
+  if (nsel > 0) load_v(0, 0);
+  for (int bi = 0; bi < nsel; ++bi) {
+    const int buf = bi & 1;
+    const int64_t j = sm.sel[bi];
+    const int nk = (int)min64(kBlock, L - j * kBlock);
+    if (bi + 1 < nsel) load_v(bi + 1, buf ^ 1);
+
+    // ---- S^T (keys x heads) for this warp's 16 keys ----
+    const int k0 = warp * 16 + gq, k1 = k0 + 8;
+    uint32_t w0[WPR], w1[WPR];
+    {
+      const uint4* r0 = reinterpret_cast<const uint4*>(kbase + (j * kBlock + (k0 < nk ? k0 : 0)) *
+                                                                   row_pitch + tq * (D / 4));
+      const uint4* r1 = reinterpret_cast<const uint4*>(kbase + (j * kBlock + (k1 < nk ? k1 : 0)) *
+                                                                   row_pitch + tq * (D / 4));
+#pragma unroll
+      for (int i = 0; i < WPR / 4; ++i) {
+        const uint4 a = __ldg(r0 + i), c = __ldg(r1 + i);
+        w0[4 * i] = a.x, w0[4 * i + 1] = a.y, w0[4 * i + 2] = a.z, w0[4 * i + 3] = a.w;
+        w1[4 * i] = c.x, w1[4 * i + 1] = c.y, w1[4 * i + 2] = c.z, w1[4 * i + 3] = c.w;
+      }
+    }
+    float sacc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_bf16_16816(sacc[nt], w0[2 * kk], w1[2 * kk], w0[2 * kk + 1], w1[2 * kk + 1],
+                       qw[nt][2 * kk], qw[nt][2 * kk + 1]);
+      // log2-domain logits; keys past the end of the sequence are masked
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = (e < 2) ? k0 : k1;
+        sacc[nt][e] = key < nk ? sacc[nt][e] * scale_log2 : -INFINITY;
+      }
+      // per-warp max of heads 2tq, 2tq+1 over its 16 keys
+      float m0 = fmaxf(sacc[nt][0], sacc[nt][2]), m1 = fmaxf(sacc[nt][1], sacc[nt][3]);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      }
+      if (gq == 0) sm.red_m[warp][nt * 8 + 2 * tq] = m0, sm.red_m[warp][nt * 8 + 2 * tq + 1] = m1;
+    }
+    __syncthreads();
+    if (tid < NT * 8) {
+      float bm = sm.red_m[0][tid];
+#pragma unroll
+      for (int w = 1; w < kAttnWarps; ++w) bm = fmaxf(bm, sm.red_m[w][tid]);
+      const float mo = sm.m_run[tid];
+      const float mn = fmaxf(mo, bm);
+      sm.alpha[tid] = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mn);
+      sm.m_run[tid] = mn;
+    }
+    __syncthreads();
+    // ---- P = exp2(S - m) in bf16 (heads x keys), row sums of the rounded values ----
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int h0 = nt * 8 + 2 * tq, h1 = h0 + 1;
+      const float mh0 = sm.m_run[h0], mh1 = sm.m_run[h1];
+      const __nv_bfloat16 p00 = __float2bfloat16_rn(fast_exp2(sacc[nt][0] - mh0));
+      const __nv_bfloat16 p01 = __float2bfloat16_rn(fast_exp2(sacc[nt][1] - mh1));
+      const __nv_bfloat16 p10 = __float2bfloat16_rn(fast_exp2(sacc[nt][2] - mh0));
+      const __nv_bfloat16 p11 = __float2bfloat16_rn(fast_exp2(sacc[nt][3] - mh1));
+      sm.p[h0][k0] = p00;
+      sm.p[h1][k0] = p01;
+      sm.p[h0][k1] = p10;
+      sm.p[h1][k1] = p11;
+      float l0 = __bfloat162float(p00) + __bfloat162float(p10);
+      float l1 = __bfloat162float(p01) + __bfloat162float(p11);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      }
+      if (gq == 0) sm.red_l[warp][h0] = l0, sm.red_l[warp][h1] = l1;
+    }
+    // this block's V tile has landed (the next one may still be in flight)
+    if (bi + 1 < nsel)
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    if (tid < NT * 8) {
+      float ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < kAttnWarps; ++w) ls += sm.red_l[w][tid];
+      sm.l_run[tid] = sm.alpha[tid] * sm.l_run[tid] + ls;
+    }
+    // ---- O^T (d x heads) = alpha * O^T + V^T P^T : warp w owns d rows 16w..16w+15 ----
+    if (warp < D / 16) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float a0 = sm.alpha[nt * 8 + 2 * tq], a1 = sm.alpha[nt * 8 + 2 * tq + 1];
+        oacc[nt][0] *= a0;
+        oacc[nt][1] *= a1;
+        oacc[nt][2] *= a0;
+        oacc[nt][3] *= a1;
+      }
+      const int dchunk = warp * 2 + ((lane >> 3) & 1);  // 16-byte chunk of d
+#pragma unroll
+      for (int kk = 0; kk < kBlock / 16; ++kk) {
+        const int key = kk * 16 + (lane & 7) + ((lane >> 4) << 3);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4_trans(a0, a1, a2, a3, &sm.v[buf][v_off<D>(key, dchunk)]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const __nv_bfloat16* prow = &sm.p[nt * 8 + gq][kk * 16 + 2 * tq];
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(prow);
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(prow + 8);
+          mma_bf16_16816(oacc[nt], a0, a1, a2, a3, b0, b1);
+        }
+      }
+    }
+    __syncthreads();  // p, red_*, alpha and this V buffer are reused next block
+  }
+
+  // ---------------- output: O / l -> bf16 [heads][d] ----------------
+  if (warp < D / 16) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int h0 = nt * 8 + 2 * tq;
+      const int d0 = warp * 16 + gq;
+      sm.o_t[h0][d0] = oacc[nt][0];
+      sm.o_t[h0 + 1][d0] = oacc[nt][1];
+      sm.o_t[h0][d0 + 8] = oacc[nt][2];
+      sm.o_t[h0 + 1][d0 + 8] = oacc[nt][3];
+    }
+  }
+  __syncthreads();
+  for (int x = tid; x < HG * (D / 8); x += kAttnThreads) {
+    const int h = x / (D / 8), c = x % (D / 8);
+    const float inv = sm.l_run[h] > 0.f ? 1.0f / sm.l_run[h] : 0.f;
+    uint4 w;
+    w.x = pack_bf16x2(sm.o_t[h][c * 8 + 0] * inv, sm.o_t[h][c * 8 + 1] * inv);
+    w.y = pack_bf16x2(sm.o_t[h][c * 8 + 2] * inv, sm.o_t[h][c * 8 + 3] * inv);
+    w.z = pack_bf16x2(sm.o_t[h][c * 8 + 4] * inv, sm.o_t[h][c * 8 + 5] * inv);
+    w.w = pack_bf16x2(sm.o_t[h][c * 8 + 6] * inv, sm.o_t[h][c * 8 + 7] * inv);
+    reinterpret_cast<uint4*>(out + ((int64_t)b * G * HG + g * HG + h) * D)[c] = w;
+  }
+}
+
+template <int D, int NT, int KSEL>
+cudaError_t launch_attend(const DecodeLaunch& p, cudaStream_t s) {
+  auto kern = decode_attend_kernel<D, NT, KSEL>;
+  const int smem = (int)sizeof(AttnSmem<D, NT>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)p.G, (unsigned)p.B);
+  kern<<<grid, kAttnThreads, smem, s>>>(
+      static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k_cache),
+      static_cast<const __nv_bfloat16*>(p.v_cache), p.cu_seqlens, p.pooled, p.pooled_cap, p.G,
+      p.H / p.G, p.top_k, p.scale * 1.4426950408889634f, p.ids,
+      static_cast<__nv_bfloat16*>(p.out));
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_attend_d(const DecodeLaunch& p, cudaStream_t s) {
+  const int HG = p.H / p.G;
+  if (HG <= 8) {
+    if (p.top_k <= 16) return launch_attend<D, 1, 15>(p, s);
+    return launch_attend<D, 1, 31>(p, s);
+  }
+  if (HG <= 16) {
+    if (p.top_k <= 16) return launch_attend<D, 2, 15>(p, s);
+    return launch_attend<D, 2, 31>(p, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -341,42 +497,13 @@ cudaError_t launch_decode(const DecodeLaunch& p, cudaStream_t s, int* launches) 
     decode_index_kernel<64><<<gi, kIdxWarps * 32, 0, s>>>(qi, ki, p.cu_seqlens, p.G, p.pooled,
                                                            p.pooled_cap, p.err);
   ++*launches;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   mark_ev(p, 1, s);
-  dim3 gt((unsigned)p.G, (unsigned)p.B);
-  if (p.top_k <= 16)
-    decode_topk_kernel<15><<<gt, 256, 0, s>>>(p.pooled, p.cu_seqlens, p.G, p.top_k, p.pooled_cap,
-                                              p.ids);
-  else
-    decode_topk_kernel<31><<<gt, 256, 0, s>>>(p.pooled, p.cu_seqlens, p.G, p.top_k, p.pooled_cap,
-                                              p.ids);
+  e = p.d == 128 ? launch_attend_d<128>(p, s) : launch_attend_d<64>(p, s);
   ++*launches;
   mark_ev(p, 2, s);
-  dim3 ga((unsigned)p.top_k, (unsigned)p.G, (unsigned)p.B);
-  const auto* q = static_cast<const __nv_bfloat16*>(p.q);
-  const auto* kc = static_cast<const __nv_bfloat16*>(p.k_cache);
-  const auto* vc = static_cast<const __nv_bfloat16*>(p.v_cache);
-  if (p.d == 128)
-    decode_attn_kernel<128><<<ga, 128, 0, s>>>(q, kc, vc, p.cu_seqlens, p.ids, p.H, p.G, p.top_k,
-                                               p.scale, p.part_o, p.part_lse, p.err);
-  else
-    decode_attn_kernel<64><<<ga, 128, 0, s>>>(q, kc, vc, p.cu_seqlens, p.ids, p.H, p.G, p.top_k,
-                                              p.scale, p.part_o, p.part_lse, p.err);
-  ++*launches;
-  mark_ev(p, 3, s);
-  MergeLaunch m{};
-  m.part_o = p.part_o;
-  m.part_lse = p.part_lse;
-  m.ids = p.ids;
-  m.rows = p.B;
-  m.H = p.H;
-  m.G = p.G;
-  m.d = p.d;
-  m.top_k = p.top_k;
-  m.out = p.out;
-  cudaError_t e = launch_merge(m, s);
-  ++*launches;
-  mark_ev(p, 4, s);
-  return e != cudaSuccess ? e : cudaGetLastError();
+  return e;
 }
 
 }  // namespace msa

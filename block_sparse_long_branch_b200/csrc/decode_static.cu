@@ -62,7 +62,7 @@ extern "C" msa_status_t msa_decode_static(const msa_config_t* cfg, const void* q
                                           int32_t* ids_out, int32_t check_device_error,
                                           msa_stream_t stream) {
   if (total_len < 1 || max_seqlen > total_len || B < 1 || B > total_len)
-    return MSA_ERR_INVALID_ARG;
+    return MSA_ERR_INVALID_ARG;  // total_len must be the sum of the sequence lengths
   size_t need = 0;
   msa_status_t st = msa_workspace_size(cfg, MSA_OP_DECODE, total_len, B, &need);
   if (st != MSA_OK) return st;

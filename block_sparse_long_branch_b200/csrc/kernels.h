@@ -93,8 +93,6 @@ struct DecodeLaunch {
   int32_t* ids;    // [B][G][top_k]
   float* pooled;   // [pooled_cap][G]
   int64_t pooled_cap;
-  __half* part_o;  // [B][G][top_k][H/G][d]
-  float* part_lse; // [B][G][top_k][H/G]
   uint32_t* err;
   int num_sms;
   void* const* events;  // optional phase events (msa_set_phase_events)

@@ -91,9 +91,8 @@ typedef enum {
  * Workspace bytes needed by `op`.
  *   SELECT_TOPK, BLOCK_QUERY_LISTS, PREFILL: n_tokens = N, batch ignored.
  *     For PREFILL this is the size that processes all N queries in one pass;
- *     msa_prefill also accepts any workspace of at least
- *     msa_workspace_size(cfg, PREFILL, 128*ceil(min(N, 16384)/128)...) -- see
- *     msa_prefill_min_workspace -- and then walks the query axis in chunks.
+ *     msa_prefill also accepts less (down to msa_prefill_min_workspace) and
+ *     then walks the query axis in chunks (msa_prefill_chunk_tokens).
  *   DECODE: n_tokens = total cache rows (sum of sequence lengths), batch = B.
  * Host-only; returns MSA_ERR_INVALID_ARG / MSA_ERR_UNSUPPORTED like the op.
  */
@@ -103,6 +102,14 @@ MSA_API msa_status_t msa_workspace_size(const msa_config_t* cfg, msa_op_t op, in
 /* Smallest workspace msa_prefill accepts for N tokens (it then processes the
  * query axis in chunks of at least 128 tokens).  Host-only. */
 MSA_API msa_status_t msa_prefill_min_workspace(const msa_config_t* cfg, int64_t N, size_t* bytes);
+
+/* Query rows per chunk msa_prefill uses with ws_bytes of workspace: N when
+ * the whole axis fits, else the largest multiple of 128 that fits.
+ * ids_returned: non-zero when msa_prefill is given ids_out (the workspace then
+ * holds no ids).  MSA_ERR_WORKSPACE if not even 128 rows fit.  Host-only. */
+MSA_API msa_status_t msa_prefill_chunk_tokens(const msa_config_t* cfg, int64_t N,
+                                              size_t ws_bytes, int32_t ids_returned,
+                                              int64_t* chunk);
 
 /*
  * Index Branch scores, pooled per block (guide, section "2段階構造の中身": token
@@ -199,9 +206,9 @@ MSA_API msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const vo
  *     and return the device error status (as msa_get_device_error would).
  * Scratch lives in a 16 MiB array compiled into this library, held on every
  * GPU that loads the library until the process exits.  A call that needs more
- * (msa_workspace_size(cfg, MSA_OP_DECODE, total_len, B) > 16 MiB; e.g. more
- * than about 28 sequences at H=64, G=8, d=128, k=16) returns
- * MSA_ERR_WORKSPACE and launches nothing.  The first call on a device looks
+ * (msa_workspace_size(cfg, MSA_OP_DECODE, total_len, B) > 16 MiB; with G=8
+ * that is about 64M cached tokens in total) returns MSA_ERR_WORKSPACE and
+ * launches nothing.  The first call on a device looks
  * up the array's address (cudaGetSymbolAddress): make it before any stream
  * capture.  All calls share the array, so calls that overlap on the GPU race;
  * the caller serialises them.  Allocates nothing: no cudaMalloc / cudaFree.
@@ -236,8 +243,8 @@ MSA_API int32_t msa_last_launch_count(void);
  *   prefill chunk c: events[5c+0] before the index kernel, [5c+1] after it,
  *     [5c+2] after the query-list kernels, [5c+3] after the Main Branch
  *     kernel, [5c+4] after the merge kernel (only while 5c+4 < count);
- *   decode: [0] before the index scan, [1] after it, [2] after the top-k
- *     kernel, [3] after the attention kernel, [4] after the merge kernel.
+ *   decode: [0] before the index scan, [1] after it, [2] after the fused
+ *     top-k + attention kernel.
  * Pass NULL to stop recording.  The events are not owned by the library.
  */
 MSA_API msa_status_t msa_set_phase_events(void* const* events, int32_t count);

@@ -35,6 +35,7 @@ __all__ = [
     "DecodeShape",
     "PREFILL_CONFIGS",
     "DECODE_CONFIG",
+    "DECODE_SMALL",
     "make_prefill_inputs",
     "make_decode_inputs",
     "sample_rows",
@@ -119,6 +120,15 @@ DECODE_CONFIG = DecodeShape(
     H=64, G=8, d=128, d_idx=128, top_k=16,
     needles_per_seq=(16,) * 16 + (64,),
     seed=SEED_BASE + 3,
+)
+
+# Smaller decode case (two 256K caches, 2.2 GB) used to size profiler captures.
+DECODE_SMALL = DecodeShape(
+    "decode_2x256k",
+    seq_lens=(262144,) * 2,
+    H=64, G=8, d=128, d_idx=128, top_k=16,
+    needles_per_seq=(16,) * 2,
+    seed=SEED_BASE + 6,
 )
 
 # Elements drawn per randn call: bounds the fp32 temporary on the device.

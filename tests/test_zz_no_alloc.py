@@ -62,11 +62,10 @@ def test_static_decode_matches_workspace_decode_twice(setup):
 
 def test_static_decode_rejects_sizes_beyond_its_array(setup):
     msa, lib, s, inp, cfg, cu, ref_out, ref_ids = setup
-    big = msa.config(64, 8, 128, 128, top_k=16)
-    # 64 sequences of this head layout need far more than the fixed array holds
-    st = lib.msa_decode_static(ctypes.byref(big), _ptr(inp["q"]), _ptr(inp["q_idx"]),
+    # 2^32 cached tokens need about 1 GiB of block scores: far beyond the fixed array
+    st = lib.msa_decode_static(ctypes.byref(cfg), _ptr(inp["q"]), _ptr(inp["q_idx"]),
                                _ptr(inp["k_cache"]), _ptr(inp["v_cache"]),
-                               _ptr(inp["k_idx_cache"]), _ptr(cu), 64, 4096, 1 << 20,
+                               _ptr(inp["k_idx_cache"]), _ptr(cu), s.B, max(s.seq_lens), 1 << 32,
                                _ptr(ref_out), None, 0, None)
     assert st == 3  # MSA_ERR_WORKSPACE, nothing launched
     assert np.isfinite(ref_out.float().cpu().numpy()).all()
