@@ -444,9 +444,9 @@ def run_ours(args, rank, world, local):
                 f"({'hbm_gbs' if dk['unit'] == 'GB/s' else tc_name})"}
 
     # ---- end to end through the public API with host buffers ----
-    e2e = run_e2e(args, msa, cfg, shape, inp if do_prefill else None,
-                  ws if do_prefill else None, dev, dec, dcfg if dec is not None else None,
-                  dws if dec is not None else None, world)
+    e2e = None if args.no_e2e else run_e2e(
+        args, msa, cfg, shape, inp if do_prefill else None, ws if do_prefill else None, dev, dec,
+        dcfg if dec is not None else None, dws if dec is not None else None, world)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -629,6 +629,8 @@ def main(argv=None):
                     help="time only the decode step (profiling)")
     ap.add_argument("--decode-workload", choices=("full", "small"), default="full")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer end-to-end leg (large workloads)")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--ws-gb", type=float, default=96.0,

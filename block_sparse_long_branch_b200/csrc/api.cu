@@ -14,7 +14,7 @@ namespace {
 
 constexpr int kBlock = 128;
 constexpr size_t kHeader = 256;  // device error word + reserved
-constexpr int kUnitTiles = 8;    // Main Branch tiles per work unit
+constexpr int kUnitTiles = 16;   // Main Branch tiles per work unit
 
 thread_local int g_launches = 0;
 thread_local void* const* g_events = nullptr;
@@ -87,7 +87,7 @@ PrefillLayout prefill_layout(const msa_config_t* c, int64_t rows, int64_t nb, bo
   L.unit_ptr = off;
   off += align256((lists + 1) * 4);
   L.unit_list = off;
-  off += align256(max_units * 4);
+  off += align256(max_units * 16);
   L.csr = off;
   off += csr_scratch_bytes(rows, (int32_t)G, (int32_t)k, nb);
   L.part_o = off;
@@ -295,7 +295,7 @@ msa_status_t msa_build_block_query_lists(const msa_config_t* cfg, const int32_t*
   p.scratch = at<void>(ws, kHeader);
   p.err = at<uint32_t>(ws, 0);
   p.unit_ptr = nullptr;
-  p.unit_list = nullptr;
+  p.unit_desc = nullptr;
   int launches = 0;
   st = cuda_status(launch_csr(p, s, &launches));
   g_launches = launches;
@@ -361,7 +361,7 @@ msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, 
     cp.scratch = at<void>(ws, L.csr);
     cp.err = err;
     cp.unit_ptr = at<int32_t>(ws, L.unit_ptr);
-    cp.unit_list = at<int32_t>(ws, L.unit_list);
+    cp.unit_desc = at<int4>(ws, L.unit_list);
     cp.tile_tokens = main_tile_tokens(H, G);
     cp.unit_tiles = kUnitTiles;
     if (launch_csr(cp, s, &launches) != cudaSuccess) return MSA_ERR_CUDA;
@@ -383,8 +383,7 @@ msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, 
     mp.row_ptr = cp.row_ptr;
     mp.entries = cp.entries;
     mp.unit_ptr = cp.unit_ptr;
-    mp.unit_list = cp.unit_list;
-    mp.unit_tiles = kUnitTiles;
+    mp.unit_desc = cp.unit_desc;
     mp.part_o = at<__half>(ws, L.part_o);
     mp.part_lse = at<float>(ws, L.part_lse);
     mp.err = err;

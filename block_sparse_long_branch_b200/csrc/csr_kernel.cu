@@ -186,11 +186,18 @@ __global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restri
   }
 }
 
-__global__ void unit_fill_kernel(const int32_t* __restrict__ unit_ptr, int64_t n_lists,
-                                 int32_t* __restrict__ unit_list) {
+// Work units of the Main Branch: list x = g*nb + j is cut into runs of at
+// most `per_unit` entries; unit u gets {g, j, first entry, end entry}.
+__global__ void unit_fill_kernel(const int32_t* __restrict__ unit_ptr,
+                                 const int32_t* __restrict__ row_ptr, int64_t n_lists, int64_t nb,
+                                 int32_t per_unit, int4* __restrict__ unit_desc) {
   const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (x < n_lists)
-    for (int32_t u = unit_ptr[x]; u < unit_ptr[x + 1]; ++u) unit_list[u] = (int32_t)x;
+  if (x >= n_lists) return;
+  const int32_t beg = row_ptr[x], end = row_ptr[x + 1];
+  const int g = (int)(x / nb), j = (int)(x - (int64_t)g * nb);
+  int32_t e0 = beg;
+  for (int32_t u = unit_ptr[x]; u < unit_ptr[x + 1]; ++u, e0 += per_unit)
+    unit_desc[u] = make_int4(g, j, e0, min(end, e0 + per_unit));
 }
 
 __global__ void unit_count_kernel(const int32_t* __restrict__ row_ptr, int64_t n_lists,
@@ -257,8 +264,8 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
     // unit_ptr[n_lists] = total units: scan n_lists+1 values with a trailing 0
     if ((e = cudaMemsetAsync(p.unit_ptr + n_lists, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
     if ((e = exclusive_scan(p.unit_ptr, n_lists + 1, tmp2, s, launches)) != cudaSuccess) return e;
-    unit_fill_kernel<<<(unsigned)((n_lists + 255) / 256), 256, 0, s>>>(p.unit_ptr, n_lists,
-                                                                      p.unit_list);
+    unit_fill_kernel<<<(unsigned)((n_lists + 255) / 256), 256, 0, s>>>(
+        p.unit_ptr, p.row_ptr, n_lists, p.nb, p.tile_tokens * p.unit_tiles, p.unit_desc);
     ++*launches;
   }
   return cudaGetLastError();

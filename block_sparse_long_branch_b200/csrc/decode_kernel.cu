@@ -300,28 +300,36 @@ __global__ void __launch_bounds__(kAttnThreads)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
 
-  if (nsel > 0) load_v(0, 0);
+  // this warp's 16 key rows of a block, lanes reading 16 contiguous bytes each
+  uint32_t w0[WPR], w1[WPR];
+  auto load_k = [&](int bi) {
+    const int64_t jj = sm.sel[bi];
+    const int nkk = (int)min64(kBlock, L - jj * kBlock);
+    const int r0i = warp * 16 + gq, r1i = r0i + 8;
+    const uint4* r0 = reinterpret_cast<const uint4*>(
+        kbase + (jj * kBlock + (r0i < nkk ? r0i : 0)) * row_pitch + tq * (D / 4));
+    const uint4* r1 = reinterpret_cast<const uint4*>(
+        kbase + (jj * kBlock + (r1i < nkk ? r1i : 0)) * row_pitch + tq * (D / 4));
+#pragma unroll
+    for (int i = 0; i < WPR / 4; ++i) {
+      const uint4 a4 = __ldg(r0 + i), c4 = __ldg(r1 + i);
+      w0[4 * i] = a4.x, w0[4 * i + 1] = a4.y, w0[4 * i + 2] = a4.z, w0[4 * i + 3] = a4.w;
+      w1[4 * i] = c4.x, w1[4 * i + 1] = c4.y, w1[4 * i + 2] = c4.z, w1[4 * i + 3] = c4.w;
+    }
+  };
+
+  if (nsel > 0) {
+    load_v(0, 0);
+    load_k(0);
+  }
   for (int bi = 0; bi < nsel; ++bi) {
     const int buf = bi & 1;
     const int64_t j = sm.sel[bi];
     const int nk = (int)min64(kBlock, L - j * kBlock);
     if (bi + 1 < nsel) load_v(bi + 1, buf ^ 1);
 
-    // ---- S^T (keys x heads) for this warp's 16 keys ----
+    // ---- S^T (keys x heads) for this warp's 16 keys (K rows loaded one block ahead) ----
     const int k0 = warp * 16 + gq, k1 = k0 + 8;
-    uint32_t w0[WPR], w1[WPR];
-    {
-      const uint4* r0 = reinterpret_cast<const uint4*>(kbase + (j * kBlock + (k0 < nk ? k0 : 0)) *
-                                                                   row_pitch + tq * (D / 4));
-      const uint4* r1 = reinterpret_cast<const uint4*>(kbase + (j * kBlock + (k1 < nk ? k1 : 0)) *
-                                                                   row_pitch + tq * (D / 4));
-#pragma unroll
-      for (int i = 0; i < WPR / 4; ++i) {
-        const uint4 a = __ldg(r0 + i), c = __ldg(r1 + i);
-        w0[4 * i] = a.x, w0[4 * i + 1] = a.y, w0[4 * i + 2] = a.z, w0[4 * i + 3] = a.w;
-        w1[4 * i] = c.x, w1[4 * i + 1] = c.y, w1[4 * i + 2] = c.z, w1[4 * i + 3] = c.w;
-      }
-    }
     float sacc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -345,6 +353,7 @@ __global__ void __launch_bounds__(kAttnThreads)
       }
       if (gq == 0) sm.red_m[warp][nt * 8 + 2 * tq] = m0, sm.red_m[warp][nt * 8 + 2 * tq + 1] = m1;
     }
+    if (bi + 1 < nsel) load_k(bi + 1);  // in flight during the softmax and PV of this block
     __syncthreads();
     if (tid < NT * 8) {
       float bm = sm.red_m[0][tid];

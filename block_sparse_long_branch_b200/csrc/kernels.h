@@ -37,7 +37,7 @@ struct CsrLaunch {
   // optional: main-branch work units (tiles of `tile_tokens` queries, at most
   // `unit_tiles` tiles per unit) per list, exclusive prefix in unit_ptr[G*nb+1]
   int32_t* unit_ptr;
-  int32_t* unit_list;  // [max units]: list index of every unit
+  int4* unit_desc;  // [max units]: {g, j, first entry, end entry} of every unit
   int32_t tile_tokens, unit_tiles;
 };
 size_t csr_scratch_bytes(int64_t rows, int32_t G, int32_t top_k, int64_t nb);
@@ -56,8 +56,7 @@ struct MainLaunch {
   const int32_t* row_ptr;   // [G*nb+1]
   const int32_t* entries;
   const int32_t* unit_ptr;   // [G*nb+1]
-  const int32_t* unit_list;  // [units]
-  int32_t unit_tiles;
+  const int4* unit_desc;     // [units] {g, j, first entry, end entry}
   __half* part_o;   // [rows][G][top_k][H/G][d] fp16
   float* part_lse;  // [rows][G][top_k][H/G] fp32
   uint32_t* err;

@@ -61,8 +61,7 @@ struct MainArgs {
   const int32_t* row_ptr;
   const int32_t* entries;
   const int32_t* unit_ptr;
-  const int32_t* unit_list;
-  int32_t per_unit;
+  const int4* unit_desc;
   __half* part_o;
   float* part_lse;
   uint32_t* err;
@@ -73,18 +72,17 @@ struct MUnit {
 };
 
 __device__ __forceinline__ MUnit decode_unit(const MainArgs& a, int u) {
+  const int4 d = __ldg(a.unit_desc + u);  // {g, j, first entry, end entry}
   MUnit m;
-  const int x = __ldg(a.unit_list + u);
-  const int c = u - __ldg(a.unit_ptr + x);
-  m.g = (int)(x / a.nb);
-  m.j = (int)(x - (int64_t)m.g * a.nb);
-  const int beg = __ldg(a.row_ptr + x), end = __ldg(a.row_ptr + x + 1);
-  m.e0 = beg + c * a.per_unit;
-  m.e1 = min(end, m.e0 + a.per_unit);
+  m.g = d.x;
+  m.j = d.y;
+  m.e0 = d.z;
+  m.e1 = d.w;
   m.ntiles = (m.e1 - m.e0 + a.TT - 1) / a.TT;
   return m;
 }
 
+// position of a tile in this CTA's sequence of units
 struct TilePos {
   int u, i;
   MUnit m;
@@ -456,32 +454,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      // pass 1: row max, streaming S from TMEM in 64-column halves
+      // pass 1: row max over the 128 scores (one TMEM round trip)
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t sv[2][32];
-        tmem_ld_32x32b_x32(lane_addr + s_col + hf * 64, sv[0]);
-        tmem_ld_32x32b_x32(lane_addr + s_col + hf * 64 + 32, sv[1]);
+      {
+        uint32_t sv[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(lane_addr + s_col + c * 32, sv[c]);
         tmem_wait();
-        reg_fence(sv[0]);
-        reg_fence(sv[1]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_fence(sv[c]);
         if (unmasked) {
-          float x0 = mx, x1 = -INFINITY;
+          float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 4; c += 2)
 #pragma unroll
-            for (int x = 0; x < 32; x += 4) {
+            for (int x = 0; x < 32; x += 2) {
               x0 = max3f(x0, __uint_as_float(sv[c][x]), __uint_as_float(sv[c][x + 1]));
-              x1 = max3f(x1, __uint_as_float(sv[c][x + 2]), __uint_as_float(sv[c][x + 3]));
+              x1 = max3f(x1, __uint_as_float(sv[c + 1][x]), __uint_as_float(sv[c + 1][x + 1]));
             }
-          mx = fmaxf(x0, x1);
+          mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
         } else {
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int x = 0; x < 32; ++x)
-              if (hf * 64 + c * 32 + x <= lim) mx = fmaxf(mx, __uint_as_float(sv[c][x]));
+              if (c * 32 + x <= lim) mx = fmaxf(mx, __uint_as_float(sv[c][x]));
         }
       }
       if (!(row_valid && good) || !(mx > -INFINITY)) mx = 0.f;
@@ -539,18 +536,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t inv2 = f2_pack(inv, inv);
       // same 128-byte-swizzled layout as P: conflict-free writes, and the TMA
       // store below undoes the swizzle on its way to global memory
-#pragma unroll 1
-      for (int hf = 0; hf < D / 64; ++hf) {
-        uint32_t o[2][32];
-        tmem_ld_32x32b_x32(lane_addr + o_col + hf * 64, o[0]);
-        tmem_ld_32x32b_x32(lane_addr + o_col + hf * 64 + 32, o[1]);
-        tmem_wait();
-        reg_fence(o[0]);
-        reg_fence(o[1]);
+      {
+        uint32_t o[D / 32][32];
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
+        for (int c = 0; c < D / 32; ++c) tmem_ld_32x32b_x32(lane_addr + o_col + c * 32, o[c]);
+        tmem_wait();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) reg_fence(o[c]);
+#pragma unroll
+        for (int c16 = 0; c16 < D / 8; ++c16) {
           uint4 w;
-          const uint32_t* src = &o[c8 >> 2][(c8 & 3) * 8];
+          const uint32_t* src = &o[c16 >> 2][(c16 & 3) * 8];
 #pragma unroll
           for (int x2 = 0; x2 < 4; ++x2) {
             float f0, f1;
@@ -559,7 +555,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       f0, f1);
             (&w.x)[x2] = pack_half2(f0, f1);
           }
-          *reinterpret_cast<uint4*>(pbuf + hf * kRows * 128 + sw128_offset(row, c8)) = w;
+          *reinterpret_cast<uint4*>(pbuf + (c16 >> 3) * kRows * 128 + sw128_offset(row, c16 & 7)) =
+              w;
         }
       }
       tc_fence_before();
@@ -622,8 +619,7 @@ cudaError_t launch_main_impl(const MainLaunch& p, cudaStream_t s) {
   a.row_ptr = p.row_ptr;
   a.entries = p.entries;
   a.unit_ptr = p.unit_ptr;
-  a.unit_list = p.unit_list;
-  a.per_unit = a.TT * p.unit_tiles;
+  a.unit_desc = p.unit_desc;
   a.part_o = p.part_o;
   a.part_lse = p.part_lse;
   a.err = p.err;
