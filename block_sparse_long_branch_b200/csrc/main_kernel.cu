@@ -17,11 +17,13 @@
 // ln rowsum) goes to slot (t, g, r, head); the merge kernel combines the <= k
 // slots of a query with log-sum-exp weights.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over units):
-//   warp 0     producer: TMA of K_j / V_j (3-D map: one group's rows), and a
-//              TMA gather of each hitting token's H/G contiguous query rows;
-//   warp 1     MMA issuer (one thread), S of tile i+1 issued before P V of
-//              tile i so the tensor core never waits on the softmax;
+// Warp roles (352 threads, one CTA per SM, persistent over units):
+//   warp 0     Q producer: a TMA gather of each hitting token's H/G
+//              contiguous query rows into a 3-stage ring;
+//   warp 10    K/V loader: TMA of K_j / V_j (3-D map: one group's rows) once
+//              per unit, plus an L2 prefetch of the next unit's blocks;
+//   warp 1     MMA issuer (one thread): issues whichever of the next S or the
+//              oldest pending PV has its inputs ready;
 //   warps 2-9  two softmax + epilogue warpgroups taking alternate tiles;
 //              thread <-> TMEM lane <-> tile row.  The epilogue stages the
 //              fp16 partials in the tile's (consumed) P buffer and writes each
@@ -35,7 +37,8 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 320;  // producer, MMA, 2 softmax warpgroups
+constexpr int kThreads = 352;  // Q producer, MMA, 2 softmax warpgroups, K/V loader
+constexpr int kKVWarp = 10;
 constexpr int kRows = 128;
 constexpr int kKeys = 128;
 constexpr int kQStages = 3;
@@ -231,40 +234,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int slot = 1 << a.log2slot;
 
   if (warp == 0) {
-    // ---------------- producer ----------------
+    // ---------------- Q gather producer ----------------
     if (lane == 0) {
       tma_prefetch_desc(&map_q);
-      tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v);
       tma_prefetch_desc(&map_o);
     }
     int qs = 0;
-    uint32_t qph = 0, kph = 0, vph = 0;
-    // last issued phase per barrier, for draining after an abort
-    int q_issued = 0;
+    uint32_t qph = 0;
+    // last issued phase per stage, for draining after an abort
     uint32_t q_last[kQStages] = {0, 0, 0};
     bool q_any[kQStages] = {false, false, false};
-    bool k_any = false, v_any = false;
-    uint32_t k_last = 0, v_last = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const MUnit m = decode_unit(a, u);
-      if (lane == 0) {
-        ok = mbar_wait(&bar_k_empty, kph ^ 1, abort_flag, a.err, kDevTimeoutMma);
-        if (ok) {
-          mbar_arrive_expect_tx(&bar_k_full, Cfg::kKVBytes);
-#pragma unroll
-          for (int ri = 0; ri < Cfg::kRegions; ++ri)
-            tma_load_3d(sK + ri * kKeys * 128, &map_k, &bar_k_full, ri * 64, m.g, m.j * kKeys);
-          k_any = true;
-          k_last = kph;
-        }
-      }
-      kph ^= 1;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
       for (int i = 0; i < m.ntiles && ok; ++i) {
         const int eb = m.e0 + i * a.TT;
         const int nt = min(a.TT, m.e1 - eb);
+        // the entry loads overlap the wait for a free stage
+        int64_t t = 0;
+        int r = 0;
+        if (lane < nt) read_entry(a, eb + lane, t, r);
         if (lane == 0) {
           ok = mbar_wait(&bar_q_empty[qs], qph ^ 1, abort_flag, a.err, kDevTimeoutMma);
           if (ok) {
@@ -276,9 +265,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane < nt) {
-          int64_t t;
-          int r;
-          read_entry(a, eb + lane, t, r);
           const int32_t qrow = (int32_t)(t * a.H + (int64_t)m.g * a.HG);
           uint8_t* dst = sQ + qs * Cfg::kQBytes + lane * slot * 128;
 #pragma unroll
@@ -286,125 +272,168 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(dst + ri * kRows * 128, &map_q, &bar_q_full[qs], ri * 64, qrow);
         }
         __syncwarp();
-        ++q_issued;
         if (++qs == kQStages) qs = 0, qph ^= 1;
-        if (i == 0) {
-          if (lane == 0) {
-            ok = mbar_wait(&bar_v_empty, vph ^ 1, abort_flag, a.err, kDevTimeoutMma);
-            if (ok) {
-              mbar_arrive_expect_tx(&bar_v_full, Cfg::kKVBytes);
-#pragma unroll
-              for (int ri = 0; ri < Cfg::kRegions; ++ri)
-                tma_load_3d(sV + ri * kKeys * 128, &map_v, &bar_v_full, ri * 64, m.g, m.j * kKeys);
-              v_any = true;
-              v_last = vph;
-            }
-          }
-          vph ^= 1;
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-        }
       }
     }
     if (lane == 0 && *abort_flag) {
       volatile int no_abort = 0;
       for (int s = 0; s < kQStages; ++s)
         if (q_any[s]) mbar_wait(&bar_q_full[s], q_last[s], &no_abort, nullptr, 0);
-      if (k_any) mbar_wait(&bar_k_full, k_last, &no_abort, nullptr, 0);
-      if (v_any) mbar_wait(&bar_v_full, v_last, &no_abort, nullptr, 0);
     }
-    (void)q_issued;
+  } else if (warp == kKVWarp) {
+    // ---------------- K/V loader ----------------
+    // K_j and V_j of each unit into their single buffers, and an L2 prefetch
+    // of the next unit's blocks so that those loads hit L2.
+    if (lane == 0) {
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      uint32_t kph = 0, vph = 0;
+      bool k_any = false, v_any = false;
+      uint32_t k_last = 0, v_last = 0;
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const MUnit m = decode_unit(a, u);
+        if (u + (int)gridDim.x < n_units) {
+          const MUnit nx = decode_unit(a, u + gridDim.x);
+#pragma unroll
+          for (int ri = 0; ri < Cfg::kRegions; ++ri) {
+            tma_prefetch_l2_3d(&map_k, ri * 64, nx.g, nx.j * kKeys);
+            tma_prefetch_l2_3d(&map_v, ri * 64, nx.g, nx.j * kKeys);
+          }
+        }
+        if (!mbar_wait(&bar_k_empty, kph ^ 1, abort_flag, a.err, kDevTimeoutMma)) break;
+        mbar_arrive_expect_tx(&bar_k_full, Cfg::kKVBytes);
+#pragma unroll
+        for (int ri = 0; ri < Cfg::kRegions; ++ri)
+          tma_load_3d(sK + ri * kKeys * 128, &map_k, &bar_k_full, ri * 64, m.g, m.j * kKeys);
+        k_any = true;
+        k_last = kph;
+        kph ^= 1;
+        if (!mbar_wait(&bar_v_empty, vph ^ 1, abort_flag, a.err, kDevTimeoutMma)) break;
+        mbar_arrive_expect_tx(&bar_v_full, Cfg::kKVBytes);
+#pragma unroll
+        for (int ri = 0; ri < Cfg::kRegions; ++ri)
+          tma_load_3d(sV + ri * kKeys * 128, &map_v, &bar_v_full, ri * 64, m.g, m.j * kKeys);
+        v_any = true;
+        v_last = vph;
+        vph ^= 1;
+      }
+      if (*abort_flag) {
+        volatile int no_abort = 0;
+        if (k_any) mbar_wait(&bar_k_full, k_last, &no_abort, nullptr, 0);
+        if (v_any) mbar_wait(&bar_v_full, v_last, &no_abort, nullptr, 0);
+      }
+    }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // One thread keeps two cursors over the same tile sequence, S ahead of
+    // PV, and issues whichever MMA has its inputs ready, so that a late Q
+    // tile or K block does not hold back the PV of a finished softmax.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kKeys, false, false);
       constexpr uint32_t idesc_o = idesc_bf16(kRows, D, false, true);
-      int qs = 0, sb = 0, pb = 0, ob = 0;
+      TilePos sc = first_tile(a, n_units), pc = sc;
+      int qs = 0, sb = 0, pb = 0;
       uint32_t qph = 0, kph = 0, vph = 0;
-      uint32_t sph[2] = {0, 0}, pph[2] = {0, 0}, oph[2] = {0, 0};
-      bool ok = true;
-      bool has_prev = false, prev_first = false, prev_last = false;
+      uint32_t sph[2] = {0, 0}, pph[2] = {0, 0};
+      bool k_ready = false, v_ready = false;
+      int64_t s_count = 0, pv_count = 0;
       bool committed = false;
       uint64_t* last_bar = nullptr;
       uint32_t last_par = 0;
-
-      auto issue_pv = [&](bool first, bool last) -> bool {
-        if (!mbar_wait(&bar_p_full[pb], pph[pb], abort_flag, a.err, kDevTimeoutConsumer)) return false;
-        if (!mbar_wait(&bar_o_empty[ob], oph[ob] ^ 1, abort_flag, a.err, kDevTimeoutConsumer))
-          return false;
-        if (first) {
-          if (!mbar_wait(&bar_v_full, vph, abort_flag, a.err, kDevTimeoutLoad)) return false;
-          vph ^= 1;
-        }
-        tc_fence_after();
-        const uint32_t p_base = smem_u32(sP + pb * Cfg::kPBytes);
-        const uint32_t v_base = smem_u32(sV);
-        const uint32_t d_tm = tmem + 256 + ob * 128;
+      uint64_t idle_since = 0;
+      bool idle = false;
+      const uint32_t k_base = smem_u32(sK);
+      const uint32_t v_base = smem_u32(sV);
+      while (pc.more) {
+        bool progress = false;
+        // ---- S = Q K^T for the next tile ----
+        if (sc.more) {
+          bool ready = true;
+          if (sc.i == 0 && !k_ready) {
+            ready = mbar_probe(&bar_k_full, kph);
+            if (ready) kph ^= 1, k_ready = true;
+          }
+          ready = ready && mbar_probe(&bar_q_full[qs], qph) &&
+                  mbar_probe(&bar_s_empty[sb], sph[sb] ^ 1);
+          if (ready) {
+            tc_fence_after();
+            const uint32_t q_base = smem_u32(sQ + qs * Cfg::kQBytes);
+            const uint32_t d_tm = tmem + sb * 128;
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint64_t ad =
-              smem_desc_sw128(p_base + (kk >> 2) * kRows * 128 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(v_base + kk * 16 * 128, kKeys * 128, 1024);
-          umma_bf16(d_tm, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&bar_p_empty[pb]);
-        umma_commit(&bar_o_full[ob]);
-        if (last) umma_commit(&bar_v_empty);
-        committed = true;
-        last_bar = &bar_o_full[ob];
-        last_par = oph[ob];
-        pph[pb] ^= 1;
-        pb ^= 1;
-        oph[ob] ^= 1;
-        ob ^= 1;
-        return true;
-      };
-
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const MUnit m = decode_unit(a, u);
-        for (int i = 0; i < m.ntiles; ++i) {
-          if (i == 0) {
-            if (!mbar_wait(&bar_k_full, kph, abort_flag, a.err, kDevTimeoutLoad)) {
-              ok = false;
-              break;
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t ad =
+                  smem_desc_sw128(q_base + (kk >> 2) * kRows * 128 + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd =
+                  smem_desc_sw128(k_base + (kk >> 2) * kKeys * 128 + (kk & 3) * 32, 16, 1024);
+              umma_bf16(d_tm, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
             }
-            kph ^= 1;
+            umma_commit(&bar_q_empty[qs]);
+            umma_commit(&bar_s_full[sb]);
+            if (sc.i == sc.m.ntiles - 1) {
+              umma_commit(&bar_k_empty);
+              k_ready = false;
+            }
+            committed = true;
+            last_bar = &bar_s_full[sb];
+            last_par = sph[sb];
+            sph[sb] ^= 1;
+            sb ^= 1;
+            if (++qs == kQStages) qs = 0, qph ^= 1;
+            ++s_count;
+            next_tile(sc, a, n_units);
+            progress = true;
           }
-          if (!mbar_wait(&bar_q_full[qs], qph, abort_flag, a.err, kDevTimeoutLoad) ||
-              !mbar_wait(&bar_s_empty[sb], sph[sb] ^ 1, abort_flag, a.err, kDevTimeoutConsumer)) {
-            ok = false;
-            break;
+        }
+        // ---- O = P V for the oldest tile whose S has been issued ----
+        if (pv_count < s_count) {
+          bool ready = true;
+          if (pc.i == 0 && !v_ready) {
+            ready = mbar_probe(&bar_v_full, vph);
+            if (ready) vph ^= 1, v_ready = true;
           }
-          tc_fence_after();
-          const uint32_t q_base = smem_u32(sQ + qs * Cfg::kQBytes);
-          const uint32_t k_base = smem_u32(sK);
-          const uint32_t d_tm = tmem + sb * 128;
+          // P buffer pb and O buffer pb are used in lockstep: one phase each
+          ready = ready && mbar_probe(&bar_p_full[pb], pph[pb]) &&
+                  mbar_probe(&bar_o_empty[pb], pph[pb] ^ 1);
+          if (ready) {
+            tc_fence_after();
+            const uint32_t p_base = smem_u32(sP + pb * Cfg::kPBytes);
+            const uint32_t d_tm = tmem + 256 + pb * 128;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad =
-                smem_desc_sw128(q_base + (kk >> 2) * kRows * 128 + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd =
-                smem_desc_sw128(k_base + (kk >> 2) * kKeys * 128 + (kk & 3) * 32, 16, 1024);
-            umma_bf16(d_tm, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kKeys / 16; ++kk) {
+              const uint64_t ad =
+                  smem_desc_sw128(p_base + (kk >> 2) * kRows * 128 + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(v_base + kk * 16 * 128, kKeys * 128, 1024);
+              umma_bf16(d_tm, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&bar_p_empty[pb]);
+            umma_commit(&bar_o_full[pb]);
+            if (pc.i == pc.m.ntiles - 1) {
+              umma_commit(&bar_v_empty);
+              v_ready = false;
+            }
+            committed = true;
+            last_bar = &bar_o_full[pb];
+            last_par = pph[pb];
+            pph[pb] ^= 1;
+            pb ^= 1;
+            ++pv_count;
+            next_tile(pc, a, n_units);
+            progress = true;
           }
-          umma_commit(&bar_q_empty[qs]);
-          umma_commit(&bar_s_full[sb]);
-          if (i == m.ntiles - 1) umma_commit(&bar_k_empty);
-          committed = true;
-          last_bar = &bar_s_full[sb];
-          last_par = sph[sb];
-          sph[sb] ^= 1;
-          sb ^= 1;
-          if (++qs == kQStages) qs = 0, qph ^= 1;
-          if (has_prev && !issue_pv(prev_first, prev_last)) {
-            ok = false;
-            break;
-          }
-          has_prev = true;
-          prev_first = (i == 0);
-          prev_last = (i == m.ntiles - 1);
+        }
+        if (progress) {
+          idle = false;
+        } else if (!idle) {
+          idle = true;
+          idle_since = global_timer_ns();
+        } else if (*abort_flag) {
+          break;
+        } else if (global_timer_ns() - idle_since > kWaitLimitNs) {
+          *abort_flag = 1;
+          record_error(a.err, kDevTimeoutConsumer);
+          break;
         }
       }
-      if (ok && has_prev) ok = issue_pv(prev_first, prev_last);
       if (*abort_flag && committed) {
         volatile int no_abort = 0;
         mbar_wait(last_bar, last_par, &no_abort, nullptr, 0);
@@ -566,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_barrier(bar_id, 128);
       if (valid) {
         const int64_t slot0 = (((t - a.row_begin) * a.G + m.g) * a.top_k + r) * a.HG;
-        a.part_lse[slot0 + hh] = mx * a.scale + logf(l);
+        a.part_lse[slot0 + hh] = mx * a.scale + __logf(l);
         if (hh == 0) {
 #pragma unroll
           for (int ri = 0; ri < Cfg::kRegions; ++ri)
