@@ -130,7 +130,14 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+// A failed launch is reported through the status; the runtime's last-error
+// slot is cleared so that the caller's next, unrelated CUDA call does not
+// see it again (a sticky error stays sticky regardless).
+msa_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MSA_OK;
+  (void)cudaGetLastError();
+  return MSA_ERR_CUDA;
+}
 
 }  // namespace
 }  // namespace msa
@@ -345,7 +352,7 @@ msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, 
     ip.ids = ids;
     ip.err = err;
     ip.num_sms = sms;
-    if (launch_index_select(ip, s) != cudaSuccess) return MSA_ERR_CUDA;
+    if (launch_index_select(ip, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
     ++launches;
     mark(ev + 1, s);
 
@@ -364,7 +371,7 @@ msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, 
     cp.unit_desc = at<int4>(ws, L.unit_list);
     cp.tile_tokens = main_tile_tokens(H, G);
     cp.unit_tiles = kUnitTiles;
-    if (launch_csr(cp, s, &launches) != cudaSuccess) return MSA_ERR_CUDA;
+    if (launch_csr(cp, s, &launches) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
     mark(ev + 2, s);
 
     MainLaunch mp{};
@@ -388,7 +395,7 @@ msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, 
     mp.part_lse = at<float>(ws, L.part_lse);
     mp.err = err;
     mp.grid = sms;
-    if (launch_main(mp, s) != cudaSuccess) return MSA_ERR_CUDA;
+    if (launch_main(mp, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
     ++launches;
     mark(ev + 3, s);
 
@@ -402,7 +409,7 @@ msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, 
     gp.d = d;
     gp.top_k = kk;
     gp.out = static_cast<uint8_t*>(out) + (size_t)t0 * H * d * 2;
-    if (launch_merge(gp, s) != cudaSuccess) return MSA_ERR_CUDA;
+    if (launch_merge(gp, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
     ++launches;
     mark(ev + 4, s);
   }

@@ -17,17 +17,18 @@
 // ln rowsum) goes to slot (t, g, r, head); the merge kernel combines the <= k
 // slots of a query with log-sum-exp weights.
 //
-// Warp roles (352 threads, one CTA per SM, persistent over units):
+// Warp roles (608 threads, one CTA per SM, persistent over units):
 //   warp 0     Q producer: a TMA gather of each hitting token's H/G
-//              contiguous query rows into a 3-stage ring;
-//   warp 10    K/V loader: TMA of K_j / V_j (3-D map: one group's rows) once
+//              contiguous query rows into a 2-stage ring;
+//   warp 18    K/V loader: TMA of K_j / V_j (3-D map: one group's rows) once
 //              per unit, plus an L2 prefetch of the next unit's blocks;
 //   warp 1     MMA issuer (one thread): issues whichever of the next S or the
 //              oldest pending PV has its inputs ready;
-//   warps 2-9  two softmax + epilogue warpgroups taking alternate tiles;
-//              thread <-> TMEM lane <-> tile row.  The epilogue stages the
-//              fp16 partials in the tile's (consumed) P buffer and writes each
-//              token's heads with one bulk copy (2 KiB for 8 heads of 128).
+//   warps 2-17 two softmax + epilogue groups of 8 warps taking alternate
+//              tiles; a tile row is split between two warps of its group
+//              (TMEM lane = row, 64 columns each).  The epilogue stages the
+//              fp16 partials in the tile's consumed P buffer and writes each
+//              token's heads with a TMA store (2 KiB for 8 heads of 128).
 // TMEM: two S buffers (2 x 128 columns) and two O buffers (2 x 128 columns),
 // buffer w belonging to warpgroup w.
 #include "kernels.h"
@@ -37,11 +38,13 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 352;  // Q producer, MMA, 2 softmax warpgroups, K/V loader
-constexpr int kKVWarp = 10;
+// Q producer, MMA issuer, 2 softmax groups of 8 warps, K/V loader
+constexpr int kThreads = 608;
+constexpr int kKVWarp = 18;
+constexpr int kGroupThreads = 256;
 constexpr int kRows = 128;
 constexpr int kKeys = 128;
-constexpr int kQStages = 3;
+constexpr int kQStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -146,20 +149,20 @@ __device__ __forceinline__ bool read_entry(const MainArgs& a, int e, int64_t& t,
   return ok;
 }
 
-// exp2 of 64 scores (one half of a row), bf16 packing into the swizzled P
-// tile, and the fp32 sum of the rounded values.  MASK: keep columns <= lim.
+// exp2 of 32 scores of a row, bf16 packing into 4 chunks (from chunk0) of the
+// row's 128-byte swizzled P region, and the fp32 sum of the rounded values.
+// MASK: keep columns <= lim (relative to the first of the 32).
 template <bool MASK>
-__device__ __forceinline__ void softmax_chunk(const uint32_t (&sv)[2][32], uint64_t k2,
-                                              uint64_t nm2, int lim, uint8_t* pdst, int row,
-                                              uint64_t& acc_a, uint64_t& acc_b) {
+__device__ __forceinline__ void softmax32(const uint32_t (&sv)[32], uint64_t k2, uint64_t nm2,
+                                          int lim, uint8_t* region, int row, int chunk0,
+                                          uint64_t& acc_a, uint64_t& acc_b) {
 #pragma unroll
-  for (int c8 = 0; c8 < 8; ++c8) {
+  for (int c8 = 0; c8 < 4; ++c8) {
     uint32_t w4[4];
 #pragma unroll
     for (int x2 = 0; x2 < 4; ++x2) {
       const int col = c8 * 8 + 2 * x2;
-      const uint64_t s2 = f2_pack(__uint_as_float(sv[col >> 5][col & 31]),
-                                  __uint_as_float(sv[col >> 5][(col & 31) + 1]));
+      const uint64_t s2 = f2_pack(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1]));
       float a0, a1;
       f2_unpack(f2_fma(s2, k2, nm2), a0, a1);
       float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
@@ -174,7 +177,8 @@ __device__ __forceinline__ void softmax_chunk(const uint32_t (&sv)[2][32], uint6
         acc_a = f2_add(acc_a, bf16x2_as_f2(w));
       w4[x2] = w;
     }
-    *reinterpret_cast<uint4*>(pdst + sw128_offset(row, c8)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    *reinterpret_cast<uint4*>(region + sw128_offset(row, chunk0 + c8)) =
+        make_uint4(w4[0], w4[1], w4[2], w4[3]);
   }
 }
 
@@ -199,6 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint64_t bar_o_full[2], bar_o_empty[2];
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
+  __shared__ float xchg_max[2][2][kRows];  // [group][column half][row]
+  __shared__ float xchg_sum[2][2][kRows];
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
@@ -213,11 +219,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar_v_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_s_full[i], 1);
-      mbar_init(&bar_s_empty[i], 128);
-      mbar_init(&bar_p_full[i], 128);
+      mbar_init(&bar_s_empty[i], kGroupThreads);
+      mbar_init(&bar_p_full[i], kGroupThreads);
       mbar_init(&bar_p_empty[i], 1);
       mbar_init(&bar_o_full[i], 1);
-      mbar_init(&bar_o_empty[i], 128);
+      mbar_init(&bar_o_empty[i], kGroupThreads);
     }
     fence_mbar_init();
   }
@@ -242,8 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int qs = 0;
     uint32_t qph = 0;
     // last issued phase per stage, for draining after an abort
-    uint32_t q_last[kQStages] = {0, 0, 0};
-    bool q_any[kQStages] = {false, false, false};
+    uint32_t q_last[kQStages] = {};
+    bool q_any[kQStages] = {};
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const MUnit m = decode_unit(a, u);
@@ -440,26 +446,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---------------- softmax + epilogue: two warpgroups ----------------
-    // warpgroup w (warps 2+4w .. 5+4w) owns the tiles of parity w, and with
-    // them S buffer w, P buffer w and O buffer w.
-    const int wg = (warp - 2) >> 2;
-    const uint32_t bar_id = 1 + wg;  // named barrier of this warpgroup
+    // ---------------- softmax + epilogue: two groups of 8 warps ----------------
+    // Group grp (warps 2+8grp .. 9+8grp) owns the tiles of parity grp, with S
+    // buffer grp, P buffer grp and O buffer grp.  Each row of a tile is split
+    // between two warps of the group (same TMEM lane quarter, column half hc),
+    // which combine their row max and row sum through shared memory.
+    const int grp = (warp - 2) >> 3;
+    const int hc = ((warp - 2) & 7) >> 2;  // column half: S/P columns 64hc..64hc+63
+    const uint32_t bar_id = 1 + grp;       // named barrier of this group (256 threads)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int ts = row >> a.log2slot;
     const int hh = row & (slot - 1);
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t s_col = wg * 128, o_col = 256 + wg * 128;
-    uint8_t* pbuf = sP + wg * Cfg::kPBytes;
+    const uint32_t s_col = grp * 128 + hc * 64, o_col = 256 + grp * 128 + hc * 64;
+    const bool has_o = hc * 64 < D;
+    uint8_t* pbuf = sP + grp * Cfg::kPBytes;
+    uint8_t* preg = pbuf + hc * kRows * 128;  // this half's 128-byte swizzle region
     uint32_t sph = 0, pph = 0, oph = 0;
     bool ok = true;
-    bool store_pending = false;  // this thread issued bulk stores from pbuf
+    bool store_pending = false;  // this thread issued TMA stores from pbuf
 
-    // Tile position in this CTA's sequence; this warpgroup takes every other
-    // tile.  The next tile's list entry is loaded one iteration ahead.
     TilePos cur = first_tile(a, n_units);
-    if (wg == 1) next_tile(cur, a, n_units);
+    if (grp == 1) next_tile(cur, a, n_units);
     int32_t cur_ent = cur.more ? prefetch_entry(a, cur, ts, hh) : -1;
 
     while (cur.more && ok) {
@@ -474,108 +483,107 @@ __global__ void __launch_bounds__(kThreads, 1)
       int r = 0;
       bool good = false;
       if (row_valid) good = check_entry(a, cur_ent, t, r);
-      const int lim = row_valid ? (int)min64(t - (int64_t)m.j * kKeys, kKeys - 1) : kKeys - 1;
-      const bool unmasked = __all_sync(0xffffffffu, lim >= kKeys - 1);
+      // last visible column of this half (keys s <= t on the local block)
+      const int lim = (row_valid ? (int)min64(t - (int64_t)m.j * kKeys, kKeys - 1) : kKeys - 1) -
+                      hc * 64;
+      const bool unmasked = __all_sync(0xffffffffu, lim >= 63);
 
-      // ---- softmax ----
-      if (!mbar_wait(&bar_s_full[wg], sph, abort_flag, a.err, kDevTimeoutMma)) {
+      // ---- pass 1: max over this half's 64 scores ----
+      if (!mbar_wait(&bar_s_full[grp], sph, abort_flag, a.err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // pass 1: row max over the 128 scores (one TMEM round trip)
-      float mx = -INFINITY;
+      float hmx = -INFINITY;
       {
-        uint32_t sv[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(lane_addr + s_col + c * 32, sv[c]);
+        uint32_t sv[2][32];
+        tmem_ld_32x32b_x32(lane_addr + s_col, sv[0]);
+        tmem_ld_32x32b_x32(lane_addr + s_col + 32, sv[1]);
         tmem_wait();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence(sv[c]);
+        reg_fence(sv[0]);
+        reg_fence(sv[1]);
         if (unmasked) {
-          float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
+          float x0 = -INFINITY, x1 = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 4; c += 2)
-#pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              x0 = max3f(x0, __uint_as_float(sv[c][x]), __uint_as_float(sv[c][x + 1]));
-              x1 = max3f(x1, __uint_as_float(sv[c + 1][x]), __uint_as_float(sv[c + 1][x + 1]));
-            }
-          mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+          for (int x = 0; x < 32; x += 2) {
+            x0 = max3f(x0, __uint_as_float(sv[0][x]), __uint_as_float(sv[0][x + 1]));
+            x1 = max3f(x1, __uint_as_float(sv[1][x]), __uint_as_float(sv[1][x + 1]));
+          }
+          hmx = fmaxf(x0, x1);
         } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int x = 0; x < 32; ++x)
-              if (c * 32 + x <= lim) mx = fmaxf(mx, __uint_as_float(sv[c][x]));
+              if (c * 32 + x <= lim) hmx = fmaxf(hmx, __uint_as_float(sv[c][x]));
         }
       }
-      if (!(row_valid && good) || !(mx > -INFINITY)) mx = 0.f;
-      const float mxs = mx * a.scale_log2;
-
-      if (!mbar_wait(&bar_p_empty[wg], pph ^ 1, abort_flag, a.err, kDevTimeoutMma)) {
-        ok = false;
-        break;
-      }
-      // the previous tile's partials are still being copied out of this buffer
+      xchg_max[grp][hc][row] = hmx;
+      // the previous tile's partials must be out of the P buffer before anyone
+      // rewrites it; the barrier also publishes both halves' maxima
       if (store_pending) {
         bulk_wait_read<0>();
         store_pending = false;
       }
-      named_barrier(bar_id, 128);
-      // pass 2: P = exp2(scale*log2e*(S - max)) in bf16, written in the K-major
-      // 128-byte-swizzled layout the PV MMA reads; l sums the rounded values
+      named_barrier(bar_id, 256);
+      float mx = fmaxf(xchg_max[grp][0][row], xchg_max[grp][1][row]);
+      if (!(row_valid && good) || !(mx > -INFINITY)) mx = 0.f;
+      const float mxs = mx * a.scale_log2;
+      if (!mbar_wait(&bar_p_empty[grp], pph ^ 1, abort_flag, a.err, kDevTimeoutMma)) {
+        ok = false;
+        break;
+      }
+
+      // ---- pass 2: P = exp2(scale*log2e*(S - max)) in bf16, 32 columns at a time ----
       const uint64_t k2 = f2_pack(a.scale_log2, a.scale_log2);
       const uint64_t nm2 = f2_pack(-mxs, -mxs);
       uint64_t acc_a = f2_pack(0.f, 0.f), acc_b = acc_a;
 #pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t sv[2][32];
-        tmem_ld_32x32b_x32(lane_addr + s_col + hf * 64, sv[0]);
-        tmem_ld_32x32b_x32(lane_addr + s_col + hf * 64 + 32, sv[1]);
+      for (int pc = 0; pc < 2; ++pc) {
+        uint32_t sv[32];
+        tmem_ld_32x32b_x32(lane_addr + s_col + pc * 32, sv);
         tmem_wait();
-        reg_fence(sv[0]);
-        reg_fence(sv[1]);
-        uint8_t* pdst = pbuf + hf * kRows * 128;
-        if (unmasked) {
-          softmax_chunk<false>(sv, k2, nm2, 0, pdst, row, acc_a, acc_b);
-        } else {
-          softmax_chunk<true>(sv, k2, nm2, lim - hf * 64, pdst, row, acc_a, acc_b);
-        }
+        reg_fence(sv);
+        if (unmasked)
+          softmax32<false>(sv, k2, nm2, 0, preg, row, pc * 4, acc_a, acc_b);
+        else
+          softmax32<true>(sv, k2, nm2, lim - pc * 32, preg, row, pc * 4, acc_a, acc_b);
       }
+      tc_fence_before();
+      mbar_arrive(&bar_s_empty[grp]);
+      sph ^= 1;
+      fence_async_smem();
+      mbar_arrive(&bar_p_full[grp]);
+      pph ^= 1;
       float la0, la1, lb0, lb1;
       f2_unpack(acc_a, la0, la1);
       f2_unpack(acc_b, lb0, lb1);
-      const float l = (la0 + la1) + (lb0 + lb1);
-      tc_fence_before();
-      mbar_arrive(&bar_s_empty[wg]);
-      sph ^= 1;
-      fence_async_smem();
-      mbar_arrive(&bar_p_full[wg]);
-      pph ^= 1;
+      xchg_sum[grp][hc][row] = (la0 + la1) + (lb0 + lb1);
+      named_barrier(bar_id, 256);
+      const float l = xchg_sum[grp][0][row] + xchg_sum[grp][1][row];
 
-      // ---- epilogue: O / l -> fp16 partial, staged in the (now free) P buffer ----
-      if (!mbar_wait(&bar_o_full[wg], oph, abort_flag, a.err, kDevTimeoutMma)) {
+      // ---- epilogue: O / l -> fp16, staged in the (consumed) P buffer ----
+      if (!mbar_wait(&bar_o_full[grp], oph, abort_flag, a.err, kDevTimeoutMma)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const bool valid = row_valid && good;
-      const float inv = 1.0f / l;
-      const uint64_t inv2 = f2_pack(inv, inv);
-      // same 128-byte-swizzled layout as P: conflict-free writes, and the TMA
-      // store below undoes the swizzle on its way to global memory
-      {
-        uint32_t o[D / 32][32];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld_32x32b_x32(lane_addr + o_col + c * 32, o[c]);
+      if (has_o) {
+        const float inv = 1.0f / l;
+        const uint64_t inv2 = f2_pack(inv, inv);
+        uint32_t o[2][32];
+        tmem_ld_32x32b_x32(lane_addr + o_col, o[0]);
+        tmem_ld_32x32b_x32(lane_addr + o_col + 32, o[1]);
         tmem_wait();
+        reg_fence(o[0]);
+        reg_fence(o[1]);
+        // same 128-byte-swizzled layout as P: conflict-free writes; the TMA
+        // store below undoes the swizzle on its way to global memory
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) reg_fence(o[c]);
-#pragma unroll
-        for (int c16 = 0; c16 < D / 8; ++c16) {
+        for (int c8 = 0; c8 < 8; ++c8) {
           uint4 w;
-          const uint32_t* src = &o[c16 >> 2][(c16 & 3) * 8];
+          const uint32_t* src = &o[c8 >> 2][(c8 & 3) * 8];
 #pragma unroll
           for (int x2 = 0; x2 < 4; ++x2) {
             float f0, f1;
@@ -584,16 +592,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                       f0, f1);
             (&w.x)[x2] = pack_half2(f0, f1);
           }
-          *reinterpret_cast<uint4*>(pbuf + (c16 >> 3) * kRows * 128 + sw128_offset(row, c16 & 7)) =
-              w;
+          *reinterpret_cast<uint4*>(preg + sw128_offset(row, c8)) = w;
         }
       }
       tc_fence_before();
-      mbar_arrive(&bar_o_empty[wg]);
+      mbar_arrive(&bar_o_empty[grp]);
       oph ^= 1;
       fence_async_smem();
-      named_barrier(bar_id, 128);
-      if (valid) {
+      named_barrier(bar_id, 256);
+      if (valid && hc == 0) {
         const int64_t slot0 = (((t - a.row_begin) * a.G + m.g) * a.top_k + r) * a.HG;
         a.part_lse[slot0 + hh] = mx * a.scale + __logf(l);
         if (hh == 0) {
