@@ -11,8 +11,10 @@
 //
 // Per tile (128 rows = TT tokens x the H/G heads of group g):
 //   S = Q_tile K_j^T            tcgen05.mma M=128 N=128 K=d   (TMEM, fp32)
-//   P = exp(scale*(S - rowmax)) softmax warps, causal mask on the local block
-//   O = P V_j                   tcgen05.mma M=128 N=d  K=128  (V is MN-major)
+//   P = exp(scale*(S - rowmax)) softmax warps, causal mask on the local block;
+//                               bf16 P overwrites the S columns already read
+//   O = P V_j                   tcgen05.mma M=128 N=d  K=128, A = P from TMEM,
+//                               B = V_j from shared memory (MN-major)
 // and the row's partial (o = O / rowsum in fp16, lse = scale*rowmax +
 // ln rowsum) goes to slot (t, g, r, head); the merge kernel combines the <= k
 // slots of a query with log-sum-exp weights.
@@ -27,10 +29,12 @@
 //   warps 2-17 two softmax + epilogue groups of 8 warps taking alternate
 //              tiles; a tile row is split between two warps of its group
 //              (TMEM lane = row, 64 columns each).  The epilogue stages the
-//              fp16 partials in the tile's consumed P buffer and writes each
-//              token's heads with a TMA store (2 KiB for 8 heads of 128).
-// TMEM: two S buffers (2 x 128 columns) and two O buffers (2 x 128 columns),
-// buffer w belonging to warpgroup w.
+//              fp16 partials in the group's shared staging buffer and writes
+//              each token's heads with a TMA store (2 KiB for 8 heads of 128).
+// TMEM: two S/P buffers (2 x 128 columns) and two O buffers (2 x 128
+// columns), buffer w belonging to softmax group w.  Keeping P in TMEM halves
+// the shared-memory operand traffic of the PV product and leaves the P
+// stores off the shared-memory pipe.
 #include "kernels.h"
 #include "sm100.cuh"
 #include "tmap.h"
@@ -47,16 +51,24 @@ constexpr int kKeys = 128;
 constexpr int kQStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Shared-memory tiles of 128 rows x D (Q, and the fp16 O staging) are kept as
+// 16 groups of 8 rows; a group holds its D/64 column chunks one after the
+// other, each chunk 8 rows x 128 bytes with the 128-byte swizzle.  The 8-row
+// group of a token's heads is then 1-2 KiB of contiguous shared memory,
+// moved by ONE 3-D TMA copy (x = 64 columns, y = rows, z = chunk; chunk
+// stride 128 bytes in global memory), and the K-major MMA operand advances by
+// D/64 KiB per 8 rows.
 template <int D>
 struct MainCfg {
   static constexpr int kRegions = D / 64;
+  static constexpr int kGroupBytes = kRegions * 1024;  // one 8-row group
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kKVBytes = kKeys * D * 2;
-  static constexpr int kPBytes = kRows * kKeys * 2;
+  static constexpr int kOBytes = kRows * D * 2;  // fp16 staging of one O tile
   static constexpr int kOffK = kQStages * kQBytes;
   static constexpr int kOffV = kOffK + kKVBytes;
-  static constexpr int kOffP = kOffV + kKVBytes;
-  static constexpr int kSmem = kOffP + 2 * kPBytes + 1024;
+  static constexpr int kOffO = kOffV + kKVBytes;
+  static constexpr int kSmem = kOffO + 2 * kOBytes + 1024;
 };
 
 struct MainArgs {
@@ -149,36 +161,31 @@ __device__ __forceinline__ bool read_entry(const MainArgs& a, int e, int64_t& t,
   return ok;
 }
 
-// exp2 of 32 scores of a row, bf16 packing into 4 chunks (from chunk0) of the
-// row's 128-byte swizzled P region, and the fp32 sum of the rounded values.
-// MASK: keep columns <= lim (relative to the first of the 32).
+// exp2 of 32 scores of a row, packed two bf16 per word (the even column in
+// the lower half, the layout of an A operand in TMEM), and the fp32 sum of the
+// rounded values.  MASK: keep columns <= lim (relative to the first of the 32).
 template <bool MASK>
 __device__ __forceinline__ void softmax32(const uint32_t (&sv)[32], uint64_t k2, uint64_t nm2,
-                                          int lim, uint8_t* region, int row, int chunk0,
-                                          uint64_t& acc_a, uint64_t& acc_b) {
+                                          int lim, uint32_t taddr, uint64_t& acc_a,
+                                          uint64_t& acc_b) {
+  uint32_t w[16];
 #pragma unroll
-  for (int c8 = 0; c8 < 4; ++c8) {
-    uint32_t w4[4];
-#pragma unroll
-    for (int x2 = 0; x2 < 4; ++x2) {
-      const int col = c8 * 8 + 2 * x2;
-      const uint64_t s2 = f2_pack(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1]));
-      float a0, a1;
-      f2_unpack(f2_fma(s2, k2, nm2), a0, a1);
-      float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
-      if (MASK) {
-        p0 = col <= lim ? p0 : 0.f;
-        p1 = col + 1 <= lim ? p1 : 0.f;
-      }
-      const uint32_t w = pack_bf16x2(p0, p1);
-      if (x2 & 1)
-        acc_b = f2_add(acc_b, bf16x2_as_f2(w));
-      else
-        acc_a = f2_add(acc_a, bf16x2_as_f2(w));
-      w4[x2] = w;
+  for (int x2 = 0; x2 < 16; ++x2) {
+    const int col = 2 * x2;
+    const uint64_t s2 = f2_pack(__uint_as_float(sv[col]), __uint_as_float(sv[col + 1]));
+    float a0, a1;
+    f2_unpack(f2_fma(s2, k2, nm2), a0, a1);
+    float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+    if (MASK) {
+      p0 = col <= lim ? p0 : 0.f;
+      p1 = col + 1 <= lim ? p1 : 0.f;
     }
-    *reinterpret_cast<uint4*>(region + sw128_offset(row, chunk0 + c8)) =
-        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    w[x2] = pack_bf16x2(p0, p1);
+    if (x2 & 1)
+      acc_b = f2_add(acc_b, bf16x2_as_f2(w[x2]));
+    else
+      acc_a = f2_add(acc_a, bf16x2_as_f2(w[x2]));
+    if ((x2 & 7) == 7) tmem_st_32x32b_x8(taddr + (x2 - 7), &w[x2 - 7]);
   }
 }
 
@@ -194,12 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem;
   uint8_t* sK = smem + Cfg::kOffK;
   uint8_t* sV = smem + Cfg::kOffV;
-  uint8_t* sP = smem + Cfg::kOffP;
+  uint8_t* sO = smem + Cfg::kOffO;
 
   __shared__ uint64_t bar_q_full[kQStages], bar_q_empty[kQStages];
   __shared__ uint64_t bar_k_full, bar_k_empty, bar_v_full, bar_v_empty;
   __shared__ uint64_t bar_s_full[2], bar_s_empty[2];
-  __shared__ uint64_t bar_p_full[2], bar_p_empty[2];
+  __shared__ uint64_t bar_p_full[2];
   __shared__ uint64_t bar_o_full[2], bar_o_empty[2];
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
@@ -219,9 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar_v_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_s_full[i], 1);
-      mbar_init(&bar_s_empty[i], kGroupThreads);
+      mbar_init(&bar_s_empty[i], 1);  // committed by the PV that read P
       mbar_init(&bar_p_full[i], kGroupThreads);
-      mbar_init(&bar_p_empty[i], 1);
       mbar_init(&bar_o_full[i], 1);
       mbar_init(&bar_o_empty[i], kGroupThreads);
     }
@@ -263,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           ok = mbar_wait(&bar_q_empty[qs], qph ^ 1, abort_flag, a.err, kDevTimeoutMma);
           if (ok) {
-            mbar_arrive_expect_tx(&bar_q_full[qs], (uint32_t)nt * a.HG * D * 2);
+            mbar_arrive_expect_tx(&bar_q_full[qs], (uint32_t)nt * slot * D * 2);
             q_any[qs] = true;
             q_last[qs] = qph;
           }
@@ -271,11 +277,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane < nt) {
+          // the token's slot rows, 8 at a time (rows past H/G are other
+          // heads' queries, never used; past the tensor end they read zero)
           const int32_t qrow = (int32_t)(t * a.H + (int64_t)m.g * a.HG);
-          uint8_t* dst = sQ + qs * Cfg::kQBytes + lane * slot * 128;
-#pragma unroll
-          for (int ri = 0; ri < Cfg::kRegions; ++ri)
-            tma_load_2d(dst + ri * kRows * 128, &map_q, &bar_q_full[qs], ri * 64, qrow);
+          uint8_t* dst = sQ + qs * Cfg::kQBytes + (lane * slot / 8) * Cfg::kGroupBytes;
+          for (int k8 = 0; k8 < slot; k8 += 8)
+            tma_load_3d(dst + (k8 / 8) * Cfg::kGroupBytes, &map_q, &bar_q_full[qs], 0,
+                        qrow + k8, 0);
         }
         __syncwarp();
         if (++qs == kQStages) qs = 0, qph ^= 1;
@@ -367,8 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t d_tm = tmem + sb * 128;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t ad =
-                  smem_desc_sw128(q_base + (kk >> 2) * kRows * 128 + (kk & 3) * 32, 16, 1024);
+              const uint64_t ad = smem_desc_sw128(q_base + (kk >> 2) * 1024 + (kk & 3) * 32, 16,
+                                                  Cfg::kGroupBytes);
               const uint64_t bd =
                   smem_desc_sw128(k_base + (kk >> 2) * kKeys * 128 + (kk & 3) * 32, 16, 1024);
               umma_bf16(d_tm, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
@@ -397,21 +405,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             ready = mbar_probe(&bar_v_full, vph);
             if (ready) vph ^= 1, v_ready = true;
           }
-          // P buffer pb and O buffer pb are used in lockstep: one phase each
+          // S/P buffer pb and O buffer pb are used in lockstep: one phase each
           ready = ready && mbar_probe(&bar_p_full[pb], pph[pb]) &&
                   mbar_probe(&bar_o_empty[pb], pph[pb] ^ 1);
           if (ready) {
             tc_fence_after();
-            const uint32_t p_base = smem_u32(sP + pb * Cfg::kPBytes);
             const uint32_t d_tm = tmem + 256 + pb * 128;
 #pragma unroll
             for (int kk = 0; kk < kKeys / 16; ++kk) {
-              const uint64_t ad =
-                  smem_desc_sw128(p_base + (kk >> 2) * kRows * 128 + (kk & 3) * 32, 16, 1024);
+              // keys 16kk..16kk+15: written by column half kk/4 as 8 packed
+              // columns at offset 8*(kk%4) of that half's S columns
+              const uint32_t a_tm = tmem + pb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
               const uint64_t bd = smem_desc_sw128(v_base + kk * 16 * 128, kKeys * 128, 1024);
-              umma_bf16(d_tm, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
+              umma_bf16_ts(d_tm, a_tm, bd, idesc_o, kk > 0 ? 1u : 0u);
             }
-            umma_commit(&bar_p_empty[pb]);
+            umma_commit(&bar_s_empty[pb]);  // P read: the S/P buffer is free
             umma_commit(&bar_o_full[pb]);
             if (pc.i == pc.m.ntiles - 1) {
               umma_commit(&bar_v_empty);
@@ -447,10 +455,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- softmax + epilogue: two groups of 8 warps ----------------
-    // Group grp (warps 2+8grp .. 9+8grp) owns the tiles of parity grp, with S
-    // buffer grp, P buffer grp and O buffer grp.  Each row of a tile is split
-    // between two warps of the group (same TMEM lane quarter, column half hc),
-    // which combine their row max and row sum through shared memory.
+    // Group grp (warps 2+8grp .. 9+8grp) owns the tiles of parity grp, with S/P
+    // buffer grp and O buffer grp.  Each row of a tile is split between two
+    // warps of the group (same TMEM lane quarter, column half hc), which
+    // combine their row max and row sum through shared memory.
+    //
+    // The epilogue of a tile runs one group iteration late, after the softmax
+    // of the group's next tile: its PV product then completes while the group
+    // works on that softmax instead of being waited for.
     const int grp = (warp - 2) >> 3;
     const int hc = ((warp - 2) & 7) >> 2;  // column half: S/P columns 64hc..64hc+63
     const uint32_t bar_id = 1 + grp;       // named barrier of this group (256 threads)
@@ -461,17 +473,92 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t s_col = grp * 128 + hc * 64, o_col = 256 + grp * 128 + hc * 64;
     const bool has_o = hc * 64 < D;
-    uint8_t* pbuf = sP + grp * Cfg::kPBytes;
-    uint8_t* preg = pbuf + hc * kRows * 128;  // this half's 128-byte swizzle region
-    uint32_t sph = 0, pph = 0, oph = 0;
+    uint8_t* obuf = sO + grp * Cfg::kOBytes;
+    // staging of this row: its 8-row group, chunk hc, line hc*rows + row%8
+    // (rows = min(H/G, 8): the height of the TMA store box)
+    const int box_rows = a.HG < 8 ? a.HG : 8;
+    uint8_t* oblk = obuf + (row >> 3) * Cfg::kGroupBytes;
+    const int oline = hc * box_rows + (row & 7);
+    const bool stage_row = (row & 7) < box_rows;
+    uint32_t sph = 0, oph = 0;
     bool ok = true;
-    bool store_pending = false;  // this thread issued TMA stores from pbuf
+    bool store_pending = false;  // this thread issued TMA stores from obuf
+
+    // the tile whose epilogue is pending (this thread's row of it): first
+    // partial row, lse and 1/rowsum
+    bool pend = false, pend_valid = false;
+    int64_t pend_slot = 0;
+    float pend_lse = 0.f, pend_inv = 1.f;
+
+    // O / l -> fp16 staged in obuf, then one TMA store per token and region
+    auto epilogue = [&]() -> bool {
+      if (!mbar_wait(&bar_o_full[grp], oph, abort_flag, a.err, kDevTimeoutMma)) return false;
+      tc_fence_after();
+      // 32 columns at a time; the O buffer is released after the last load
+      const uint64_t inv2 = f2_pack(pend_inv, pend_inv);
+#pragma unroll 1
+      for (int oc = 0; oc < 2; ++oc) {
+        uint32_t o[32];
+        if (has_o) {
+          tmem_ld_32x32b_x32(lane_addr + o_col + oc * 32, o);
+          tmem_wait();
+          reg_fence(o);
+        }
+        if (oc == 1) {
+          tc_fence_before();
+          mbar_arrive(&bar_o_empty[grp]);
+          oph ^= 1;
+        }
+        if (has_o && stage_row) {
+          // 128-byte-swizzled staging: conflict-free writes; the TMA store
+          // below undoes the swizzle on its way to global memory
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint4 w;
+#pragma unroll
+            for (int x2 = 0; x2 < 4; ++x2) {
+              float f0, f1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[c4 * 8 + 2 * x2]),
+                                       __uint_as_float(o[c4 * 8 + 2 * x2 + 1])),
+                               inv2),
+                        f0, f1);
+              (&w.x)[x2] = pack_half2(f0, f1);
+            }
+            *reinterpret_cast<uint4*>(oblk + sw128_offset(oline, oc * 4 + c4)) = w;
+          }
+        }
+      }
+      fence_async_smem();
+      named_barrier(bar_id, 256);
+      if (pend_valid && hc == 0) {
+        a.part_lse[pend_slot + hh] = pend_lse;
+        if ((hh & 7) == 0) {
+          // this row's 8-row group: all of its column chunks in one copy
+          tma_store_3d(&map_o, oblk, 0, (int32_t)(pend_slot + hh), 0);
+          bulk_commit();
+          store_pending = true;
+        }
+      }
+      return true;
+    };
 
     TilePos cur = first_tile(a, n_units);
     if (grp == 1) next_tile(cur, a, n_units);
     int32_t cur_ent = cur.more ? prefetch_entry(a, cur, ts, hh) : -1;
 
-    while (cur.more && ok) {
+    // one pass per tile of this group, plus a last one that only drains the
+    // pending epilogue
+    while (cur.more || pend) {
+      if (!cur.more) {
+        // staging must be free: wait for the last store's read
+        if (store_pending) {
+          bulk_wait_read<0>();
+          store_pending = false;
+        }
+        named_barrier(bar_id, 256);
+        if (!epilogue()) ok = false;
+        break;
+      }
       TilePos nxt = cur;
       next_tile(nxt, a, n_units);
       next_tile(nxt, a, n_units);
@@ -519,8 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       xchg_max[grp][hc][row] = hmx;
-      // the previous tile's partials must be out of the P buffer before anyone
-      // rewrites it; the barrier also publishes both halves' maxima
+      // the previous tile's partials must be out of the staging buffer before
+      // the epilogue rewrites it; the barrier also publishes both maxima
       if (store_pending) {
         bulk_wait_read<0>();
         store_pending = false;
@@ -529,12 +616,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       float mx = fmaxf(xchg_max[grp][0][row], xchg_max[grp][1][row]);
       if (!(row_valid && good) || !(mx > -INFINITY)) mx = 0.f;
       const float mxs = mx * a.scale_log2;
-      if (!mbar_wait(&bar_p_empty[grp], pph ^ 1, abort_flag, a.err, kDevTimeoutMma)) {
-        ok = false;
-        break;
-      }
 
       // ---- pass 2: P = exp2(scale*log2e*(S - max)) in bf16, 32 columns at a time ----
+      // chunk pc of this half's S columns becomes 16 packed P columns written
+      // over S columns this thread has already read (s_col + 16pc ..)
       const uint64_t k2 = f2_pack(a.scale_log2, a.scale_log2);
       const uint64_t nm2 = f2_pack(-mxs, -mxs);
       uint64_t acc_a = f2_pack(0.f, 0.f), acc_b = acc_a;
@@ -544,17 +629,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(lane_addr + s_col + pc * 32, sv);
         tmem_wait();
         reg_fence(sv);
+        const uint32_t p_addr = lane_addr + s_col + pc * 16;
         if (unmasked)
-          softmax32<false>(sv, k2, nm2, 0, preg, row, pc * 4, acc_a, acc_b);
+          softmax32<false>(sv, k2, nm2, 0, p_addr, acc_a, acc_b);
         else
-          softmax32<true>(sv, k2, nm2, lim - pc * 32, preg, row, pc * 4, acc_a, acc_b);
+          softmax32<true>(sv, k2, nm2, lim - pc * 32, p_addr, acc_a, acc_b);
       }
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar_s_empty[grp]);
-      sph ^= 1;
-      fence_async_smem();
       mbar_arrive(&bar_p_full[grp]);
-      pph ^= 1;
+      sph ^= 1;
       float la0, la1, lb0, lb1;
       f2_unpack(acc_a, la0, la1);
       f2_unpack(acc_b, lb0, lb1);
@@ -562,56 +646,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_barrier(bar_id, 256);
       const float l = xchg_sum[grp][0][row] + xchg_sum[grp][1][row];
 
-      // ---- epilogue: O / l -> fp16, staged in the (consumed) P buffer ----
-      if (!mbar_wait(&bar_o_full[grp], oph, abort_flag, a.err, kDevTimeoutMma)) {
+      // ---- epilogue of the group's previous tile ----
+      if (pend && !epilogue()) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      const bool valid = row_valid && good;
-      if (has_o) {
-        const float inv = 1.0f / l;
-        const uint64_t inv2 = f2_pack(inv, inv);
-        uint32_t o[2][32];
-        tmem_ld_32x32b_x32(lane_addr + o_col, o[0]);
-        tmem_ld_32x32b_x32(lane_addr + o_col + 32, o[1]);
-        tmem_wait();
-        reg_fence(o[0]);
-        reg_fence(o[1]);
-        // same 128-byte-swizzled layout as P: conflict-free writes; the TMA
-        // store below undoes the swizzle on its way to global memory
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          uint4 w;
-          const uint32_t* src = &o[c8 >> 2][(c8 & 3) * 8];
-#pragma unroll
-          for (int x2 = 0; x2 < 4; ++x2) {
-            float f0, f1;
-            f2_unpack(f2_mul(f2_pack(__uint_as_float(src[2 * x2]), __uint_as_float(src[2 * x2 + 1])),
-                             inv2),
-                      f0, f1);
-            (&w.x)[x2] = pack_half2(f0, f1);
-          }
-          *reinterpret_cast<uint4*>(preg + sw128_offset(row, c8)) = w;
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bar_o_empty[grp]);
-      oph ^= 1;
-      fence_async_smem();
-      named_barrier(bar_id, 256);
-      if (valid && hc == 0) {
-        const int64_t slot0 = (((t - a.row_begin) * a.G + m.g) * a.top_k + r) * a.HG;
-        a.part_lse[slot0 + hh] = mx * a.scale + __logf(l);
-        if (hh == 0) {
-#pragma unroll
-          for (int ri = 0; ri < Cfg::kRegions; ++ri)
-            tma_store_2d(&map_o, pbuf + ri * kRows * 128 + (ts << a.log2slot) * 128, ri * 64,
-                         (int32_t)slot0);
-          bulk_commit();
-          store_pending = true;
-        }
-      }
+      pend = true;
+      pend_valid = row_valid && good;
+      pend_slot = (((t - a.row_begin) * a.G + m.g) * a.top_k + r) * a.HG;
+      pend_lse = mx * a.scale + __logf(l);
+      pend_inv = 1.0f / l;
       cur = nxt;
       cur_ent = nxt_ent;
     }
@@ -630,10 +674,12 @@ cudaError_t launch_main_impl(const MainLaunch& p, cudaStream_t s) {
   const int slot = HG < 8 ? 8 : HG;
   CUtensorMap mq, mk, mv, mo;
   const uint64_t part_rows = (uint64_t)p.rows * p.G * p.top_k * HG;
-  if (!make_tmap_bf16_2d(&mq, p.q, (uint64_t)p.N * p.H, D, D, (uint32_t)HG, 64,
+  const uint32_t box_rows = HG < 8 ? HG : 8;
+  // [rows][D] viewed as (64 columns, rows, D/64 chunks)
+  if (!make_tmap_bf16_3d(&mq, p.q, 64, (uint64_t)p.N * p.H, D / 64, D, 64, 64, 8, D / 64,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&mo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.part_o, part_rows, D, D,
-                    (uint32_t)HG, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_3d(&mo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.part_o, 64, part_rows, D / 64, D, 64,
+                    64, box_rows, D / 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_bf16_3d(&mk, p.k, D, p.G, p.N, D, (uint64_t)p.G * D, 64, 1, kKeys,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_bf16_3d(&mv, p.v, D, p.G, p.N, D, (uint64_t)p.G * D, 64, 1, kKeys,

@@ -47,21 +47,30 @@ inline bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows,
                       box_rows, box_cols, swizzle);
 }
 
-// 3-D bf16 view [d2][d1][d0] (element strides: 1, pitch1, pitch2), box
-// [b2][b1][b0].  Used for one group's rows of a [tokens][groups][dim] tensor.
-inline bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
-                              uint64_t d2, uint64_t pitch1_elems, uint64_t pitch2_elems,
-                              uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle swizzle) {
+// 3-D view [d2][d1][d0] of 16-bit elements (element strides: 1, pitch1,
+// pitch2; the strides need not grow with the dimension), box [b2][b1][b0].
+inline bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType type, const void* base,
+                         uint64_t d0, uint64_t d1, uint64_t d2, uint64_t pitch1_elems,
+                         uint64_t pitch2_elems, uint32_t b0, uint32_t b1, uint32_t b2,
+                         CUtensorMapSwizzle swizzle) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {pitch1_elems * 2, pitch2_elems * 2};
   cuuint32_t box[3] = {b0, b1, b2};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, type, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// bf16 version; used e.g. for one group's rows of a [tokens][groups][dim] tensor.
+inline bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                              uint64_t d2, uint64_t pitch1_elems, uint64_t pitch2_elems,
+                              uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle swizzle) {
+  return make_tmap_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, d0, d1, d2, pitch1_elems,
+                      pitch2_elems, b0, b1, b2, swizzle);
 }
 
 }  // namespace msa
