@@ -19,13 +19,15 @@
 // ln rowsum) goes to slot (t, g, r, head); the merge kernel combines the <= k
 // slots of a query with log-sum-exp weights.
 //
-// Warp roles (608 threads, one CTA per SM, persistent over units):
+// Warp roles (640 threads, one CTA per SM, persistent over units):
 //   warp 0     Q producer: a TMA gather of each hitting token's H/G
 //              contiguous query rows into a 2-stage ring;
 //   warp 18    K/V loader: TMA of K_j / V_j (3-D map: one group's rows) once
 //              per unit, plus an L2 prefetch of the next unit's blocks;
-//   warp 1     MMA issuer (one thread): issues whichever of the next S or the
-//              oldest pending PV has its inputs ready;
+//   warp 1     S issuer (one thread): S MMAs of all tiles in order;
+//   warp 19    PV issuer (one thread): PV MMAs of all tiles in order.  Two
+//              issuing threads on different schedulers keep the tensor pipe
+//              fed: one thread issuing both would be busy most of the time;
 //   warps 2-17 two softmax + epilogue groups of 8 warps taking alternate
 //              tiles; a tile row is split between two warps of its group
 //              (TMEM lane = row, 64 columns each).  The epilogue stages the
@@ -42,9 +44,10 @@
 namespace msa {
 namespace {
 
-// Q producer, MMA issuer, 2 softmax groups of 8 warps, K/V loader
-constexpr int kThreads = 608;
+// Q producer, S issuer, 2 softmax groups of 8 warps, K/V loader, PV issuer
+constexpr int kThreads = 640;
 constexpr int kKVWarp = 18;
+constexpr int kPVWarp = 19;
 constexpr int kGroupThreads = 256;
 constexpr int kRows = 128;
 constexpr int kKeys = 128;
@@ -338,115 +341,96 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    // One thread keeps two cursors over the same tile sequence, S ahead of
-    // PV, and issues whichever MMA has its inputs ready, so that a late Q
-    // tile or K block does not hold back the PV of a finished softmax.
+    // ---------------- S issuer (one thread) ----------------
+    // S = Q K^T for every tile in order, into S buffer n%2 once the PV of
+    // tile n-2 has released it.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kKeys, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16(kRows, D, false, true);
-      TilePos sc = first_tile(a, n_units), pc = sc;
-      int qs = 0, sb = 0, pb = 0;
-      uint32_t qph = 0, kph = 0, vph = 0;
-      uint32_t sph[2] = {0, 0}, pph[2] = {0, 0};
-      bool k_ready = false, v_ready = false;
-      int64_t s_count = 0, pv_count = 0;
+      TilePos sc = first_tile(a, n_units);
+      int qs = 0, sb = 0;
+      uint32_t qph = 0, kph = 0;
+      uint32_t sph[2] = {0, 0};
       bool committed = false;
       uint64_t* last_bar = nullptr;
       uint32_t last_par = 0;
-      uint64_t idle_since = 0;
-      bool idle = false;
       const uint32_t k_base = smem_u32(sK);
+      while (sc.more) {
+        if (sc.i == 0) {
+          if (!mbar_wait(&bar_k_full, kph, abort_flag, a.err, kDevTimeoutLoad)) break;
+          kph ^= 1;
+        }
+        if (!mbar_wait(&bar_q_full[qs], qph, abort_flag, a.err, kDevTimeoutLoad)) break;
+        if (!mbar_wait(&bar_s_empty[sb], sph[sb] ^ 1, abort_flag, a.err, kDevTimeoutMma)) break;
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(sQ + qs * Cfg::kQBytes);
+        const uint32_t d_tm = tmem + sb * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(q_base + (kk >> 2) * 1024 + (kk & 3) * 32, 16,
+                                              Cfg::kGroupBytes);
+          const uint64_t bd =
+              smem_desc_sw128(k_base + (kk >> 2) * kKeys * 128 + (kk & 3) * 32, 16, 1024);
+          umma_bf16(d_tm, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar_q_empty[qs]);
+        umma_commit(&bar_s_full[sb]);
+        if (sc.i == sc.m.ntiles - 1) umma_commit(&bar_k_empty);
+        committed = true;
+        last_bar = &bar_s_full[sb];
+        last_par = sph[sb];
+        sph[sb] ^= 1;
+        sb ^= 1;
+        if (++qs == kQStages) qs = 0, qph ^= 1;
+        next_tile(sc, a, n_units);
+      }
+      if (*abort_flag && committed) {
+        volatile int no_abort = 0;
+        mbar_wait(last_bar, last_par, &no_abort, nullptr, 0);
+      }
+    }
+  } else if (warp == kPVWarp) {
+    // ---------------- PV issuer (one thread) ----------------
+    // O = P V for every tile in order: A = P from the tile's S/P buffer in
+    // TMEM, B = V_j from shared memory, into O buffer n%2 once the epilogue
+    // of tile n-2 has read it.
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = idesc_bf16(kRows, D, false, true);
+      TilePos pc = first_tile(a, n_units);
+      int pb = 0;
+      uint32_t vph = 0;
+      uint32_t pph[2] = {0, 0};
+      bool committed = false;
+      uint64_t* last_bar = nullptr;
+      uint32_t last_par = 0;
       const uint32_t v_base = smem_u32(sV);
       while (pc.more) {
-        bool progress = false;
-        // ---- S = Q K^T for the next tile ----
-        if (sc.more) {
-          bool ready = true;
-          if (sc.i == 0 && !k_ready) {
-            ready = mbar_probe(&bar_k_full, kph);
-            if (ready) kph ^= 1, k_ready = true;
-          }
-          ready = ready && mbar_probe(&bar_q_full[qs], qph) &&
-                  mbar_probe(&bar_s_empty[sb], sph[sb] ^ 1);
-          if (ready) {
-            tc_fence_after();
-            const uint32_t q_base = smem_u32(sQ + qs * Cfg::kQBytes);
-            const uint32_t d_tm = tmem + sb * 128;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t ad = smem_desc_sw128(q_base + (kk >> 2) * 1024 + (kk & 3) * 32, 16,
-                                                  Cfg::kGroupBytes);
-              const uint64_t bd =
-                  smem_desc_sw128(k_base + (kk >> 2) * kKeys * 128 + (kk & 3) * 32, 16, 1024);
-              umma_bf16(d_tm, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(&bar_q_empty[qs]);
-            umma_commit(&bar_s_full[sb]);
-            if (sc.i == sc.m.ntiles - 1) {
-              umma_commit(&bar_k_empty);
-              k_ready = false;
-            }
-            committed = true;
-            last_bar = &bar_s_full[sb];
-            last_par = sph[sb];
-            sph[sb] ^= 1;
-            sb ^= 1;
-            if (++qs == kQStages) qs = 0, qph ^= 1;
-            ++s_count;
-            next_tile(sc, a, n_units);
-            progress = true;
-          }
+        if (pc.i == 0) {
+          if (!mbar_wait(&bar_v_full, vph, abort_flag, a.err, kDevTimeoutLoad)) break;
+          vph ^= 1;
         }
-        // ---- O = P V for the oldest tile whose S has been issued ----
-        if (pv_count < s_count) {
-          bool ready = true;
-          if (pc.i == 0 && !v_ready) {
-            ready = mbar_probe(&bar_v_full, vph);
-            if (ready) vph ^= 1, v_ready = true;
-          }
-          // S/P buffer pb and O buffer pb are used in lockstep: one phase each
-          ready = ready && mbar_probe(&bar_p_full[pb], pph[pb]) &&
-                  mbar_probe(&bar_o_empty[pb], pph[pb] ^ 1);
-          if (ready) {
-            tc_fence_after();
-            const uint32_t d_tm = tmem + 256 + pb * 128;
-#pragma unroll
-            for (int kk = 0; kk < kKeys / 16; ++kk) {
-              // keys 16kk..16kk+15: written by column half kk/4 as 8 packed
-              // columns at offset 8*(kk%4) of that half's S columns
-              const uint32_t a_tm = tmem + pb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
-              const uint64_t bd = smem_desc_sw128(v_base + kk * 16 * 128, kKeys * 128, 1024);
-              umma_bf16_ts(d_tm, a_tm, bd, idesc_o, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(&bar_s_empty[pb]);  // P read: the S/P buffer is free
-            umma_commit(&bar_o_full[pb]);
-            if (pc.i == pc.m.ntiles - 1) {
-              umma_commit(&bar_v_empty);
-              v_ready = false;
-            }
-            committed = true;
-            last_bar = &bar_o_full[pb];
-            last_par = pph[pb];
-            pph[pb] ^= 1;
-            pb ^= 1;
-            ++pv_count;
-            next_tile(pc, a, n_units);
-            progress = true;
-          }
-        }
-        if (progress) {
-          idle = false;
-        } else if (!idle) {
-          idle = true;
-          idle_since = global_timer_ns();
-        } else if (*abort_flag) {
+        // S/P buffer pb and O buffer pb are used in lockstep: one phase each
+        if (!mbar_wait(&bar_p_full[pb], pph[pb], abort_flag, a.err, kDevTimeoutConsumer)) break;
+        if (!mbar_wait(&bar_o_empty[pb], pph[pb] ^ 1, abort_flag, a.err, kDevTimeoutConsumer))
           break;
-        } else if (global_timer_ns() - idle_since > kWaitLimitNs) {
-          *abort_flag = 1;
-          record_error(a.err, kDevTimeoutConsumer);
-          break;
+        tc_fence_after();
+        const uint32_t d_tm = tmem + 256 + pb * 128;
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          // keys 16kk..16kk+15: written by column half kk/4 as 8 packed
+          // columns at offset 8*(kk%4) of that half's S columns
+          const uint32_t a_tm = tmem + pb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+          const uint64_t bd = smem_desc_sw128(v_base + kk * 16 * 128, kKeys * 128, 1024);
+          umma_bf16_ts(d_tm, a_tm, bd, idesc_o, kk > 0 ? 1u : 0u);
         }
+        umma_commit(&bar_s_empty[pb]);  // P read: the S/P buffer is free
+        umma_commit(&bar_o_full[pb]);
+        if (pc.i == pc.m.ntiles - 1) umma_commit(&bar_v_empty);
+        committed = true;
+        last_bar = &bar_o_full[pb];
+        last_par = pph[pb];
+        pph[pb] ^= 1;
+        pb ^= 1;
+        next_tile(pc, a, n_units);
       }
       if (*abort_flag && committed) {
         volatile int no_abort = 0;
