@@ -442,15 +442,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Group grp (warps 2+8grp .. 9+8grp) owns the tiles of parity grp, with S/P
     // buffer grp and O buffer grp.  Each row of a tile is split between two
     // warps of the group (same TMEM lane quarter, column half hc), which
-    // combine their row max and row sum through shared memory.
+    // combine their row max and row sum through shared memory.  Warp w reaches
+    // TMEM lane quarter w%4, so warps 2+8grp+i (hc = 0) and 6+8grp+i (hc = 1)
+    // hold the same quarter (2+i)%4.
     //
     // The epilogue of a tile runs one group iteration late, after the softmax
     // of the group's next tile: its PV product then completes while the group
     // works on that softmax instead of being waited for.
     const int grp = (warp - 2) >> 3;
     const int hc = ((warp - 2) & 7) >> 2;  // column half: S/P columns 64hc..64hc+63
-    const uint32_t bar_id = 1 + grp;       // named barrier of this group (256 threads)
     const int quarter = warp & 3;
+    // The two warps of a lane quarter (hc = 0, 1) share their 32 rows: the
+    // max and sum exchanges and the staging of a row group's partials only
+    // couple this pair, so they synchronise with a 64-thread named barrier.
+    const uint32_t bar_id = 1 + grp * 4 + quarter;
     const int row = quarter * 32 + lane;
     const int ts = row >> a.log2slot;
     const int hh = row & (slot - 1);
@@ -513,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_async_smem();
-      named_barrier(bar_id, 256);
+      named_barrier(bar_id, 64);
       if (pend_valid && hc == 0) {
         a.part_lse[pend_slot + hh] = pend_lse;
         if ((hh & 7) == 0) {
@@ -539,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_wait_read<0>();
           store_pending = false;
         }
-        named_barrier(bar_id, 256);
+        named_barrier(bar_id, 64);
         if (!epilogue()) ok = false;
         break;
       }
@@ -596,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_wait_read<0>();
         store_pending = false;
       }
-      named_barrier(bar_id, 256);
+      named_barrier(bar_id, 64);
       float mx = fmaxf(xchg_max[grp][0][row], xchg_max[grp][1][row]);
       if (!(row_valid && good) || !(mx > -INFINITY)) mx = 0.f;
       const float mxs = mx * a.scale_log2;
@@ -627,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       f2_unpack(acc_a, la0, la1);
       f2_unpack(acc_b, lb0, lb1);
       xchg_sum[grp][hc][row] = (la0 + la1) + (lb0 + lb1);
-      named_barrier(bar_id, 256);
+      named_barrier(bar_id, 64);
       const float l = xchg_sum[grp][0][row] + xchg_sum[grp][1][row];
 
       // ---- epilogue of the group's previous tile ----
