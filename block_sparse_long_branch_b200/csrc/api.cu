@@ -116,13 +116,25 @@ int64_t prefill_chunk(const msa_config_t* cfg, int64_t N, size_t ws_bytes, bool 
   return lo * kBlock;
 }
 
-// decode workspace: header | ids | pooled block scores (the rest)
-size_t decode_fixed_bytes(const msa_config_t* c, int32_t B, size_t* off_ids) {
+// decode workspace: header | split tickets | ids | split partials | pooled
+// block scores (the rest).  The header and the tickets are zeroed by one
+// memset per call.
+struct DecodeLayout {
+  size_t tickets, ids, part, fixed;
+};
+DecodeLayout decode_layout(const msa_config_t* c, int32_t B) {
   const int64_t G = c->num_groups, k = c->top_k;
+  DecodeLayout l;
   size_t off = kHeader;
-  *off_ids = off;
+  l.tickets = off;
+  off += align256((size_t)B * G * 4);
+  l.ids = off;
   off += align256((size_t)B * G * k * 4);
-  return off;
+  l.part = off;
+  off += align256((size_t)B * G * kDecodeMaxSplit *
+                  decode_partial_floats(c->num_heads, c->num_groups, c->head_dim) * 4);
+  l.fixed = off;
+  return l;
 }
 
 template <typename T>
@@ -177,8 +189,7 @@ msa_status_t msa_workspace_size(const msa_config_t* cfg, msa_op_t op, int64_t n_
     // total cache rows over all sequences; only per-sequence lengths are bounded
     if (n_tokens < 1 || batch < 1 || batch > n_tokens || n_tokens >= (int64_t(1) << 40))
       return MSA_ERR_INVALID_ARG;
-    size_t a;
-    *bytes = decode_fixed_bytes(cfg, batch, &a) +
+    *bytes = decode_layout(cfg, batch).fixed +
              decode_pooled_rows(n_tokens, batch) * cfg->num_groups * sizeof(float);
     return MSA_OK;
   }
@@ -432,12 +443,13 @@ msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_id
     return MSA_ERR_INVALID_ARG;
   if ((st = check_tokens(cfg, max_seqlen)) != MSA_OK) return st;
   if (!ws || !aligned16(ws)) return MSA_ERR_WORKSPACE;
-  size_t off_ids;
-  const size_t fixed = decode_fixed_bytes(cfg, B, &off_ids);
+  const DecodeLayout lay = decode_layout(cfg, B);
+  const size_t fixed = lay.fixed;
   const size_t row_bytes = (size_t)cfg->num_groups * sizeof(float);
   if (ws_bytes < fixed + row_bytes * (size_t)(B + 1)) return MSA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  // error word and split tickets
+  if (cudaMemsetAsync(ws, 0, lay.ids, s) != cudaSuccess) return MSA_ERR_CUDA;
   DecodeLaunch p{};
   p.q = q;
   p.q_idx = q_idx;
@@ -454,11 +466,19 @@ msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_id
   p.max_seqlen = max_seqlen;
   p.scale = cfg->softmax_scale;
   p.out = out;
-  p.ids = ids_out ? ids_out : at<int32_t>(ws, off_ids);
+  p.ids = ids_out ? ids_out : at<int32_t>(ws, lay.ids);
   p.pooled = at<float>(ws, fixed);
   p.pooled_cap = (int64_t)((ws_bytes - fixed) / row_bytes);
   p.err = at<uint32_t>(ws, 0);
   p.num_sms = sm_count();
+  // enough CTAs for about three per SM, at most kDecodeMaxSplit per (b, g)
+  {
+    const int64_t pairs = (int64_t)B * cfg->num_groups;
+    const int64_t want = (3 * (int64_t)p.num_sms) / pairs;
+    p.n_split = (int32_t)(want < 1 ? 1 : (want > kDecodeMaxSplit ? kDecodeMaxSplit : want));
+  }
+  p.part = at<float>(ws, lay.part);
+  p.tickets = at<int32_t>(ws, lay.tickets);
   p.events = g_events;
   p.n_events = g_n_events;
   int launches = 0;

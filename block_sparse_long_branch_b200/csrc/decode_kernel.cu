@@ -9,7 +9,8 @@
 //      mma.sync m16n8k16 (keys as M, groups as N).  The reduction axis is
 //      permuted identically for both operands so that every lane reads 16
 //      contiguous bytes of a key row straight from global memory.
-//      Writes the pooled (max) score of every non-local block.
+//      Writes the pooled (max) score of every non-local block, [G][nb] per
+//      sequence so that each group's scores are contiguous.
 //   2. decode_topk_kernel  : per (sequence, group), the best k-1 non-local
 //      blocks under (score desc, id asc), plus the local block, ascending.
 //   3. decode_attn_kernel  : per (sequence, group, slot), softmax of the
@@ -113,8 +114,8 @@ __global__ void __launch_bounds__(kIdxWarps * 32)
       }
       if (gq == 0) {
         const int g0 = nt * 8 + 2 * tq;
-        if (g0 < G) pout[j * G + g0] = m0;
-        if (g0 + 1 < G) pout[j * G + g0 + 1] = m1;
+        if (g0 < G) pout[(int64_t)g0 * nb + j] = m0;
+        if (g0 + 1 < G) pout[(int64_t)(g0 + 1) * nb + j] = m1;
       }
     }
   }
@@ -159,19 +160,32 @@ __device__ __forceinline__ bool better(float sa, int32_t ia, float sb, int32_t i
 
 constexpr int kAttnThreads = 256;
 constexpr int kAttnWarps = kAttnThreads / 32;
+constexpr int kCandCap = 256;  // candidates kept for the exact ranking step
 
-template <int D, int NT>
+template <int D, int NT, int KSEL>
 struct AttnSmem {
-  __nv_bfloat16 v[2][kBlock * D];       // V tiles, 16-byte chunks swizzled by key
+  union {
+    __nv_bfloat16 v[2][kBlock * D];  // attention: V tiles, 16-byte chunks swizzled by key
+    struct {                         // selection scratch (done before the first V copy)
+      float wl_s[kAttnWarps][KSEL];  // each warp's best candidates, best first
+      int32_t wl_i[kAttnWarps][KSEL];
+      float tm_s[kAttnThreads];      // each warp's best thread bests
+      int32_t tm_i[kAttnThreads];
+      float cand_s[kCandCap];        // candidates not worse than the threshold
+      int32_t cand_i[kCandCap];
+    };
+  };
   __nv_bfloat16 p[NT * 8][kBlock + 8];  // P (heads x keys), padded rows
   float red_m[kAttnWarps][NT * 8];
   float red_l[kAttnWarps][NT * 8];
   float m_run[NT * 8], l_run[NT * 8], alpha[NT * 8];
   float o_t[NT * 8][D + 4];             // final O (heads x d) for coalesced stores
-  float ws_s[kAttnWarps];
-  int32_t ws_i[kAttnWarps];
-  int32_t sel[32];
-  int32_t nsel;
+  int32_t pick[32];  // the best non-local blocks, best first
+  int32_t sel[32];   // all selected blocks, ascending
+  int32_t mine[32];  // the selected blocks this CTA attends to
+  float thr_s;
+  int32_t thr_i, ncand;
+  int32_t nsel, nmine, last;
 };
 
 // smem offset (elements) of 16-byte chunk c of key row s in a swizzled V tile
@@ -187,11 +201,16 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t& r0, uint32_t& r1, ui
                : "r"(smem_u32(p)));
 }
 
-// One CTA per (group g, sequence b):
+// n_split CTAs per (group g, sequence b), split z taking the selected blocks
+// z, z + n_split, ...:
 //   1. top-k over the pooled scores of the sequence's non-local blocks
-//      (register lists per thread, then k-1 rounds of a block arg-max);
-//   2. attention of the group's H/G heads over the selected blocks with an
-//      online softmax across blocks.  S^T = K Q^T on mma.sync (K rows read
+//      (register lists per thread, then k-1 rounds of a block arg-max); every
+//      split computes the same selection;
+//   2. attention of the group's H/G heads over this split's blocks with an
+//      online softmax across blocks;
+//   3. with several splits, each writes its unnormalised O and (max, sum) to
+//      the workspace and the last split to finish (a ticket per (b, g)) merges
+//      them with log-sum-exp weights.  S^T = K Q^T on mma.sync (K rows read
 //      straight from global memory with the permuted reduction axis, Q in
 //      registers), P to shared memory, O^T += V^T P^T on mma.sync with V in a
 //      swizzled shared tile (ldmatrix.trans).  The next block's V is copied in
@@ -202,65 +221,183 @@ __global__ void __launch_bounds__(kAttnThreads)
                          const __nv_bfloat16* __restrict__ vc, const int64_t* __restrict__ cu,
                          const float* __restrict__ pooled, int64_t pooled_cap, int32_t G,
                          int32_t HG, int32_t top_k, float scale_log2,
-                         int32_t* __restrict__ ids_out, __nv_bfloat16* __restrict__ out) {
+                         int32_t* __restrict__ ids_out, __nv_bfloat16* __restrict__ out,
+                         int32_t n_split, float* __restrict__ part, int32_t* __restrict__ tickets) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  AttnSmem<D, NT>& sm = *reinterpret_cast<AttnSmem<D, NT>*>(smem_raw);
-  const int g = blockIdx.x, b = blockIdx.y;
+  AttnSmem<D, NT, KSEL>& sm = *reinterpret_cast<AttnSmem<D, NT, KSEL>*>(smem_raw);
+  const int g = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t s0 = cu[b];
   const int64_t L = cu[b + 1] - s0;
   const int64_t nb = (L + kBlock - 1) / kBlock;
 
   // ---------------- 1. selection ----------------
+  // The best `want` non-local blocks under (score desc, id asc), a strict
+  // total order:
+  //  (a) each thread finds its best candidate (j = tid + 256 i);
+  //  (b) each warp takes the best R = ceil(want/8) of its threads' bests
+  //      (R rounds of a warp arg-max), and thr = the want-th best of those
+  //      8R distinct candidates.  Every one of the best `want` is then not
+  //      worse than thr;
+  //  (c) every candidate not worse than thr is collected (usually a few more
+  //      than `want`) and ranked exactly by counting.
+  // If more than kCandCap candidates pass (heavy ties), per-thread lists and
+  // warp tournaments are used instead.  Finally the picks and the local block
+  // are put in ascending id order, again by counting.
   {
     const int64_t n_cand = (pooled_offset(cu, b) + nb > pooled_cap) ? 0 : nb - 1;
-    const float* ps = pooled + pooled_offset(cu, b) * G + g;
-    TopList<KSEL> list;
-    list.init();
-    for (int64_t j = tid; j < n_cand; j += kAttnThreads) list.insert(ps[j * G], (int32_t)j);
+    const float* ps = pooled + pooled_offset(cu, b) * G + (int64_t)g * nb;  // [G][nb] per sequence
     const int want = (int)min64(top_k - 1, n_cand);
-    for (int round = 0; round < want; ++round) {
-      float sc = list.sc[0];
-      int32_t id = list.id[0];
+    constexpr int kBatch = 8;
+    float best_s = -INFINITY;
+    int32_t best_i = 0x7FFFFFFF;
+    for (int64_t j0 = tid; j0 < n_cand; j0 += kBatch * kAttnThreads) {
+      float v[kBatch];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float s2 = __shfl_xor_sync(0xffffffffu, sc, o);
-        const int32_t i2 = __shfl_xor_sync(0xffffffffu, id, o);
-        if (better(s2, i2, sc, id)) sc = s2, id = i2;
+      for (int c = 0; c < kBatch; ++c) {
+        const int64_t j = j0 + (int64_t)c * kAttnThreads;
+        v[c] = j < n_cand ? __ldg(ps + j) : -INFINITY;
       }
-      if (lane == 0) sm.ws_s[warp] = sc, sm.ws_i[warp] = id;
-      __syncthreads();
-      float bs = sm.ws_s[0];
-      int32_t bi = sm.ws_i[0];
 #pragma unroll
-      for (int w = 1; w < kAttnWarps; ++w)
-        if (better(sm.ws_s[w], sm.ws_i[w], bs, bi)) bs = sm.ws_s[w], bi = sm.ws_i[w];
-      if (list.id[0] == bi) list.pop();  // ids are unique: exactly one owner pops
-      if (tid == 0) sm.sel[round] = bi;
-      __syncthreads();
+      for (int c = 0; c < kBatch; ++c) {
+        const int64_t j = j0 + (int64_t)c * kAttnThreads;
+        if (j < n_cand && better(v[c], (int32_t)j, best_s, best_i)) best_s = v[c], best_i = (int32_t)j;
+      }
+    }
+    // (b) per warp: its best R thread bests into tm[warp * R + round]
+    const int R = (want + kAttnWarps - 1) / kAttnWarps;
+    {
+      float ms = best_s;
+      int32_t mi = best_i;
+      for (int round = 0; round < R; ++round) {
+        float sc = ms;
+        int32_t id = mi;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float s2 = __shfl_xor_sync(0xffffffffu, sc, o);
+          const int32_t i2 = __shfl_xor_sync(0xffffffffu, id, o);
+          if (better(s2, i2, sc, id)) sc = s2, id = i2;
+        }
+        if (mi == id) ms = -INFINITY, mi = 0x7FFFFFFF;  // the owner drops it
+        if (lane == 0) sm.tm_s[warp * R + round] = sc, sm.tm_i[warp * R + round] = id;
+      }
     }
     if (tid == 0) {
-      // ascending: insertion of the local block (largest id) into sorted picks
-      int n = want;
-      for (int x = 1; x < n; ++x)
-        for (int y = x; y > 0 && sm.sel[y - 1] > sm.sel[y]; --y) {
-          const int32_t t = sm.sel[y];
-          sm.sel[y] = sm.sel[y - 1];
-          sm.sel[y - 1] = t;
+      sm.ncand = 0;
+      // the worst possible key: kept if fewer than `want` of the 8R are real
+      // candidates, and then every candidate is collected
+      sm.thr_s = -INFINITY;
+      sm.thr_i = 0x7FFFFFFF;
+    }
+    __syncthreads();
+    if (warp == 0 && want > 0) {
+      // thr = the want-th best of the 8R collected (lane x ranks entry x)
+      for (int x = lane; x < kAttnWarps * R; x += 32) {
+        const float sx = sm.tm_s[x];
+        const int32_t ix = sm.tm_i[x];
+        int rank = 0;
+        for (int y = 0; y < kAttnWarps * R; ++y) rank += better(sm.tm_s[y], sm.tm_i[y], sx, ix);
+        if (rank == want - 1) sm.thr_s = sx, sm.thr_i = ix;
+      }
+    }
+    __syncthreads();
+    // (c) collect the candidates not worse than thr
+    if (want > 0) {
+      const float ts = sm.thr_s;
+      const int32_t ti = sm.thr_i;
+      for (int64_t j0 = tid; j0 < n_cand; j0 += kBatch * kAttnThreads) {
+        float v[kBatch];
+#pragma unroll
+        for (int c = 0; c < kBatch; ++c) {
+          const int64_t j = j0 + (int64_t)c * kAttnThreads;
+          v[c] = j < n_cand ? __ldg(ps + j) : -INFINITY;
         }
-      sm.sel[n++] = (int32_t)(nb - 1);
-      sm.nsel = n;
-      int32_t* dst = ids_out + ((int64_t)b * G + g) * top_k;
-      for (int r = 0; r < top_k; ++r) dst[r] = r < n ? sm.sel[r] : -1;
+#pragma unroll
+        for (int c = 0; c < kBatch; ++c) {
+          const int64_t j = j0 + (int64_t)c * kAttnThreads;
+          if (j < n_cand && !better(ts, ti, v[c], (int32_t)j)) {
+            const int x = atomicAdd(&sm.ncand, 1);
+            if (x < kCandCap) sm.cand_s[x] = v[c], sm.cand_i[x] = (int32_t)j;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    const int nc = sm.ncand;
+    if (nc <= kCandCap) {
+      // exact ranks among the collected: the best `want` go to pick[0..want)
+      for (int x = tid; x < nc; x += kAttnThreads) {
+        const float s_x = sm.cand_s[x];
+        const int32_t i_x = sm.cand_i[x];
+        int rank = 0;
+        for (int y = 0; y < nc; ++y) rank += better(sm.cand_s[y], sm.cand_i[y], s_x, i_x);
+        if (rank < want) sm.pick[rank] = i_x;
+      }
+    } else {
+      // fallback: per-thread lists, then warp tournaments
+      TopList<KSEL> list;
+      list.init();
+      for (int64_t j = tid; j < n_cand; j += kAttnThreads) list.insert(__ldg(ps + j), (int32_t)j);
+      for (int round = 0; round < want; ++round) {
+        float sc = list.sc[0];
+        int32_t id = list.id[0];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float s2 = __shfl_xor_sync(0xffffffffu, sc, o);
+          const int32_t i2 = __shfl_xor_sync(0xffffffffu, id, o);
+          if (better(s2, i2, sc, id)) sc = s2, id = i2;
+        }
+        if (list.id[0] == id) list.pop();  // real ids are unique; empty heads pop harmlessly
+        if (lane == 0) sm.wl_s[warp][round] = sc, sm.wl_i[warp][round] = id;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        TopList<KSEL> wl;
+        wl.init();
+#pragma unroll
+        for (int i = 0; i < KSEL; ++i)
+          if (lane < kAttnWarps && i < want) wl.sc[i] = sm.wl_s[lane][i], wl.id[i] = sm.wl_i[lane][i];
+        for (int round = 0; round < want; ++round) {
+          float sc = wl.sc[0];
+          int32_t id = wl.id[0];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const float s2 = __shfl_xor_sync(0xffffffffu, sc, o);
+            const int32_t i2 = __shfl_xor_sync(0xffffffffu, id, o);
+            if (better(s2, i2, sc, id)) sc = s2, id = i2;
+          }
+          if (wl.id[0] == id) wl.pop();
+          if (lane == 0) sm.pick[round] = id;
+        }
+      }
+    }
+    __syncthreads();
+    // ascending ids: the picks by counting, then the local block (the largest)
+    const int n = want + 1;
+    if (tid < want) {
+      const int32_t my = sm.pick[tid];
+      int pos = 0;
+      for (int y = 0; y < want; ++y) pos += sm.pick[y] < my;
+      sm.sel[pos] = my;
+    } else if (tid == want) {
+      sm.sel[want] = (int32_t)(nb - 1);
     }
     if (tid < NT * 8) sm.m_run[tid] = -INFINITY, sm.l_run[tid] = 0.f;
+    __syncthreads();
+    if (tid < n && tid % n_split == split) sm.mine[tid / n_split] = sm.sel[tid];
+    if (split == 0 && tid < top_k)
+      ids_out[((int64_t)b * G + g) * top_k + tid] = tid < n ? sm.sel[tid] : -1;
+    if (tid == 0) {
+      sm.nsel = n;
+      sm.nmine = n > split ? (n - split - 1) / n_split + 1 : 0;
+    }
     __syncthreads();
   }
 
   // ---------------- 2. attention ----------------
   constexpr int WPR = D / 8;  // 32-bit words per lane per row (permuted reduction axis)
   const int gq = lane >> 2, tq = lane & 3;
-  const int nsel = sm.nsel;
+  const int nsel = sm.nmine;
   const __nv_bfloat16* kbase = kc + (s0 * G + g) * (int64_t)D;
   const __nv_bfloat16* vbase = vc + (s0 * G + g) * (int64_t)D;
   const int64_t row_pitch = (int64_t)G * D;
@@ -286,7 +423,7 @@ __global__ void __launch_bounds__(kAttnThreads)
   }
 
   auto load_v = [&](int bi, int buf) {
-    const int64_t j = sm.sel[bi];
+    const int64_t j = sm.mine[bi];
     const int nk = (int)min64(kBlock, L - j * kBlock);
     for (int x = tid; x < kBlock * (D / 8); x += kAttnThreads) {
       const int s = x / (D / 8), c = x % (D / 8);
@@ -303,7 +440,7 @@ __global__ void __launch_bounds__(kAttnThreads)
   // this warp's 16 key rows of a block, lanes reading 16 contiguous bytes each
   uint32_t w0[WPR], w1[WPR];
   auto load_k = [&](int bi) {
-    const int64_t jj = sm.sel[bi];
+    const int64_t jj = sm.mine[bi];
     const int nkk = (int)min64(kBlock, L - jj * kBlock);
     const int r0i = warp * 16 + gq, r1i = r0i + 8;
     const uint4* r0 = reinterpret_cast<const uint4*>(
@@ -324,7 +461,7 @@ __global__ void __launch_bounds__(kAttnThreads)
   }
   for (int bi = 0; bi < nsel; ++bi) {
     const int buf = bi & 1;
-    const int64_t j = sm.sel[bi];
+    const int64_t j = sm.mine[bi];
     const int nk = (int)min64(kBlock, L - j * kBlock);
     if (bi + 1 < nsel) load_v(bi + 1, buf ^ 1);
 
@@ -427,7 +564,7 @@ __global__ void __launch_bounds__(kAttnThreads)
     __syncthreads();  // p, red_*, alpha and this V buffer are reused next block
   }
 
-  // ---------------- output: O / l -> bf16 [heads][d] ----------------
+  // ---------------- output ----------------
   if (warp < D / 16) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -440,30 +577,80 @@ __global__ void __launch_bounds__(kAttnThreads)
     }
   }
   __syncthreads();
+  __nv_bfloat16* orow = out + ((int64_t)b * G * HG + g * HG) * D;
+  if (n_split == 1) {
+    // O / l -> bf16 [heads][d]
+    for (int x = tid; x < HG * (D / 8); x += kAttnThreads) {
+      const int h = x / (D / 8), c = x % (D / 8);
+      const float inv = sm.l_run[h] > 0.f ? 1.0f / sm.l_run[h] : 0.f;
+      uint4 w;
+      w.x = pack_bf16x2(sm.o_t[h][c * 8 + 0] * inv, sm.o_t[h][c * 8 + 1] * inv);
+      w.y = pack_bf16x2(sm.o_t[h][c * 8 + 2] * inv, sm.o_t[h][c * 8 + 3] * inv);
+      w.z = pack_bf16x2(sm.o_t[h][c * 8 + 4] * inv, sm.o_t[h][c * 8 + 5] * inv);
+      w.w = pack_bf16x2(sm.o_t[h][c * 8 + 6] * inv, sm.o_t[h][c * 8 + 7] * inv);
+      reinterpret_cast<uint4*>(orow + (int64_t)h * D)[c] = w;
+    }
+    return;
+  }
+  // this split's partial: O [NT*8][D] (unnormalised), then max and sum (log2 domain)
+  constexpr int kPart = NT * 8 * (D + 2);
+  const int64_t pg = (int64_t)b * G + g;
+  float* mypart = part + (pg * n_split + split) * kPart;
+  for (int x = tid; x < NT * 8 * (D / 4); x += kAttnThreads) {
+    const int h = x / (D / 4), c = x % (D / 4);
+    reinterpret_cast<float4*>(mypart + h * D)[c] =
+        make_float4(sm.o_t[h][4 * c], sm.o_t[h][4 * c + 1], sm.o_t[h][4 * c + 2],
+                    sm.o_t[h][4 * c + 3]);
+  }
+  if (tid < NT * 8) {
+    mypart[NT * 8 * D + tid] = sm.m_run[tid];
+    mypart[NT * 8 * D + NT * 8 + tid] = sm.l_run[tid];
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sm.last = atomicAdd(tickets + pg, 1) == n_split - 1;
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
+  // last split: out = sum_z 2^(m_z - M) O_z / sum_z 2^(m_z - M) l_z
+  const float* gpart = part + pg * n_split * kPart;
   for (int x = tid; x < HG * (D / 8); x += kAttnThreads) {
     const int h = x / (D / 8), c = x % (D / 8);
-    const float inv = sm.l_run[h] > 0.f ? 1.0f / sm.l_run[h] : 0.f;
+    float M = -INFINITY;
+    for (int z = 0; z < n_split; ++z) M = fmaxf(M, __ldcg(gpart + z * kPart + NT * 8 * D + h));
+    float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int z = 0; z < n_split; ++z) {
+      const float* pz = gpart + z * kPart;
+      const float mz = __ldcg(pz + NT * 8 * D + h);
+      const float wz = mz == -INFINITY ? 0.f : fast_exp2(mz - M);
+      L += wz * __ldcg(pz + NT * 8 * D + NT * 8 + h);
+      const float4 a = __ldcg(reinterpret_cast<const float4*>(pz + h * D + c * 8));
+      const float4 e = __ldcg(reinterpret_cast<const float4*>(pz + h * D + c * 8 + 4));
+      acc[0] += wz * a.x, acc[1] += wz * a.y, acc[2] += wz * a.z, acc[3] += wz * a.w;
+      acc[4] += wz * e.x, acc[5] += wz * e.y, acc[6] += wz * e.z, acc[7] += wz * e.w;
+    }
+    const float inv = L > 0.f ? 1.0f / L : 0.f;
     uint4 w;
-    w.x = pack_bf16x2(sm.o_t[h][c * 8 + 0] * inv, sm.o_t[h][c * 8 + 1] * inv);
-    w.y = pack_bf16x2(sm.o_t[h][c * 8 + 2] * inv, sm.o_t[h][c * 8 + 3] * inv);
-    w.z = pack_bf16x2(sm.o_t[h][c * 8 + 4] * inv, sm.o_t[h][c * 8 + 5] * inv);
-    w.w = pack_bf16x2(sm.o_t[h][c * 8 + 6] * inv, sm.o_t[h][c * 8 + 7] * inv);
-    reinterpret_cast<uint4*>(out + ((int64_t)b * G * HG + g * HG + h) * D)[c] = w;
+    w.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    w.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    w.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+    w.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+    reinterpret_cast<uint4*>(orow + (int64_t)h * D)[c] = w;
   }
 }
 
 template <int D, int NT, int KSEL>
 cudaError_t launch_attend(const DecodeLaunch& p, cudaStream_t s) {
   auto kern = decode_attend_kernel<D, NT, KSEL>;
-  const int smem = (int)sizeof(AttnSmem<D, NT>);
+  const int smem = (int)sizeof(AttnSmem<D, NT, KSEL>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)p.G, (unsigned)p.B);
+  dim3 grid((unsigned)p.G, (unsigned)p.B, (unsigned)p.n_split);
   kern<<<grid, kAttnThreads, smem, s>>>(
       static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k_cache),
       static_cast<const __nv_bfloat16*>(p.v_cache), p.cu_seqlens, p.pooled, p.pooled_cap, p.G,
       p.H / p.G, p.top_k, p.scale * 1.4426950408889634f, p.ids,
-      static_cast<__nv_bfloat16*>(p.out));
+      static_cast<__nv_bfloat16*>(p.out), p.n_split, p.part, p.tickets);
   return cudaGetLastError();
 }
 
@@ -482,6 +669,12 @@ cudaError_t launch_attend_d(const DecodeLaunch& p, cudaStream_t s) {
 }
 
 }  // namespace
+
+size_t decode_partial_floats(int32_t H, int32_t G, int32_t d) {
+  const int HG = H / G;
+  const int heads = HG <= 8 ? 8 : 16;  // NT * 8
+  return (size_t)heads * (d + 2);
+}
 
 size_t decode_pooled_rows(int64_t total_len, int32_t B) {
   return (size_t)(total_len / kBlock + B + 1);

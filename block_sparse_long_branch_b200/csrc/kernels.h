@@ -90,14 +90,20 @@ struct DecodeLaunch {
   float scale;
   void* out;       // [B][H][d] bf16
   int32_t* ids;    // [B][G][top_k]
-  float* pooled;   // [pooled_cap][G]
+  float* pooled;   // pooled_cap rows of G: sequence b owns rows from cu[b]/128 + b, as [G][nb_b]
   int64_t pooled_cap;
+  int32_t n_split;   // CTAs per (sequence, group) in the attention step
+  float* part;       // [B][G][n_split][partial]: split partials (n_split > 1)
+  int32_t* tickets;  // [B][G], zero at launch: arrivals of the splits
   uint32_t* err;
   int num_sms;
   void* const* events;  // optional phase events (msa_set_phase_events)
   int n_events;
 };
 size_t decode_pooled_rows(int64_t total_len, int32_t B);
+// floats of one split partial of the decode attention: [heads][d] + max + sum
+size_t decode_partial_floats(int32_t H, int32_t G, int32_t d);
+constexpr int kDecodeMaxSplit = 4;
 cudaError_t launch_decode(const DecodeLaunch& p, cudaStream_t s, int* launches);
 
 }  // namespace msa

@@ -113,3 +113,41 @@ def test_decode_full_config_every_query(msa):
     inp = synth.make_decode_inputs(s, device="cuda")
     n_ties = _check(msa, s, inp)
     assert n_ties <= 8
+
+
+def test_decode_all_scores_tied(msa):
+    """Every index key zero: all pooled scores tie at 0, so the lowest block ids win
+    (ties go to the lower id), plus the local block."""
+    s = synth.DecodeShape("dtie", seq_lens=(128 * 600 + 17, 128 * 40), H=16, G=2, d=64,
+                          d_idx=64, top_k=16, seed=14)
+    inp = synth.make_decode_inputs(s, device="cuda")
+    inp["k_idx_cache"].zero_()
+    g_out, g_ids = _run(msa, s, inp)
+    for b, L in enumerate(s.seq_lens):
+        nb = (L + s.block - 1) // s.block
+        want = list(range(min(s.top_k - 1, nb - 1))) + [nb - 1]
+        want += [-1] * (s.top_k - len(want))
+        for g in range(s.G):
+            assert g_ids[b, g].tolist() == want, (b, g)
+        ids, pooled, out, _ = _oracle_one(inp, s, b)
+        assert (ids == np.asarray(want)[None, :]).all()
+        parity.check_output(g_out[b], out)
+
+
+def test_decode_clustered_high_scores(msa):
+    """The high-scoring blocks all fall on the candidates of one warp of the
+    selection (block ids j with j mod 256 < 32), so the threshold taken from
+    per-warp bests is weak and the exhaustive per-thread-list path decides."""
+    s = synth.DecodeShape("dclu", seq_lens=(128 * 2048, 128 * 300), H=16, G=2, d=64, d_idx=128,
+                          top_k=16, seed=15)
+    inp = synth.make_decode_inputs(s, device="cuda")
+    kic = inp["k_idx_cache"]
+    cu = inp["cu_seqlens"].tolist()
+    for b in range(s.B):
+        u = inp["q_idx"][b, 0].double() + inp["q_idx"][b, 1].double()
+        nb = (s.seq_lens[b] + s.block - 1) // s.block
+        for j in range(nb - 1):
+            if j % 256 < 32:
+                r0 = cu[b] + j * s.block
+                kic[r0:r0 + s.block] = (u * (1.0 + 1e-3 * j)).to(torch.bfloat16)
+    _check(msa, s, inp)
