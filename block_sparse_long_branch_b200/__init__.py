@@ -25,6 +25,7 @@ __all__ = [
     "msa_index_scores", "msa_select_topk",
     "msa_build_block_query_lists", "msa_prefill", "msa_decode", "msa_get_device_error",
     "msa_status_string", "msa_last_launch_count", "msa_set_phase_events", "msa_decode_static",
+    "msa_selftest_wait_timeout",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -97,6 +98,7 @@ def load_library():
     lib.msa_decode.argtypes = [C, P, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
     lib.msa_decode_static.argtypes = [C, P, P, P, P, P, P, I32, I64, I64, P, P, I32, P]
     lib.msa_get_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.msa_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
     lib.msa_status_string.argtypes = [ctypes.c_int]
     lib.msa_status_string.restype = ctypes.c_char_p
     lib.msa_set_phase_events.argtypes = [P, I32]
@@ -106,7 +108,7 @@ def load_library():
     for name in ("msa_workspace_size", "msa_prefill_min_workspace", "msa_prefill_chunk_tokens",
                  "msa_index_scores",
                  "msa_select_topk", "msa_build_block_query_lists", "msa_prefill", "msa_decode",
-                 "msa_decode_static", "msa_get_device_error"):
+                 "msa_decode_static", "msa_get_device_error", "msa_selftest_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -360,6 +362,14 @@ def msa_set_phase_events(events) -> None:
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _phase_keep = (arr, events)
     _check(lib.msa_set_phase_events(arr, len(events)), "msa_set_phase_events")
+
+
+def msa_selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int, stream=None) -> None:
+    """Launch the planted-timeout self-test (see include/msa.h); read the result
+    with msa_get_device_error."""
+    _check(load_library().msa_selftest_wait_timeout(_dev(workspace, torch.uint8, "workspace"),
+                                                    int(limit_ns), _stream(stream)),
+           "msa_selftest_wait_timeout")
 
 
 def msa_get_device_error(workspace: torch.Tensor, stream=None) -> int:

@@ -21,6 +21,7 @@ enum DeviceError : uint32_t {
   kDevTimeoutLoad = 0x101,     // a TMA / bulk-copy completion never arrived
   kDevTimeoutMma = 0x102,      // a tensor-core commit never arrived
   kDevTimeoutConsumer = 0x103, // an epilogue/softmax hand-off never arrived
+  kDevSelfTest = 0x1FE,        // msa_selftest_wait_timeout: the planted wait ran out
   kDevBadIndex = 0x201,        // an id or list entry outside its range
 };
 
@@ -89,8 +90,9 @@ __device__ __forceinline__ bool mbar_probe(uint64_t* bar, uint32_t parity) {
 // if the CTA-wide abort flag is raised (by this or another thread) or the
 // time limit passes; in the latter case the abort flag and the error word are
 // set.  `abort_flag` lives in shared memory.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* err, uint32_t code) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, uint32_t* err,
+                                              uint32_t code, uint64_t limit_ns) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_test(addr, parity)) return true;
   const uint64_t t0 = global_timer_ns();
@@ -98,12 +100,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_test(addr, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) break;
+      if (global_timer_ns() - t0 > limit_ns) break;
     }
   }
   *abort_flag = 1;
   record_error(err, code);
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* err, uint32_t code) {
+  return mbar_wait_for(bar, parity, abort_flag, err, code, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------------------

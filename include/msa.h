@@ -229,6 +229,20 @@ MSA_API msa_status_t msa_decode_static(const msa_config_t* cfg, const void* q, c
  */
 MSA_API msa_status_t msa_get_device_error(void* ws, msa_stream_t stream, uint32_t* code);
 
+/*
+ * Self-test of the kernels' failure path; the pages have no counterpart.
+ * Launches one CTA that waits, with the same bounded mbarrier wait every
+ * kernel of this library uses, on a barrier that nothing ever arrives on.
+ * After `limit_ns` (device %globaltimer; 1000 .. 10^9) the wait gives up,
+ * records 0x1FE in the device error word of `ws` and the kernel returns, so
+ * the context stays usable.  Read the result with msa_get_device_error, which
+ * then returns MSA_ERR_DEVICE_TIMEOUT with *code = 0x1FE.
+ *   ws: device workspace of at least 256 bytes (its error word is cleared
+ *       first).  Returns MSA_ERR_INVALID_ARG for a null/misaligned ws or a
+ *       limit out of range, MSA_ERR_CUDA if the launch fails.
+ */
+MSA_API msa_status_t msa_selftest_wait_timeout(void* ws, uint64_t limit_ns, msa_stream_t stream);
+
 /* Static description of a status code. */
 MSA_API const char* msa_status_string(msa_status_t status);
 

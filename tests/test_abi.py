@@ -115,3 +115,12 @@ def test_missing_workspace_rejected():
 def test_status_strings():
     for s in range(7):
         assert msa.msa_status_string(s)
+
+
+def test_selftest_arguments_checked_before_any_launch():
+    lib = msa.load_library()
+    p = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced: rejected first
+    assert lib.msa_selftest_wait_timeout(None, 10_000, None) == 1
+    assert lib.msa_selftest_wait_timeout(ctypes.c_void_p((1 << 20) + 4), 10_000, None) == 1
+    assert lib.msa_selftest_wait_timeout(p, 999, None) == 1
+    assert lib.msa_selftest_wait_timeout(p, 10 ** 9 + 1, None) == 1
