@@ -197,6 +197,13 @@ def barrier(world: int):
         dist.barrier()
 
 
+def replica_rate(units_per_rank: float, ms_local: float, world: int):
+    """Whole-job rate of `world` replicas that each processed `units_per_rank`
+    units: the total over the slowest rank's time (max over ranks)."""
+    ms = reduce_max(ms_local, world)
+    return world * units_per_rank / (ms * 1e-3), ms
+
+
 # --------------------------------------------------------------------------
 # CPU oracle timing (the baseline arm)
 # --------------------------------------------------------------------------
@@ -407,7 +414,7 @@ def run_ours(args, rank, world, local):
         # per step, per phase: summed over the chunks of the query axis
         pre_ph = np.array([[sum(e[5 * c + ph].elapsed_time(e[5 * c + ph + 1])
                                 for c in range(chunks_run)) for ph in range(4)] for e in pev])
-        pre_ms = reduce_max(float(pre_ph.sum(axis=1).mean()), world)
+        value, pre_ms = replica_rate(N, float(pre_ph.sum(axis=1).mean()), world)
         ids_np = ids.cpu().numpy()
         pw = prefill_work(ids_np, shape.H, shape.d, shape.block)
         idx_f = index_flops(N, shape.G, shape.d_idx, shape.block)
@@ -418,7 +425,6 @@ def run_ours(args, rank, world, local):
                                                    (kernels["main_branch"]["ms"] * 1e-3) / 1e12)
         kernels["main_branch"]["tensor_frac"] = kernels["main_branch"]["tensor_tflops"] / tc_peak
         add("merge", pre_ph[:, 3], "hbm", pw["merge_bytes"], True)
-        value = world * N / (pre_ms * 1e-3)
         prefill_obj = {"value": value, "unit": "tokens/s", "ms_per_step": pre_ms,
                        "query_chunks": chunks_run, "dense_flops": dense_flops(N, shape.H, shape.d),
                        "msa_flops": idx_f + pw["main_flops"],
@@ -426,12 +432,12 @@ def run_ours(args, rank, world, local):
     decode_obj = None
     if dec is not None:
         dec_ph = np.array([_phase_ms(e, 2) for e in dev_ev])
-        dec_ms = reduce_max(float(dec_ph.sum(axis=1).mean()), world)
+        dec_rate, dec_ms = replica_rate(dc.B, float(dec_ph.sum(axis=1).mean()), world)
         dw = decode_work(dc.seq_lens, dc.H, dc.G, dc.d, dc.d_idx, dids.cpu().numpy(), dc.block)
         add("decode_index", dec_ph[:, 0], "hbm", dw["idx_bytes"], True)
         add("decode_select_attend", dec_ph[:, 1], "hbm", dw["attn_bytes"], True)
         dstep_bytes = dw["bytes"]
-        decode_obj = {"value": world * dc.B / (dec_ms * 1e-3), "unit": "tokens/s",
+        decode_obj = {"value": dec_rate, "unit": "tokens/s",
                       "ms_per_step": dec_ms,
                       "hbm_frac": dstep_bytes / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                       "bytes_per_step": dstep_bytes}
@@ -618,7 +624,7 @@ def _e2e_decode(args, msa, dec, dcfg, dws, dev, world):
             "ms_per_step": dms}
 
 
-def main(argv=None):
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -641,6 +647,11 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
+    return args
+
+
+def main(argv=None):
+    args = parse_args(argv)
     rank, world, local = dist_setup(init_group=args.impl == "ours")
     if args.gpus != world and world > 1:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
