@@ -194,3 +194,57 @@ def test_prefill_32k_sampled_rows(msa):
     # properties that hold at every row: the forced local block and the budget
     parity.check_id_rows_valid(ids, np.arange(s.N), s.block, s.top_k)
     assert torch.isfinite(out.float()).all()
+
+
+def _check_sampled_large(msa, s, n_rows, ws_bytes, seed):
+    """Prefill of a long workload in the benchmark's launch configuration
+    (chunked query axis when the workspace is capped), checked on sampled rows
+    against the oracle; only the sampled rows' queries leave the device."""
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    ws = torch.empty(max(ws_bytes, msa.msa_prefill_min_workspace(cfg, s.N)), dtype=torch.uint8,
+                     device="cuda")
+    out, ids = msa.msa_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                               ids_out=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_error(ws) == 0
+    needle_rows = [t for (_, _, t) in inp["needles"]][:24]
+    rows = synth.sample_rows(s.N, n_rows, seed=seed, extra=needle_rows)
+    rows_dev = torch.from_numpy(rows).cuda()
+    nb = s.nb
+    qi = oracle.as_bf16_bits(inp["q_idx"][rows_dev])
+    pooled = oracle.pooled_scores(qi, rows, inp["k_idx"], s.block, nb)
+    ref_ids = oracle.select_blocks(pooled, rows, s.block, s.top_k)
+    g_ids = ids[rows_dev].cpu().numpy()
+    parity.check_id_rows_valid(g_ids, rows, s.block, s.top_k)
+    ties = parity.compare_ids(g_ids, ref_ids, pooled, rows, s.block, s.top_k)
+    # Main Branch of the oracle on the GPU's selection (equal to the oracle's
+    # own except at listed near-ties)
+    sel = g_ids if ties else ref_ids
+    qr = oracle.as_bf16_bits(inp["q"][rows_dev])
+    ref_out = oracle.block_attention(qr, rows, inp["k"], inp["v"], sel, s.scale, s.block)
+    parity.check_output(out[rows_dev].float().cpu().numpy(), ref_out)
+    # every needle's query selected its block
+    ids_np = ids.cpu().numpy()
+    for (j, g, t) in inp["needles"]:
+        assert j in ids_np[t, g], (j, g, t)
+    return len(ties)
+
+
+@pytest.mark.slow
+def test_prefill_128k_sampled_rows(msa):
+    """128K tokens, one pass over the query axis, 64 sampled rows plus needles."""
+    s = synth.PREFILL_CONFIGS["prefill_128k"]
+    n_ties = _check_sampled_large(msa, s, 64, 96 << 30, seed=7)
+    assert n_ties <= 8
+
+
+@pytest.mark.slow
+def test_prefill_1m_sampled_rows_chunked(msa):
+    """1M tokens with a 40 GiB workspace: the query axis runs in chunks, as in
+    the benchmark; 48 sampled rows plus needles."""
+    s = synth.PREFILL_CONFIGS["prefill_1m"]
+    cfg = _cfg(msa, s)
+    assert msa.msa_prefill_chunk_tokens(cfg, s.N, 40 << 30) < s.N
+    n_ties = _check_sampled_large(msa, s, 48, 40 << 30, seed=8)
+    assert n_ties <= 8
