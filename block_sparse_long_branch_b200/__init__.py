@@ -25,7 +25,7 @@ __all__ = [
     "msa_index_scores", "msa_select_topk",
     "msa_build_block_query_lists", "msa_prefill", "msa_decode", "msa_get_device_error",
     "msa_status_string", "msa_last_launch_count", "msa_set_phase_events", "msa_decode_static",
-    "msa_selftest_wait_timeout",
+    "msa_selftest_wait_timeout", "msa_prefill_varlen",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -95,6 +95,7 @@ def load_library():
     lib.msa_select_topk.argtypes = [C, P, P, I64, P, P, SZ, P]
     lib.msa_build_block_query_lists.argtypes = [C, P, I64, P, P, P, SZ, P]
     lib.msa_prefill.argtypes = [C, P, P, P, P, P, I64, P, P, P, SZ, P]
+    lib.msa_prefill_varlen.argtypes = [C, P, P, P, P, P, P, I32, P, P, P, SZ, P]
     lib.msa_decode.argtypes = [C, P, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
     lib.msa_decode_static.argtypes = [C, P, P, P, P, P, P, I32, I64, I64, P, P, I32, P]
     lib.msa_get_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
@@ -107,7 +108,8 @@ def load_library():
     lib.msa_last_launch_count.restype = I32
     for name in ("msa_workspace_size", "msa_prefill_min_workspace", "msa_prefill_chunk_tokens",
                  "msa_index_scores",
-                 "msa_select_topk", "msa_build_block_query_lists", "msa_prefill", "msa_decode",
+                 "msa_select_topk", "msa_build_block_query_lists", "msa_prefill",
+                 "msa_prefill_varlen", "msa_decode",
                  "msa_decode_static", "msa_get_device_error", "msa_selftest_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -257,6 +259,40 @@ def msa_prefill(cfg: MsaConfig, q, k, v, q_idx, k_idx, out: Optional[torch.Tenso
                          _dev(out, torch.bfloat16, "out", (N, H, d)), ids_ptr,
                          _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(st, "msa_prefill")
+    return out if ids_out is None else (out, ids_out)
+
+
+def msa_prefill_varlen(cfg: MsaConfig, q, k, v, q_idx, k_idx, cu_seqlens,
+                       out: Optional[torch.Tensor] = None, ids_out=None,
+                       workspace: Optional[torch.Tensor] = None, stream=None):
+    """Prefill of sequences packed along the token axis (host ``cu_seqlens``,
+    any int sequence of B+1 offsets).  Returns ``out`` or ``(out, ids)``."""
+    lib = load_library()
+    import numpy as _np
+    cu = _np.ascontiguousarray(_np.asarray(
+        cu_seqlens.cpu() if isinstance(cu_seqlens, torch.Tensor) else cu_seqlens,
+        dtype=_np.int64))
+    B = len(cu) - 1
+    T = q.shape[0]
+    H, G, d, di, kk = cfg.num_heads, cfg.num_groups, cfg.head_dim, cfg.index_dim, cfg.top_k
+    if B < 1 or int(cu[-1]) != T:
+        raise ValueError(f"cu_seqlens must end at the packed length {T}")
+    if out is None:
+        out = torch.empty((T, H, d), dtype=torch.bfloat16, device=q.device)
+    if ids_out is True:
+        ids_out = torch.empty((T, G, kk), dtype=torch.int32, device=q.device)
+    max_len = int(_np.max(_np.diff(cu)))
+    ws = _workspace(workspace, msa_workspace_size(cfg, OP_PREFILL, max(max_len, 1)), q.device)
+    ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (T, G, kk))
+    st = lib.msa_prefill_varlen(ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (T, H, d)),
+                                _dev(k, torch.bfloat16, "k", (T, G, d)),
+                                _dev(v, torch.bfloat16, "v", (T, G, d)),
+                                _dev(q_idx, torch.bfloat16, "q_idx", (T, G, di)),
+                                _dev(k_idx, torch.bfloat16, "k_idx", (T, di)),
+                                cu.ctypes.data_as(ctypes.c_void_p), B,
+                                _dev(out, torch.bfloat16, "out", (T, H, d)), ids_ptr,
+                                _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(st, "msa_prefill_varlen")
     return out if ids_out is None else (out, ids_out)
 
 

@@ -320,24 +320,25 @@ msa_status_t msa_build_block_query_lists(const msa_config_t* cfg, const int32_t*
   return st;
 }
 
-msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, const void* v,
+}  // extern "C"
+
+namespace {
+
+// One causal prefill of N tokens whose arguments were validated: index ->
+// lists -> Main Branch -> merge per chunk of the query axis.  The workspace's
+// error word is not cleared here.  Phase events are recorded when `events`.
+msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, const void* v,
                          const void* q_idx, const void* k_idx, int64_t N, void* out,
-                         int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream) {
-  g_launches = 0;
-  msa_status_t st = check_cfg(cfg);
-  if (st != MSA_OK) return st;
-  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
-  if (!q || !k || !v || !q_idx || !k_idx || !out) return MSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_idx) || !aligned16(k_idx) ||
-      !aligned16(out) || (ids_out && !aligned16(ids_out)))
-    return MSA_ERR_INVALID_ARG;
-  if (!ws || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+                         int32_t* ids_out, void* ws, size_t ws_bytes, cudaStream_t s,
+                         bool events, int* launches_out) {
   const int64_t nb = n_blocks(N);
+  (void)nb;
   const bool own_ids = ids_out == nullptr;
   const int64_t chunk = prefill_chunk(cfg, N, ws_bytes, own_ids);
   if (chunk == 0) return MSA_ERR_WORKSPACE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  auto mark = [&](int i, cudaStream_t st) {
+    if (events) ::mark(i, st);
+  };
   const int G = cfg->num_groups, H = cfg->num_heads, d = cfg->head_dim, kk = cfg->top_k;
   const int sms = sm_count();
   uint32_t* err = at<uint32_t>(ws, 0);
@@ -423,6 +424,86 @@ msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, 
     if (launch_merge(gp, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
     ++launches;
     mark(ev + 4, s);
+  }
+  *launches_out += launches;
+  return MSA_OK;
+}
+
+msa_status_t check_prefill_ptrs(const void* q, const void* k, const void* v, const void* q_idx,
+                                const void* k_idx, const void* out, const int32_t* ids_out,
+                                const void* ws) {
+  if (!q || !k || !v || !q_idx || !k_idx || !out) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_idx) || !aligned16(k_idx) ||
+      !aligned16(out) || (ids_out && !aligned16(ids_out)))
+    return MSA_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  return MSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, const void* v,
+                         const void* q_idx, const void* k_idx, int64_t N, void* out,
+                         int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  if ((st = check_prefill_ptrs(q, k, v, q_idx, k_idx, out, ids_out, ws)) != MSA_OK) return st;
+  if (prefill_chunk(cfg, N, ws_bytes, ids_out == nullptr) == 0) return MSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  int launches = 0;
+  st = prefill_run(cfg, q, k, v, q_idx, k_idx, N, out, ids_out, ws, ws_bytes, s, true, &launches);
+  g_launches = launches;
+  return st;
+}
+
+msa_status_t msa_prefill_varlen(const msa_config_t* cfg, const void* q, const void* k,
+                                const void* v, const void* q_idx, const void* k_idx,
+                                const int64_t* cu_seqlens, int32_t B, void* out,
+                                int32_t* ids_out, void* ws, size_t ws_bytes,
+                                msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if (!cu_seqlens || B < 1 || cu_seqlens[0] != 0) return MSA_ERR_INVALID_ARG;
+  int64_t max_len = 0;
+  const int64_t ids_row_bytes = (int64_t)cfg->num_groups * cfg->top_k * 4;
+  for (int32_t b = 0; b < B; ++b) {
+    const int64_t L = cu_seqlens[b + 1] - cu_seqlens[b];
+    if (L < 0) return MSA_ERR_INVALID_ARG;
+    if (L > max_len) max_len = L;
+    // every sequence's rows of ids_out must start 16-byte aligned
+    if (ids_out && L > 0 && (cu_seqlens[b] * ids_row_bytes) % 16 != 0)
+      return MSA_ERR_UNSUPPORTED;
+  }
+  if (max_len == 0) return MSA_ERR_INVALID_ARG;
+  if ((st = check_tokens(cfg, max_len)) != MSA_OK) return st;
+  if ((st = check_prefill_ptrs(q, k, v, q_idx, k_idx, out, ids_out, ws)) != MSA_OK) return st;
+  // every sequence fits the workspace if the longest does
+  if (prefill_chunk(cfg, max_len, ws_bytes, ids_out == nullptr) == 0) return MSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  const int64_t H = cfg->num_heads, G = cfg->num_groups, d = cfg->head_dim;
+  const int64_t di = cfg->index_dim, kk = cfg->top_k;
+  int launches = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    const int64_t r0 = cu_seqlens[b], L = cu_seqlens[b + 1] - r0;
+    if (L == 0) continue;
+    // the sequence's rows of every packed tensor (16-byte aligned: rows are
+    // whole multiples of 16 bytes for the supported shapes)
+    const auto* qb = static_cast<const uint8_t*>(q) + r0 * H * d * 2;
+    const auto* kb = static_cast<const uint8_t*>(k) + r0 * G * d * 2;
+    const auto* vb = static_cast<const uint8_t*>(v) + r0 * G * d * 2;
+    const auto* qib = static_cast<const uint8_t*>(q_idx) + r0 * G * di * 2;
+    const auto* kib = static_cast<const uint8_t*>(k_idx) + r0 * di * 2;
+    auto* ob = static_cast<uint8_t*>(out) + r0 * H * d * 2;
+    int32_t* idb = ids_out ? ids_out + r0 * G * kk : nullptr;
+    st = prefill_run(cfg, qb, kb, vb, qib, kib, L, ob, idb, ws, ws_bytes, s, false, &launches);
+    if (st != MSA_OK) return st;
   }
   g_launches = launches;
   return MSA_OK;

@@ -177,6 +177,30 @@ MSA_API msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const v
                          int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream);
 
 /*
+ * Prefill of B independent sequences packed along the token axis (no
+ * attention across sequences); each is the causal prefill msa_prefill
+ * computes.  The pages serve MSA to batched requests but describe no batched
+ * kernel; this entry point runs the same kernels once per sequence, in
+ * order, on `stream` and `ws`.
+ *   q [T][H][d], k/v [T][G][d], q_idx [T][G][d_idx], k_idx [T][d_idx] bf16,
+ *     T = cu_seqlens[B]; sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1
+ *     and its token i is position i of that sequence.
+ *   cu_seqlens [B+1] int64, HOST pointer: cu_seqlens[0] = 0, non-decreasing,
+ *     at least one non-empty sequence; empty sequences are skipped.
+ *   out [T][H][d] bf16 out; ids_out [T][G][k] int32 out, nullable (ids are
+ *     block numbers within the token's own sequence; every sequence's rows
+ *     must start 16-byte aligned, else MSA_ERR_UNSUPPORTED).
+ *   ws: at least msa_prefill_min_workspace() for the longest sequence; every
+ *     sequence then runs in query chunks that fit, as in msa_prefill.
+ * Phase events (msa_set_phase_events) are not recorded by this call.
+ */
+MSA_API msa_status_t msa_prefill_varlen(const msa_config_t* cfg, const void* q, const void* k,
+                                        const void* v, const void* q_idx, const void* k_idx,
+                                        const int64_t* cu_seqlens, int32_t B, void* out,
+                                        int32_t* ids_out, void* ws, size_t ws_bytes,
+                                        msa_stream_t stream);
+
+/*
  * One decode step for B sequences.  The pages give decode speed-ups only
  * (zhaixingw M3 review, section "这套注意力到底怎么省的"); the plainest reading,
  * used here, is the same two branches for the newest query row, which sits at

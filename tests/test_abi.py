@@ -124,3 +124,20 @@ def test_selftest_arguments_checked_before_any_launch():
     assert lib.msa_selftest_wait_timeout(ctypes.c_void_p((1 << 20) + 4), 10_000, None) == 1
     assert lib.msa_selftest_wait_timeout(p, 999, None) == 1
     assert lib.msa_selftest_wait_timeout(p, 10 ** 9 + 1, None) == 1
+
+
+def test_varlen_offsets_checked_before_any_launch():
+    lib = msa.load_library()
+    cfg = _cfg()
+    p = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 21)
+
+    def call(cu):
+        arr = (ctypes.c_int64 * len(cu))(*cu)
+        return lib.msa_prefill_varlen(ctypes.byref(cfg), p, p, p, p, p, arr, len(cu) - 1, p, None,
+                                      ws, 1 << 30, None)
+    assert call([1, 5]) == 1        # must start at 0
+    assert call([0, 5, 3]) == 1     # decreasing offsets
+    assert call([0, 0, 0]) == 1     # nothing to do
+    assert lib.msa_prefill_varlen(ctypes.byref(cfg), p, p, p, p, p, None, 1, p, None, ws, 1 << 30,
+                                  None) == 1

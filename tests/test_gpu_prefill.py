@@ -249,3 +249,55 @@ def test_prefill_1m_sampled_rows_chunked(msa):
     assert msa.msa_prefill_chunk_tokens(cfg, s.N, 40 << 30) < s.N
     n_ties = _check_sampled_large(msa, s, 2048, 40 << 30, seed=8)
     assert n_ties <= 64
+
+
+def test_prefill_varlen_matches_per_sequence_oracle(msa):
+    """Packed sequences of mixed lengths (one empty, one of a single token):
+    each must equal its own causal prefill, ids counted within the sequence."""
+    lens = [700, 0, 4096 + 5, 128, 1, 2049]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    s = synth.PrefillShape("varlen", N=int(cu[-1]), H=16, G=2, d=128, d_idx=64, top_k=8,
+                           n_needles=6, seed=41)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    out, ids = msa.msa_prefill_varlen(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"],
+                                      inp["k_idx"], cu, ids_out=True)
+    torch.cuda.synchronize()
+    assert msa.msa_last_launch_count() > 0
+    for b, L in enumerate(lens):
+        if L == 0:
+            continue
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        ref = oracle.prefill(inp["q"][s0:s1], inp["k"][s0:s1], inp["v"][s0:s1],
+                             inp["q_idx"][s0:s1], inp["k_idx"][s0:s1], block=s.block,
+                             top_k=s.top_k, scale=s.scale)
+        rows = np.arange(L)
+        g_ids = ids[s0:s1].cpu().numpy()
+        parity.check_id_rows_valid(g_ids, rows, s.block, s.top_k)
+        ties = parity.compare_ids(g_ids, ref["ids"], ref["pooled"], rows, s.block, s.top_k)
+        ref_out = ref["out"]
+        if ties:
+            ref_out = oracle.block_attention(oracle.as_bf16_bits(inp["q"][s0:s1]), rows,
+                                             inp["k"][s0:s1], inp["v"][s0:s1], g_ids, s.scale,
+                                             s.block)
+        parity.check_output(out[s0:s1].float().cpu().numpy(), ref_out)
+
+
+def test_prefill_varlen_small_workspace_chunks_each_sequence(msa):
+    """With the minimum workspace every sequence runs in query chunks; the
+    result equals the one-shot call bit for bit."""
+    lens = [3000, 5000]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    s = synth.PrefillShape("varlen2", N=int(cu[-1]), H=8, G=2, d=64, d_idx=64, top_k=4, seed=42)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    full = msa.msa_prefill_varlen(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                                  cu)
+    ws = torch.empty(msa.msa_prefill_min_workspace(cfg, max(lens)), dtype=torch.uint8,
+                     device="cuda")
+    assert msa.msa_prefill_chunk_tokens(cfg, max(lens), ws.numel(), ids_returned=False) < max(lens)
+    small = msa.msa_prefill_varlen(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"],
+                                   inp["k_idx"], cu, workspace=ws)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_error(ws) == 0
+    assert torch.equal(full, small)
