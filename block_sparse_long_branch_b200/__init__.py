@@ -25,7 +25,7 @@ __all__ = [
     "msa_index_scores", "msa_select_topk",
     "msa_build_block_query_lists", "msa_prefill", "msa_decode", "msa_get_device_error",
     "msa_status_string", "msa_last_launch_count", "msa_set_phase_events", "msa_decode_static",
-    "msa_selftest_wait_timeout", "msa_prefill_varlen",
+    "msa_selftest_wait_timeout", "msa_prefill_varlen", "msa_prefill_block_alignment",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -96,6 +96,7 @@ def load_library():
     lib.msa_build_block_query_lists.argtypes = [C, P, I64, P, P, P, SZ, P]
     lib.msa_prefill.argtypes = [C, P, P, P, P, P, I64, P, P, P, SZ, P]
     lib.msa_prefill_varlen.argtypes = [C, P, P, P, P, P, P, I32, P, P, P, SZ, P]
+    lib.msa_prefill_block_alignment.argtypes = [C, P, P, P, P, P, I64, P, P, P, P, P, P, SZ, P]
     lib.msa_decode.argtypes = [C, P, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
     lib.msa_decode_static.argtypes = [C, P, P, P, P, P, P, I32, I64, I64, P, P, I32, P]
     lib.msa_get_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
@@ -109,7 +110,7 @@ def load_library():
     for name in ("msa_workspace_size", "msa_prefill_min_workspace", "msa_prefill_chunk_tokens",
                  "msa_index_scores",
                  "msa_select_topk", "msa_build_block_query_lists", "msa_prefill",
-                 "msa_prefill_varlen", "msa_decode",
+                 "msa_prefill_varlen", "msa_prefill_block_alignment", "msa_decode",
                  "msa_decode_static", "msa_get_device_error", "msa_selftest_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -260,6 +261,33 @@ def msa_prefill(cfg: MsaConfig, q, k, v, q_idx, k_idx, out: Optional[torch.Tenso
                          _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(st, "msa_prefill")
     return out if ids_out is None else (out, ids_out)
+
+
+def msa_prefill_block_alignment(cfg: MsaConfig, q, k, v, q_idx, k_idx,
+                                workspace: Optional[torch.Tensor] = None, stream=None):
+    """Prefill plus the KL-alignment data (see include/msa.h).
+
+    Returns ``(out, ids, block_score, block_mass, kl)``.
+    """
+    lib = load_library()
+    N = q.shape[0]
+    H, G, d, di, kk = cfg.num_heads, cfg.num_groups, cfg.head_dim, cfg.index_dim, cfg.top_k
+    dev = q.device
+    out = torch.empty((N, H, d), dtype=torch.bfloat16, device=dev)
+    ids = torch.empty((N, G, kk), dtype=torch.int32, device=dev)
+    score = torch.empty((N, G, kk), dtype=torch.float32, device=dev)
+    mass = torch.empty((N, G, kk), dtype=torch.float32, device=dev)
+    kl = torch.empty((N, G), dtype=torch.float32, device=dev)
+    ws = _workspace(workspace, msa_workspace_size(cfg, OP_PREFILL, N), dev)
+    st = lib.msa_prefill_block_alignment(
+        ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (N, H, d)),
+        _dev(k, torch.bfloat16, "k", (N, G, d)), _dev(v, torch.bfloat16, "v", (N, G, d)),
+        _dev(q_idx, torch.bfloat16, "q_idx", (N, G, di)), _dev(k_idx, torch.bfloat16, "k_idx", (N, di)),
+        N, _dev(out, torch.bfloat16, "out"), _dev(ids, torch.int32, "ids"),
+        _dev(score, torch.float32, "block_score"), _dev(mass, torch.float32, "block_mass"),
+        _dev(kl, torch.float32, "kl"), _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(st, "msa_prefill_block_alignment")
+    return out, ids, score, mass, kl
 
 
 def msa_prefill_varlen(cfg: MsaConfig, q, k, v, q_idx, k_idx, cu_seqlens,

@@ -327,10 +327,12 @@ namespace {
 // One causal prefill of N tokens whose arguments were validated: index ->
 // lists -> Main Branch -> merge per chunk of the query axis.  The workspace's
 // error word is not cleared here.  Phase events are recorded when `events`.
+// With block_mass non-null, also the block-alignment outputs (all three).
 msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, const void* v,
                          const void* q_idx, const void* k_idx, int64_t N, void* out,
                          int32_t* ids_out, void* ws, size_t ws_bytes, cudaStream_t s,
-                         bool events, int* launches_out) {
+                         bool events, int* launches_out, float* block_score = nullptr,
+                         float* block_mass = nullptr, float* kl = nullptr) {
   const int64_t nb = n_blocks(N);
   (void)nb;
   const bool own_ids = ids_out == nullptr;
@@ -384,6 +386,24 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
     cp.tile_tokens = main_tile_tokens(H, G);
     cp.unit_tiles = kUnitTiles;
     if (launch_csr(cp, s, &launches) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
+    if (block_mass) {
+      BlockScoreLaunch bp{};
+      bp.q_idx = q_idx;
+      bp.k_idx = k_idx;
+      bp.N = N;
+      bp.G = G;
+      bp.d_idx = cfg->index_dim;
+      bp.top_k = kk;
+      bp.nb = nbc;
+      bp.row_begin = t0;
+      bp.rows = rows;
+      bp.row_ptr = cp.row_ptr;
+      bp.entries = cp.entries;
+      bp.score = block_score + t0 * G * kk;
+      bp.err = err;
+      if (launch_block_scores(bp, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
+      ++launches;
+    }
     mark(ev + 2, s);
 
     MainLaunch mp{};
@@ -421,6 +441,11 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
     gp.d = d;
     gp.top_k = kk;
     gp.out = static_cast<uint8_t*>(out) + (size_t)t0 * H * d * 2;
+    if (block_mass) {
+      gp.block_score = block_score + t0 * G * kk;
+      gp.block_mass = block_mass + t0 * G * kk;
+      gp.kl = kl + t0 * G;
+    }
     if (launch_merge(gp, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
     ++launches;
     mark(ev + 4, s);
@@ -457,6 +482,29 @@ msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, 
   if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
   int launches = 0;
   st = prefill_run(cfg, q, k, v, q_idx, k_idx, N, out, ids_out, ws, ws_bytes, s, true, &launches);
+  g_launches = launches;
+  return st;
+}
+
+msa_status_t msa_prefill_block_alignment(const msa_config_t* cfg, const void* q, const void* k,
+                                         const void* v, const void* q_idx, const void* k_idx,
+                                         int64_t N, void* out, int32_t* ids_out,
+                                         float* block_score, float* block_mass, float* kl,
+                                         void* ws, size_t ws_bytes, msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  if ((st = check_prefill_ptrs(q, k, v, q_idx, k_idx, out, ids_out, ws)) != MSA_OK) return st;
+  if (!block_score || !block_mass || !kl || !aligned16(block_score) || !aligned16(block_mass) ||
+      !aligned16(kl))
+    return MSA_ERR_INVALID_ARG;
+  if (prefill_chunk(cfg, N, ws_bytes, ids_out == nullptr) == 0) return MSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  int launches = 0;
+  st = prefill_run(cfg, q, k, v, q_idx, k_idx, N, out, ids_out, ws, ws_bytes, s, true, &launches,
+                   block_score, block_mass, kl);
   g_launches = launches;
   return st;
 }

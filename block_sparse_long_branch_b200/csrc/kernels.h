@@ -74,8 +74,27 @@ struct MergeLaunch {
   int64_t rows;
   int32_t H, G, d, top_k;
   void* out;  // [rows][H][d] bf16 (already offset to row_begin)
+  // optional block-alignment outputs (all three or none; offset to row_begin):
+  float* block_score;        // in:  [rows][G][top_k] pooled index scores (empty slots
+                             //      are set to -inf here)
+  float* block_mass;         // out: [rows][G][top_k] attention mass, mean over the group's heads
+  float* kl;                 // out: [rows][G] KL(mass || softmax of the scores over the slots)
 };
 cudaError_t launch_merge(const MergeLaunch& p, cudaStream_t s);
+
+// Block-alignment diagnostic: pooled index score of every listed (t, r).
+struct BlockScoreLaunch {
+  const void* q_idx;  // [N][G][d_idx] bf16
+  const void* k_idx;  // [N][d_idx] bf16
+  int64_t N;
+  int32_t G, d_idx, top_k;
+  int64_t nb, row_begin, rows;
+  const int32_t* row_ptr;  // [G*nb+1] lists of the query chunk
+  const int32_t* entries;
+  float* score;  // [rows][G][top_k]; slots without a list entry are not written
+  uint32_t* err;
+};
+cudaError_t launch_block_scores(const BlockScoreLaunch& p, cudaStream_t s);
 
 // ---- decode (decode_kernel.cu) --------------------------------------------
 struct DecodeLaunch {

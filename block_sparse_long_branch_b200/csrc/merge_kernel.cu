@@ -19,11 +19,15 @@ namespace {
 
 constexpr int kWarps = 8;
 
-template <int CPL, int KMAX>
+// ALIGN: also the block-alignment outputs (see MergeLaunch): the attention
+// mass of every slot, averaged over the group's heads, and the KL divergence
+// of that mass from the softmax of the slots' pooled index scores.
+template <int CPL, int KMAX, bool ALIGN>
 __global__ void __launch_bounds__(kWarps * 32)
     merge_kernel(const __half* __restrict__ part_o, const float* __restrict__ part_lse,
                  const int32_t* __restrict__ ids, int64_t rows, int32_t G, int32_t HG, int32_t d,
-                 int32_t top_k, __nv_bfloat16* __restrict__ out) {
+                 int32_t top_k, __nv_bfloat16* __restrict__ out, float* __restrict__ block_score,
+                 float* __restrict__ block_mass, float* __restrict__ kl) {
   const int64_t tg = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (tg >= rows * G) return;
   const int lane = threadIdx.x & 31;
@@ -31,8 +35,9 @@ __global__ void __launch_bounds__(kWarps * 32)
   const uint32_t valid = __ballot_sync(0xffffffffu, idv >= 0);  // bit r: slot r holds a block
   const int chunks = HG * d / 8;
   const int c0 = lane * CPL;
-  if (c0 >= chunks) return;
-  const int h = (c0 * 8) / d;
+  if (!ALIGN && c0 >= chunks) return;
+  const bool active = c0 < chunks;
+  const int h = active ? (c0 * 8) / d : 0;
   const int64_t slot_elems = (int64_t)HG * d;
   const __half* o_tg = part_o + tg * top_k * slot_elems + (int64_t)c0 * 8;
   const float* l_tg = part_lse + tg * top_k * HG + h;
@@ -41,8 +46,49 @@ __global__ void __launch_bounds__(kWarps * 32)
   float m = -INFINITY;
 #pragma unroll
   for (int r = 0; r < KMAX; ++r) {
-    lse[r] = (r < top_k && (valid >> r & 1u)) ? __ldg(l_tg + r * HG) : -INFINITY;
+    lse[r] = (active && r < top_k && (valid >> r & 1u)) ? __ldg(l_tg + r * HG) : -INFINITY;
     m = fmaxf(m, lse[r]);
+  }
+  if (ALIGN) {
+    // per slot: this head's softmax weight; summed over the head leaders
+    // (the first lane of each head) and divided by H/G
+    float ws = 0.f;
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r)
+      if (r < top_k && (valid >> r & 1u)) ws += __expf(lse[r] - m);
+    const bool leader = active && (c0 * 8) % d == 0;
+    float mass[KMAX];
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r) {
+      float w = (leader && r < top_k && (valid >> r & 1u)) ? __expf(lse[r] - m) / ws : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
+      mass[r] = w / (float)HG;
+    }
+    // KL(mass || softmax over the filled slots of their pooled index scores)
+    float smax = -INFINITY;
+    float sc[KMAX];
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r) {
+      sc[r] = (r < top_k && (valid >> r & 1u)) ? block_score[tg * top_k + r] : -INFINITY;
+      smax = fmaxf(smax, sc[r]);
+    }
+    float z = 0.f;
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r)
+      if (r < top_k && (valid >> r & 1u)) z += __expf(sc[r] - smax);
+    const float logz = __logf(z) + smax;
+    float div = 0.f;
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r)
+      if (r < top_k && (valid >> r & 1u) && mass[r] > 0.f)
+        div += mass[r] * (__logf(mass[r]) - (sc[r] - logz));
+    if (lane < top_k) {
+      block_mass[tg * top_k + lane] = (valid >> lane & 1u) ? mass[lane] : 0.f;
+      if (!(valid >> lane & 1u)) block_score[tg * top_k + lane] = -INFINITY;
+    }
+    if (lane == 0) kl[tg] = div;
+    if (!active) return;
   }
   float acc[CPL * 8];
 #pragma unroll
@@ -79,24 +125,24 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
-template <int KMAX>
+template <int KMAX, bool ALIGN>
 cudaError_t launch_k(const MergeLaunch& p, cudaStream_t s, unsigned grid) {
   const int chunks = (p.H / p.G) * p.d / 8;  // 16-byte chunks per slot, a power of two >= 8
   auto* o = static_cast<__nv_bfloat16*>(p.out);
   const int HG = p.H / p.G;
-  if (chunks >= 256) {
-    merge_kernel<8, KMAX><<<grid, kWarps * 32, 0, s>>>(p.part_o, p.part_lse, p.ids, p.rows, p.G,
-                                                        HG, p.d, p.top_k, o);
-  } else if (chunks >= 128) {
-    merge_kernel<4, KMAX><<<grid, kWarps * 32, 0, s>>>(p.part_o, p.part_lse, p.ids, p.rows, p.G,
-                                                        HG, p.d, p.top_k, o);
-  } else if (chunks >= 64) {
-    merge_kernel<2, KMAX><<<grid, kWarps * 32, 0, s>>>(p.part_o, p.part_lse, p.ids, p.rows, p.G,
-                                                        HG, p.d, p.top_k, o);
-  } else {
-    merge_kernel<1, KMAX><<<grid, kWarps * 32, 0, s>>>(p.part_o, p.part_lse, p.ids, p.rows, p.G,
-                                                        HG, p.d, p.top_k, o);
-  }
+#define MSA_MERGE(CPL)                                                                       \
+  merge_kernel<CPL, KMAX, ALIGN><<<grid, kWarps * 32, 0, s>>>(                               \
+      p.part_o, p.part_lse, p.ids, p.rows, p.G, HG, p.d, p.top_k, o, p.block_score,          \
+      p.block_mass, p.kl)
+  if (chunks >= 256)
+    MSA_MERGE(8);
+  else if (chunks >= 128)
+    MSA_MERGE(4);
+  else if (chunks >= 64)
+    MSA_MERGE(2);
+  else
+    MSA_MERGE(1);
+#undef MSA_MERGE
   return cudaGetLastError();
 }
 
@@ -108,8 +154,10 @@ cudaError_t launch_merge(const MergeLaunch& p, cudaStream_t s) {
   const int chunks = (p.H / p.G) * p.d / 8;
   if (chunks > 32 * 8) return cudaErrorInvalidValue;  // H/G * d > 2048: not instantiated
   const unsigned grid = (unsigned)((warps + kWarps - 1) / kWarps);
-  if (p.top_k <= 16) return launch_k<16>(p, s, grid);
-  return launch_k<32>(p, s, grid);
+  const bool align = p.block_mass != nullptr;
+  if (align && (!p.block_score || !p.kl)) return cudaErrorInvalidValue;
+  if (p.top_k <= 16) return align ? launch_k<16, true>(p, s, grid) : launch_k<16, false>(p, s, grid);
+  return align ? launch_k<32, true>(p, s, grid) : launch_k<32, false>(p, s, grid);
 }
 
 }  // namespace msa

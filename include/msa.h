@@ -177,6 +177,32 @@ MSA_API msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const v
                          int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream);
 
 /*
+ * msa_prefill plus the data of the Index Branch's KL alignment, forward only:
+ * the Index Branch is trained to bring its distribution of block scores
+ * close to the distribution of where the Main Branch's exact attention went
+ * (ai-tool-zukan "MiniMax MSA guide", section "選択を学習可能にするKL損失").
+ * The pages do not define the two distributions; the readings used are, per
+ * (token t, group g, slot r) of the selection ids[t][g][r]:
+ *   block_score [N][G][k] fp32 out: the pooled index score of block
+ *     ids[t][g][r] (max over its visible keys of <q_idx[t][g], k_idx[s]>,
+ *     the score the selection ranks by; the forced local block included);
+ *     -inf for an empty slot.
+ *   block_mass  [N][G][k] fp32 out: the share of the Main Branch softmax of
+ *     token t that falls on the keys of that block, averaged over the H/G
+ *     heads of group g (sums to 1 over the slots); 0 for an empty slot.
+ *   kl [N][G] fp32 out: KL(block_mass || softmax over the filled slots of
+ *     block_score), in nats.
+ * Other arguments and the workspace as for msa_prefill.  The default
+ * msa_prefill path does none of this extra work.
+ */
+MSA_API msa_status_t msa_prefill_block_alignment(const msa_config_t* cfg, const void* q,
+                                                 const void* k, const void* v, const void* q_idx,
+                                                 const void* k_idx, int64_t N, void* out,
+                                                 int32_t* ids_out, float* block_score,
+                                                 float* block_mass, float* kl, void* ws,
+                                                 size_t ws_bytes, msa_stream_t stream);
+
+/*
  * Prefill of B independent sequences packed along the token axis (no
  * attention across sequences); each is the causal prefill msa_prefill
  * computes.  The pages serve MSA to batched requests but describe no batched
