@@ -379,35 +379,6 @@ def msa_decode_static(cfg: MsaConfig, q, q_idx, k_cache, v_cache, k_idx_cache, c
     return out if ids_out is None else (out, ids_out)
 
 
-def msa_decode_static(cfg: MsaConfig, q, q_idx, k_cache, v_cache, k_idx_cache, cu_seqlens,
-                      max_seqlen: int, total_len: int, out: Optional[torch.Tensor] = None,
-                      ids_out=None, check_device_error: bool = False, stream=None):
-    """msa_decode with the library's fixed scratch array instead of a workspace.
-
-    For callers that cannot allocate device memory: the library allocates
-    nothing either.  ``out``/``ids_out`` must then be passed in by the caller.
-    """
-    lib = load_library()
-    B = q.shape[0]
-    H, G, d, di, kk = cfg.num_heads, cfg.num_groups, cfg.head_dim, cfg.index_dim, cfg.top_k
-    total = k_cache.shape[0]
-    if out is None:
-        out = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
-    if ids_out is True:
-        ids_out = torch.empty((B, G, kk), dtype=torch.int32, device=q.device)
-    ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (B, G, kk))
-    st = lib.msa_decode_static(ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (B, H, d)),
-                               _dev(q_idx, torch.bfloat16, "q_idx", (B, G, di)),
-                               _dev(k_cache, torch.bfloat16, "k_cache", (total, G, d)),
-                               _dev(v_cache, torch.bfloat16, "v_cache", (total, G, d)),
-                               _dev(k_idx_cache, torch.bfloat16, "k_idx_cache", (total, di)),
-                               _dev(cu_seqlens, torch.int64, "cu_seqlens", (B + 1,)), B,
-                               max_seqlen, total_len, _dev(out, torch.bfloat16, "out", (B, H, d)),
-                               ids_ptr, 1 if check_device_error else 0, _stream(stream))
-    _check(st, "msa_decode_static")
-    return out if ids_out is None else (out, ids_out)
-
-
 _phase_keep = None
 
 
