@@ -62,3 +62,67 @@ def test_two_gloo_ranks_rate_and_reference_arm():
         assert rate == pytest.approx(2 * 1000 / 0.030)
     assert res[0][2] == ("reference", 2, True)
     assert res[1][2] is None
+
+
+def _shard_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank), OMP_NUM_THREADS="2")
+    import torch
+    import torch.distributed as dist
+    import oracle
+    import synth
+    import block_sparse_long_branch_b200 as msa
+    from block_sparse_long_branch_b200 import shard
+    dist.init_process_group("gloo")
+    try:
+        s = synth.PrefillShape("shard", N=640, H=8, G=4, d=64, d_idx=64, top_k=4, n_needles=4,
+                               seed=61)
+        inp = synth.make_prefill_inputs(s, device="cpu")
+        cfg = msa.config(s.H, s.G, s.d, s.d_idx, top_k=s.top_k, scale=s.scale)
+
+        def oracle_slice(c, qq, kk, vv, qi, ki):
+            r = oracle.prefill(qq, kk, vv, qi, ki, block=c.block_size, top_k=c.top_k,
+                               scale=c.softmax_scale)
+            assert qq.shape[1] == c.num_heads and kk.shape[1] == c.num_groups
+            return torch.from_numpy(r["out"]), torch.from_numpy(r["ids"])
+
+        out, ids = shard.head_sharded_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"],
+                                              inp["k_idx"], prefill=oracle_slice)
+        if rank == 0:
+            full = oracle.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                                  block=s.block, top_k=s.top_k, scale=s.scale)
+            same = (torch.equal(out, torch.from_numpy(full["out"])) and
+                    torch.equal(ids, torch.from_numpy(full["ids"])))
+            q.put(("ok", same, tuple(out.shape), tuple(ids.shape)))
+    except Exception as e:  # report instead of hanging the parent
+        q.put(("error", repr(e), None, None))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+def test_head_sharded_prefill_equals_one_rank():
+    """Two gloo ranks, two GQA groups each, the oracle standing in for the
+    per-rank prefill: the gathered output and ids equal the unsharded oracle."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    status, same, oshape, ishape = q.get(timeout=240)
+    for p in procs:
+        p.join(timeout=60)
+    assert status == "ok", same
+    assert same and oshape == (640, 8, 64) and ishape == (640, 4, 4)
+    for p in procs:
+        assert p.exitcode == 0
+
+
+def test_group_range_splits_evenly():
+    from block_sparse_long_branch_b200 import shard
+    assert [shard.group_range(8, r, 4) for r in range(4)] == [(0, 2), (2, 4), (4, 6), (6, 8)]
+    with pytest.raises(ValueError):
+        shard.group_range(8, 0, 3)

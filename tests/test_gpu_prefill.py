@@ -301,3 +301,30 @@ def test_prefill_varlen_small_workspace_chunks_each_sequence(msa):
     torch.cuda.synchronize()
     assert msa.msa_get_device_error(ws) == 0
     assert torch.equal(full, small)
+
+
+def test_head_shards_equal_whole_prefill(msa):
+    """The head-sharded plan on one GPU: each rank's group slice computed by
+    its own msa_prefill call (one after another here, no collective), the
+    slices concatenated along the heads, equal the single call bit for bit."""
+    from block_sparse_long_branch_b200 import shard
+    s = synth.PrefillShape("shards", N=3000, H=16, G=4, d=128, d_idx=128, top_k=8, n_needles=4,
+                           seed=62)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    whole_out, whole_ids = msa.msa_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"],
+                                           inp["k_idx"], ids_out=True)
+    for world in (2, 4):
+        outs, idss = [], []
+        for rank in range(world):
+            g0, g1 = shard.group_range(s.G, rank, world)
+            c = msa.config((g1 - g0) * (s.H // s.G), g1 - g0, s.d, s.d_idx, top_k=s.top_k,
+                           scale=s.scale)
+            o, i = msa.msa_prefill(c, *shard.shard_inputs(inp["q"], inp["k"], inp["v"],
+                                                          inp["q_idx"], inp["k_idx"], s.H, s.G,
+                                                          rank, world), ids_out=True)
+            outs.append(o)
+            idss.append(i)
+        torch.cuda.synchronize()
+        assert torch.equal(torch.cat(idss, dim=1), whole_ids)
+        assert torch.equal(torch.cat(outs, dim=1), whole_out)
