@@ -22,7 +22,7 @@ __all__ = [
     "MsaConfig", "MsaError", "config", "library_path", "load_library",
     "OP_SELECT_TOPK", "OP_BLOCK_QUERY_LISTS", "OP_PREFILL", "OP_DECODE",
     "msa_workspace_size", "msa_prefill_min_workspace", "msa_prefill_chunk_tokens",
-    "msa_index_scores", "msa_select_topk",
+    "msa_index_scores", "msa_select_topk", "msa_quantize_index_fp8", "msa_select_topk_fp8",
     "msa_build_block_query_lists", "msa_prefill", "msa_decode", "msa_get_device_error",
     "msa_status_string", "msa_last_launch_count", "msa_set_phase_events", "msa_decode_static",
     "msa_selftest_wait_timeout", "msa_prefill_varlen", "msa_prefill_block_alignment",
@@ -93,6 +93,8 @@ def load_library():
     lib.msa_prefill_chunk_tokens.argtypes = [C, I64, SZ, I32, ctypes.POINTER(I64)]
     lib.msa_index_scores.argtypes = [C, P, P, I64, I64, I64, P, P]
     lib.msa_select_topk.argtypes = [C, P, P, I64, P, P, SZ, P]
+    lib.msa_quantize_index_fp8.argtypes = [C, P, P, I64, P, P, P, P]
+    lib.msa_select_topk_fp8.argtypes = [C, P, P, P, I64, P, P, SZ, P]
     lib.msa_build_block_query_lists.argtypes = [C, P, I64, P, P, P, SZ, P]
     lib.msa_prefill.argtypes = [C, P, P, P, P, P, I64, P, P, P, SZ, P]
     lib.msa_prefill_varlen.argtypes = [C, P, P, P, P, P, P, I32, P, P, P, SZ, P]
@@ -109,7 +111,8 @@ def load_library():
     lib.msa_last_launch_count.restype = I32
     for name in ("msa_workspace_size", "msa_prefill_min_workspace", "msa_prefill_chunk_tokens",
                  "msa_index_scores",
-                 "msa_select_topk", "msa_build_block_query_lists", "msa_prefill",
+                 "msa_select_topk", "msa_quantize_index_fp8", "msa_select_topk_fp8",
+                 "msa_build_block_query_lists", "msa_prefill",
                  "msa_prefill_varlen", "msa_prefill_block_alignment", "msa_decode",
                  "msa_decode_static", "msa_get_device_error", "msa_selftest_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
@@ -216,6 +219,47 @@ def msa_select_topk(cfg: MsaConfig, q_idx: torch.Tensor, k_idx: torch.Tensor,
                              _dev(ids, torch.int32, "ids", (N, G, k)), _dev(ws, torch.uint8, "ws"),
                              ws.numel(), _stream(stream))
     _check(st, "msa_select_topk")
+    return ids
+
+
+def msa_quantize_index_fp8(cfg: MsaConfig, q_idx: torch.Tensor, k_idx: torch.Tensor,
+                           stream=None):
+    """(q_idx [N,G,128], k_idx [N,128] bf16) -> (q_idx8, k_idx8 uint8 e4m3 bytes,
+    k_scale [ceil(N/128)] float32)."""
+    lib = load_library()
+    N = q_idx.shape[0]
+    G, di = cfg.num_groups, cfg.index_dim
+    dev = q_idx.device
+    q8 = torch.empty((N, G, di), dtype=torch.uint8, device=dev)
+    k8 = torch.empty((N, di), dtype=torch.uint8, device=dev)
+    ks = torch.empty(((N + cfg.block_size - 1) // cfg.block_size,), dtype=torch.float32,
+                     device=dev)
+    st = lib.msa_quantize_index_fp8(ctypes.byref(cfg),
+                                    _dev(q_idx, torch.bfloat16, "q_idx", (N, G, di)),
+                                    _dev(k_idx, torch.bfloat16, "k_idx", (N, di)), N,
+                                    _dev(q8, torch.uint8, "q_idx8"), _dev(k8, torch.uint8, "k_idx8"),
+                                    _dev(ks, torch.float32, "k_scale"), _stream(stream))
+    _check(st, "msa_quantize_index_fp8")
+    return q8, k8, ks
+
+
+def msa_select_topk_fp8(cfg: MsaConfig, q_idx8: torch.Tensor, k_idx8: torch.Tensor,
+                        k_scale: torch.Tensor, ids: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """msa_select_topk on e4m3 index tensors with per-block key scales."""
+    lib = load_library()
+    N = q_idx8.shape[0]
+    G, di, k = cfg.num_groups, cfg.index_dim, cfg.top_k
+    nb = (N + cfg.block_size - 1) // cfg.block_size
+    if ids is None:
+        ids = torch.empty((N, G, k), dtype=torch.int32, device=q_idx8.device)
+    ws = _workspace(workspace, msa_workspace_size(cfg, OP_SELECT_TOPK, N), q_idx8.device)
+    st = lib.msa_select_topk_fp8(ctypes.byref(cfg), _dev(q_idx8, torch.uint8, "q_idx8", (N, G, di)),
+                                 _dev(k_idx8, torch.uint8, "k_idx8", (N, di)),
+                                 _dev(k_scale, torch.float32, "k_scale", (nb,)), N,
+                                 _dev(ids, torch.int32, "ids", (N, G, k)),
+                                 _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(st, "msa_select_topk_fp8")
     return ids
 
 

@@ -288,6 +288,63 @@ msa_status_t msa_select_topk(const msa_config_t* cfg, const void* q_idx, const v
   return st;
 }
 
+msa_status_t msa_quantize_index_fp8(const msa_config_t* cfg, const void* q_idx, const void* k_idx,
+                                    int64_t N, void* q_idx8, void* k_idx8, float* k_scale,
+                                    msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  if (cfg->index_dim != 128) return MSA_ERR_UNSUPPORTED;
+  if (!q_idx || !k_idx || !q_idx8 || !k_idx8 || !k_scale) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q_idx8) || !aligned16(k_idx8) ||
+      !aligned16(k_scale))
+    return MSA_ERR_INVALID_ARG;
+  QuantLaunch p{};
+  p.q_idx = q_idx;
+  p.k_idx = k_idx;
+  p.N = N;
+  p.G = cfg->num_groups;
+  p.d_idx = cfg->index_dim;
+  p.q_idx8 = q_idx8;
+  p.k_idx8 = k_idx8;
+  p.kscale = k_scale;
+  st = cuda_status(launch_quantize_index(p, reinterpret_cast<cudaStream_t>(stream)));
+  g_launches = 2;
+  return st;
+}
+
+msa_status_t msa_select_topk_fp8(const msa_config_t* cfg, const void* q_idx8, const void* k_idx8,
+                                 const float* k_scale, int64_t N, int32_t* ids, void* ws,
+                                 size_t ws_bytes, msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  if (cfg->index_dim != 128) return MSA_ERR_UNSUPPORTED;
+  if (!q_idx8 || !k_idx8 || !k_scale || !ids) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx8) || !aligned16(k_idx8) || !aligned16(ids)) return MSA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < kHeader || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  IndexLaunch p{};
+  p.q_idx = q_idx8;
+  p.k_idx = k_idx8;
+  p.kscale = k_scale;
+  p.N = N;
+  p.G = cfg->num_groups;
+  p.d_idx = cfg->index_dim;
+  p.top_k = cfg->top_k;
+  p.row_begin = 0;
+  p.row_end = N;
+  p.ids = ids;
+  p.err = at<uint32_t>(ws, 0);
+  p.num_sms = sm_count();
+  st = cuda_status(launch_index_select(p, s));
+  g_launches = 1;
+  return st;
+}
+
 msa_status_t msa_build_block_query_lists(const msa_config_t* cfg, const int32_t* ids, int64_t N,
                                          int32_t* row_ptr, int32_t* entries, void* ws,
                                          size_t ws_bytes, msa_stream_t stream) {

@@ -11,8 +11,11 @@
 // query block times all G groups, i.e. 128 contiguous rows of q_idx viewed as
 // [N*G][d_idx].  Every key block j < blk(t) is fully visible to every token of
 // the tile, so selection needs no causal mask: the local block is forced in
-// and never scored.  One tcgen05.mma of M=128 x N=256 x K=16 covers two key
-// blocks; d_idx/16 of them accumulate a 128x256 fp32 score tile in TMEM.
+// and never scored.  One tcgen05.mma chain of M=128 x N=256 covers two key
+// blocks (K=16 per bf16 instruction, K=32 per e4m3 one) and accumulates a
+// 128x256 fp32 score tile in TMEM.  (N=128 per block would re-read the A
+// tile from shared memory twice as often, which then runs at the tensor
+// pipe's own rate.)
 //
 // Warp roles (192 threads, one CTA per SM, persistent over tiles):
 //   warp 0  TMA producer: q_idx tile once per tile, k_idx pairs into a ring
@@ -20,9 +23,11 @@
 //   warp 1  MMA issuer: one elected thread, double-buffered TMEM accumulators
 //           (2 x 256 columns), tcgen05.commit -> mbarriers;
 //   warps 2-5  epilogue: thread <-> TMEM lane <-> tile row; tcgen05.ld the
-//           row's 256 scores, max per block, insert into a register-resident
-//           sorted list of the best (k-1) blocks (strict '>' keeps the lower id
-//           on equal scores, since blocks arrive in increasing id order).
+//           row's 256 scores in 32-column chunks, each load in flight while
+//           the previous chunk is folded into eight independent max chains;
+//           max per block, then a one-step insert into a register-resident
+//           sorted list of the best (k-1) blocks (an equal score keeps the
+//           lower id, since blocks arrive in increasing id order).
 //
 // Tiles are ordered longest first (latest query block first) and dealt to
 // the CTAs round-robin.
@@ -33,19 +38,40 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 192;
 constexpr int kRows = 128;      // UMMA M: index-query rows per tile
 constexpr int kPairKeys = 256;  // UMMA N: two key blocks per MMA
 constexpr int kBlock = 128;     // B_k
 
-template <int DI>
+// FP8: e4m3 index queries and keys (kind::f8f6f4, 32 elements per MMA K
+// step) with one fp32 scale per 128-key block; otherwise bf16 (kind::f16,
+// 16 per step).  Either way a K step is 32 bytes of a 128-byte swizzled row.
+template <int DI, bool FP8 = false>
 struct IdxCfg {
-  static constexpr int kRegions = DI / 64;  // 128-byte swizzle spans per row
-  static constexpr int kABytes = kRows * DI * 2;
-  static constexpr int kBBytes = kPairKeys * DI * 2;
-  static constexpr int kStages = DI == 128 ? 3 : 5;
+  static constexpr int kElemBytes = FP8 ? 1 : 2;
+  static constexpr int kRowBytes = DI * kElemBytes;
+  static constexpr int kRegions = kRowBytes / 128;  // 128-byte swizzle spans per row
+  static constexpr int kRegionElems = 128 / kElemBytes;
+  static constexpr int kKSteps = kRowBytes / 32;
+  static constexpr int kABytes = kRows * kRowBytes;
+  static constexpr int kBBytes = kPairKeys * kRowBytes;
+  static constexpr int kStages = kRowBytes == 256 ? 3 : 5;
   static constexpr int kSmem = kABytes + kStages * kBBytes + 1024;
 };
+constexpr int kThreads = 192;
+
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// instruction descriptor of kind::f8f6f4: D fp32, A and B e4m3 (format 0), K-major
+__host__ __device__ constexpr uint32_t idesc_e4m3(uint32_t M, uint32_t N) {
+  return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
 
 struct IdxArgs {
   int64_t N;
@@ -55,6 +81,7 @@ struct IdxArgs {
   int64_t nb;
   int32_t* ids;
   float* scores;
+  const float* kscale;  // FP8 only: [nb] scale of each key block
   uint32_t* err;
 };
 
@@ -81,15 +108,21 @@ __device__ __forceinline__ Unit make_unit(const IdxArgs& a, int v) {
   return u;
 }
 
-__device__ __forceinline__ float max4(float a, float b, float c, float d) {
-  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+
+// folds 32 fp32 scores held as raw TMEM words into eight running max chains
+// (three-input max; consecutive instructions are independent), in program
+// order with the surrounding TMEM loads and waits
+__device__ __forceinline__ void max_chains_ordered(float (&x)[8], const uint32_t (&r)[32]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    x[i & 7] = fmax3_ordered(x[i & 7], __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
 }
 
-template <int DI, int MAXSEL, bool SCORES>
+template <int DI, int MAXSEL, bool SCORES, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     index_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                  const IdxArgs a) {
-  using Cfg = IdxCfg<DI>;
+  using Cfg = IdxCfg<DI, FP8>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -149,7 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bar_a_full, Cfg::kABytes);
 #pragma unroll
         for (int r = 0; r < Cfg::kRegions; ++r)
-          tma_load_2d(sA + r * kRows * 128, &map_q, &bar_a_full, r * 64, (int32_t)u.row0);
+          tma_load_2d(sA + r * kRows * 128, &map_q, &bar_a_full, r * Cfg::kRegionElems,
+                      (int32_t)u.row0);
         a_issued = true;
         a_last = aphase;
         aphase ^= 1;
@@ -162,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int r = 0; r < Cfg::kRegions; ++r)
             tma_load_2d(sB + stage * Cfg::kBBytes + r * kPairKeys * 128, &map_k, &bar_b_full[stage],
-                        r * 64, p * kPairKeys);
+                        r * Cfg::kRegionElems, p * kPairKeys);
           b_issued[stage] = true;
           b_last[stage] = sphase;
           if (++stage == S) stage = 0, sphase ^= 1;
@@ -179,7 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kRows, kPairKeys, false, false);
+      constexpr uint32_t idesc =
+          FP8 ? idesc_e4m3(kRows, kPairKeys) : idesc_bf16(kRows, kPairKeys, false, false);
       int stage = 0, acc = 0;
       uint32_t sphase = 0, aphase = 0;
       uint32_t accphase[2] = {0, 0};
@@ -203,12 +238,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_base = smem_u32(sB + stage * Cfg::kBBytes);
           const uint32_t d = tmem + acc * kPairKeys;
 #pragma unroll
-          for (int kk = 0; kk < DI / 16; ++kk) {
+          for (int kk = 0; kk < Cfg::kKSteps; ++kk) {
             const uint64_t ad = smem_desc_sw128(a_base + (kk >> 2) * kRows * 128 + (kk & 3) * 32,
                                                 16, 1024);
             const uint64_t bd = smem_desc_sw128(
                 b_base + (kk >> 2) * kPairKeys * 128 + (kk & 3) * 32, 16, 1024);
-            umma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            if constexpr (FP8)
+              umma_e4m3(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            else
+              umma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
           umma_commit(&bar_b_empty[stage]);
           umma_commit(&bar_acc_full[acc]);
@@ -258,37 +296,53 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        const uint32_t col = lane_addr + acc * kPairKeys;
         float m[2];
+        if (SCORES) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t r[4][32];
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[4][32];
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tmem_ld_32x32b_x32(lane_addr + acc * kPairKeys + h * 128 + c * 32, r[c]);
-          tmem_wait();
+            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(col + h * 128 + c * 32, r[c]);
+            tmem_wait();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) reg_fence(r[c]);
-          const int j = 2 * p + h;
-          if (SCORES && j == u.b) {
+            for (int c = 0; c < 4; ++c) reg_fence(r[c]);
+            const int j = 2 * p + h;
             float mx = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (c * 32 + i <= lim) mx = fmaxf(mx, __uint_as_float(r[c][i]));
+                if (j != u.b || c * 32 + i <= lim) mx = fmaxf(mx, __uint_as_float(r[c][i]));
             m[h] = mx;
-          } else {
-            float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
+          }
+        } else {
+          // eight 32-column chunks, double-buffered: the next chunk's TMEM load
+          // is in flight while this one is folded into eight max chains
+          uint32_t ra[32], rb[32];
+          float x[8];
+          tmem_ld_32x32b_x32(col, ra);
+          tmem_wait();
+          reg_fence(ra);
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 8; c += 2) {
+            if ((c & 3) == 0) {
 #pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                x0 = fmaxf(x0, __uint_as_float(r[c][i]));
-                x1 = fmaxf(x1, __uint_as_float(r[c][i + 1]));
-                x2 = fmaxf(x2, __uint_as_float(r[c][i + 2]));
-                x3 = fmaxf(x3, __uint_as_float(r[c][i + 3]));
-              }
-            m[h] = max4(x0, x1, x2, x3);
+              for (int i = 0; i < 8; ++i) x[i] = -INFINITY;
+            }
+            tmem_ld_32x32b_x32(col + (c + 1) * 32, rb);
+            max_chains_ordered(x, ra);
+            tmem_wait();
+            reg_fence(rb);
+            if (c + 2 < 8) tmem_ld_32x32b_x32(col + (c + 2) * 32, ra);
+            max_chains_ordered(x, rb);
+            if ((c & 3) == 2)
+              m[c >> 2] = fmax3_ordered(fmax3_ordered(x[0], x[1], x[2]),
+                                        fmax3_ordered(x[3], x[4], x[5]), fmaxf(x[6], x[7]));
+            if (c + 2 < 8) {
+              tmem_wait();
+              reg_fence(ra);
+            }
           }
         }
         tc_fence_before();
@@ -299,24 +353,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < 2; ++h) {
           const int j = 2 * p + h;
           if (j >= u.nblk) continue;
+          // the keys of block j were quantised with the block's scale (> 0)
+          const float mj = FP8 ? m[h] * __ldg(a.kscale + j) : m[h];
           if constexpr (SCORES) {
-            if (row_out) srow[j] = m[h];
+            if (row_out) srow[j] = mj;
           } else {
-            // strict '>' : an equal score arriving later (higher id) ranks lower
-            if (m[h] > sc[MAXSEL - 1]) {
-              sc[MAXSEL - 1] = m[h];
-              id[MAXSEL - 1] = j;
+            if (mj > sc[MAXSEL - 1]) {
+              // insert into the descending list in one step: slot i keeps its
+              // entry when that entry is not below mj (an equal, earlier block
+              // ranks higher), takes mj at the first slot below it, and takes
+              // slot i-1's entry after that
 #pragma unroll
               for (int i = MAXSEL - 1; i > 0; --i) {
-                if (sc[i] > sc[i - 1]) {
-                  const float ts = sc[i];
-                  sc[i] = sc[i - 1];
-                  sc[i - 1] = ts;
-                  const int32_t ti = id[i];
-                  id[i] = id[i - 1];
-                  id[i - 1] = ti;
-                }
+                const bool keep = sc[i] >= mj;
+                const bool here = sc[i - 1] >= mj;
+                id[i] = keep ? id[i] : (here ? j : id[i - 1]);
+                sc[i] = fmaxf(fminf(sc[i - 1], mj), sc[i]);
               }
+              id[0] = sc[0] >= mj ? id[0] : j;
+              sc[0] = fmaxf(sc[0], mj);
             }
           }
         }
@@ -355,14 +410,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <int DI, int MAXSEL, bool SCORES>
+template <int DI, int MAXSEL, bool SCORES, bool FP8 = false>
 cudaError_t launch_impl(const IndexLaunch& p, cudaStream_t s) {
-  using Cfg = IdxCfg<DI>;
+  using Cfg = IdxCfg<DI, FP8>;
   CUtensorMap mq, mk;
-  if (!make_tmap_bf16_2d(&mq, p.q_idx, (uint64_t)p.N * p.G, DI, DI, kRows, 64,
-                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_bf16_2d(&mk, p.k_idx, (uint64_t)p.N, DI, DI, kPairKeys, 64,
-                         CU_TENSOR_MAP_SWIZZLE_128B))
+  // rows of DI elements; make_tmap_2d counts the pitch in 2-byte units
+  const CUtensorMapDataType type =
+      FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_tmap_2d(&mq, type, p.q_idx, (uint64_t)p.N * p.G, DI, Cfg::kRowBytes / 2, kRows,
+                    Cfg::kRegionElems, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&mk, type, p.k_idx, (uint64_t)p.N, DI, Cfg::kRowBytes / 2, kPairKeys,
+                    Cfg::kRegionElems, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   IdxArgs a;
   a.N = p.N;
@@ -376,10 +434,11 @@ cudaError_t launch_impl(const IndexLaunch& p, cudaStream_t s) {
   a.nb = (p.N + kBlock - 1) / kBlock;
   a.ids = p.ids;
   a.scores = p.scores;
+  a.kscale = p.kscale;
   a.err = p.err;
   const int n_units = a.n_qblocks * p.G;
   const int grid = n_units < p.num_sms ? n_units : p.num_sms;
-  auto kern = index_kernel<DI, MAXSEL, SCORES>;
+  auto kern = index_kernel<DI, MAXSEL, SCORES, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, Cfg::kSmem, s>>>(mq, mk, a);
@@ -389,6 +448,11 @@ cudaError_t launch_impl(const IndexLaunch& p, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_index_select(const IndexLaunch& p, cudaStream_t s) {
+  if (p.kscale) {  // e4m3 index tensors: d_idx = 128 only
+    if (p.d_idx != 128) return cudaErrorInvalidValue;
+    if (p.top_k <= 16) return launch_impl<128, 15, false, true>(p, s);
+    return launch_impl<128, 31, false, true>(p, s);
+  }
   if (p.d_idx == 128) {
     if (p.top_k <= 16) return launch_impl<128, 15, false>(p, s);
     return launch_impl<128, 31, false>(p, s);

@@ -11,13 +11,14 @@ namespace msa {
 
 // ---- Index Branch (index_kernel.cu) ---------------------------------------
 struct IndexLaunch {
-  const void* q_idx;  // [N][G][d_idx] bf16
-  const void* k_idx;  // [N][d_idx] bf16
+  const void* q_idx;  // [N][G][d_idx] bf16, or e4m3 when kscale is set
+  const void* k_idx;  // [N][d_idx] bf16, or e4m3 when kscale is set
   int64_t N;
   int32_t G, d_idx, top_k;
   int64_t row_begin, row_end;  // query rows processed: [row_begin, row_end)
   int32_t* ids;                // selection mode: [row_end-row_begin][G][top_k]
   float* scores;               // scores mode: [row_end-row_begin][G][nb]
+  const float* kscale;         // e4m3 selection only: [nb] scale of each key block
   uint32_t* err;
   int num_sms;
 };
@@ -81,6 +82,19 @@ struct MergeLaunch {
   float* kl;                 // out: [rows][G] KL(mass || softmax of the scores over the slots)
 };
 cudaError_t launch_merge(const MergeLaunch& p, cudaStream_t s);
+
+// e4m3 index tensors (quant_kernel.cu): q_idx8 [N][G][d_idx], k_idx8 [N][d_idx],
+// kscale [ceil(N/128)] (one scale per 128-key block); d_idx = 128.
+struct QuantLaunch {
+  const void* q_idx;  // bf16
+  const void* k_idx;  // bf16
+  int64_t N;
+  int32_t G, d_idx;
+  void* q_idx8;
+  void* k_idx8;
+  float* kscale;
+};
+cudaError_t launch_quantize_index(const QuantLaunch& p, cudaStream_t s);
 
 // Block-alignment diagnostic: pooled index score of every listed (t, r).
 struct BlockScoreLaunch {

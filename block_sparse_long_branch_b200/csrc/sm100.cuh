@@ -318,6 +318,21 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100 and later);
+// a NaN operand is ignored as fmaxf ignores it.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// The same, kept in program order with the other volatile asm (TMEM loads and
+// waits), so a reduction is not deferred past the load that follows it.
+__device__ __forceinline__ float fmax3_ordered(float a, float b, float c) {
+  float d;
+  asm volatile("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Shared-memory matrix descriptor for tcgen05.mma, 128-byte swizzle, sm_100
 // layout (version field = 1).  For a K-major operand the 8-row groups are
 // `sbo` bytes apart and `lbo` is unused; for an MN-major operand `lbo` is the

@@ -177,6 +177,35 @@ MSA_API msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const v
                          int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream);
 
 /*
+ * Quantised Index Branch (e4m3).  The pages report the sparse attention's
+ * indexer and main branch moving from Q8KV8 to Q8KV4 in a later model
+ * (dot-ai "MiniMax M3.1 Flashとは？428BのMoEモデルがウェイト公開", the passage on
+ * the ModelScope model card's quantisation) but give no number format; the
+ * reading used here, for the indexer only, with d_idx = 128:
+ *   per index-query row (t, g) and per 128-key block j of the index keys,
+ *   s = max|x| / 448 (fp32, nearest; 1 when the max is 0), x8 = e4m3(x / s)
+ *   (fp32 division, nearest even, saturating at +-448).
+ * msa_quantize_index_fp8: q_idx [N][G][128], k_idx [N][128] bf16 ->
+ *   q_idx8 [N][G][128], k_idx8 [N][128] e4m3 bytes, k_scale [ceil(N/128)] fp32
+ *   (the query rows' scales are not kept: see below).
+ * msa_select_topk_fp8: as msa_select_topk, ranking block j of a query row by
+ *   k_scale[j] * max over its keys of <q_idx8[t][g], k_idx8[s]> (fp32
+ *   accumulation on kind::f8f6f4 tensor cores).  A row's own scale is a
+ *   positive factor of all its scores and cannot change its ranking.
+ *   k_scale: device, [ceil(N/128)] fp32, every entry finite and > 0 (the
+ *   quantiser writes 1 for an all-zero block); not checked on the device.
+ *   ws: at least msa_workspace_size(cfg, MSA_OP_SELECT_TOPK, N, 0).
+ * d_idx other than 128 -> MSA_ERR_UNSUPPORTED.
+ */
+MSA_API msa_status_t msa_quantize_index_fp8(const msa_config_t* cfg, const void* q_idx,
+                                            const void* k_idx, int64_t N, void* q_idx8,
+                                            void* k_idx8, float* k_scale, msa_stream_t stream);
+MSA_API msa_status_t msa_select_topk_fp8(const msa_config_t* cfg, const void* q_idx8,
+                                         const void* k_idx8, const float* k_scale, int64_t N,
+                                         int32_t* ids, void* ws, size_t ws_bytes,
+                                         msa_stream_t stream);
+
+/*
  * msa_prefill plus the data of the Index Branch's KL alignment, forward only:
  * the Index Branch is trained to bring its distribution of block scores
  * close to the distribution of where the Main Branch's exact attention went

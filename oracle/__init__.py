@@ -4,9 +4,11 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The product library
 (``block_sparse_long_branch_b200``) never imports it and has no CPU fallback.
 
-The arithmetic lives in ``msa_oracle.c`` (plain loops, fp64); this module only
-marshals numpy arrays through ctypes.  Each wrapper names the passage of the
-pages it follows; the C file carries the same citations.
+The attention arithmetic lives in ``msa_oracle.c`` (plain loops, fp64); this
+module marshals numpy arrays through ctypes, and holds in numpy the e4m3
+codec and quantiser of the quantised Index Branch (format arithmetic only).
+Each wrapper names the passage of the pages it follows; the C file carries the
+same citations.
 """
 from __future__ import annotations
 
@@ -31,6 +33,8 @@ def _load():
         I32 = ctypes.c_int32
         lib.msa_oracle_pooled_scores.argtypes = [P, P, I64, P, I32, I32, I32, I64, P]
         lib.msa_oracle_pooled_scores.restype = None
+        lib.msa_oracle_pooled_scores_f64.argtypes = [P, P, I64, P, I32, I32, I32, I64, P]
+        lib.msa_oracle_pooled_scores_f64.restype = None
         lib.msa_oracle_select_blocks.argtypes = [P, P, I64, I32, I64, I32, I32, P]
         lib.msa_oracle_select_blocks.restype = None
         lib.msa_oracle_block_attention.argtypes = [P, P, I64, P, P, I32, I32, I32, I32, I32,
@@ -208,3 +212,87 @@ def decode(q, q_idx, k_cache, v_cache, k_idx_cache, cu_seqlens, *, block: int, t
         out[b] = o[0]
         pooled[b] = p[0]
     return dict(ids=ids, out=out, pooled=pooled)
+
+
+# ---------------------------------------------------------------------------
+# Quantised Index Branch (e4m3).  The pages report the indexer and main branch
+# moving from Q8KV8 to Q8KV4 in a later model (dot-ai "MiniMax M3.1 Flashとは？
+# 428BのMoEモデルがウェイト公開", the passage on the ModelScope model card's
+# quantisation) with no number format; the reading used: per index-query row
+# and per 128-key block of index keys, s = max|x| / 448 in fp32 (1 when the
+# max is 0) and x8 = e4m3(x / s), fp32 division, nearest even, saturating.
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(b: np.ndarray) -> np.ndarray:
+    """e4m3 bytes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+    infinities, 0x7F/0xFF are NaN) -> fp64."""
+    b = np.asarray(b, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = b & 7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    val = np.where((b & 0x7F) == 0x7F, np.nan, val)
+    return sign * val
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """fp32 values -> nearest e4m3 byte (ties to even), saturating at +-448."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    sign = np.where(np.signbit(x), 0x80, 0).astype(np.int64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    # quantum of the binade: 2^(e-3) for normals (e >= -6), 2^-9 below
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)
+    q = 2.0 ** (e - 3)
+    n = np.rint(a / q)  # round half to even
+    v = n * q           # the e4m3 value (may reach the next binade)
+    e2 = np.floor(np.log2(np.where(v > 0, v, 1.0)))
+    normal = v >= 2.0 ** -6
+    ef = np.where(normal, e2 + 7, 0).astype(np.int64)
+    mf = np.where(normal, np.rint((v / 2.0 ** e2 - 1.0) * 8.0), np.rint(v / 2.0 ** -9))
+    code = (ef << 3) | mf.astype(np.int64)
+    code = np.where(v == 0, 0, code)
+    return (sign | code).astype(np.uint8)
+
+
+def _scale(amax: np.ndarray) -> np.ndarray:
+    amax = np.asarray(amax, dtype=np.float32)
+    return np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+
+
+def quantize_index_fp8(q_idx, k_idx, block: int = 128):
+    """(q_idx [N,G,d] bf16, k_idx [N,d] bf16) -> (q8 [N,G,d] u8, k8 [N,d] u8,
+    k_scale [ceil(N/block)] f32)."""
+    qf = bf16_bits_to_f64(as_bf16_bits(q_idx)).astype(np.float32)
+    kf = bf16_bits_to_f64(as_bf16_bits(k_idx)).astype(np.float32)
+    sq = _scale(np.abs(qf).max(axis=2))
+    q8 = e4m3_encode(qf / sq[:, :, None])
+    N = kf.shape[0]
+    nb = (N + block - 1) // block
+    amax = np.array([np.abs(kf[j * block:(j + 1) * block]).max() for j in range(nb)],
+                    dtype=np.float32)
+    sk = _scale(amax)
+    k8 = e4m3_encode(kf / np.repeat(sk, block)[:N, None])
+    return q8, k8, sk
+
+
+def pooled_scores_fp8(q8_rows, pos, k8, k_scale, block: int, nb_out: int) -> np.ndarray:
+    """Pooled scores of the quantised Index Branch: the max over visible keys of
+    <e4m3(q8), e4m3(k8) * k_scale[block of the key]> (fp64)."""
+    lib = _load()
+    qv = np.ascontiguousarray(e4m3_decode(q8_rows), dtype=np.float64)
+    kv = e4m3_decode(k8) * np.repeat(np.asarray(k_scale, dtype=np.float64),
+                                     block)[:np.asarray(k8).shape[0], None]
+    kv = np.ascontiguousarray(kv, dtype=np.float64)
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int64))
+    n, G, di = qv.shape
+    assert kv.shape[1] == di and pos.shape == (n,)
+    assert n == 0 or kv.shape[0] > int(pos.max())
+    out = np.empty((n, G, nb_out), dtype=np.float64)
+    lib.msa_oracle_pooled_scores_f64(_ptr(qv), _ptr(pos), n, _ptr(kv), G, di, block, nb_out,
+                                     _ptr(out))
+    return out

@@ -97,6 +97,37 @@ ORACLE_API void msa_oracle_pooled_scores(const uint16_t* qi_rows, const int64_t*
     }
 }
 
+/*
+ * The same pooled scores for inputs given in fp64 (the quantised Index
+ * Branch: dequantised e4m3 values times their scales).
+ *
+ * qi_rows : [n][G][di] fp64, k_rows : [T][di] fp64; other arguments and
+ * pooled as msa_oracle_pooled_scores.
+ */
+ORACLE_API void msa_oracle_pooled_scores_f64(const double* qi_rows, const int64_t* pos,
+                                             int64_t n, const double* k_rows, int32_t G,
+                                             int32_t di, int32_t block, int64_t nb_out,
+                                             double* pooled)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t t = pos[i];
+        for (int32_t g = 0; g < G; ++g) {
+            const double* qv = qi_rows + ((size_t)i * G + g) * di;
+            double* out = pooled + ((size_t)i * G + g) * nb_out;
+            for (int64_t j = 0; j < nb_out; ++j) out[j] = -INFINITY;
+            for (int64_t s = 0; s <= t; ++s) {
+                const int64_t j = s / block;
+                if (j >= nb_out) break;
+                const double* kv = k_rows + (size_t)s * di;
+                double dot = 0.0;
+                for (int32_t c = 0; c < di; ++c) dot += qv[c] * kv[c];
+                if (dot > out[j]) out[j] = dot;
+            }
+        }
+    }
+}
+
 typedef struct {
     double score;
     int64_t id;
