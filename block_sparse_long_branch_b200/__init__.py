@@ -38,7 +38,7 @@ OP_DECODE = 3
 
 STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
                 3: "MSA_ERR_WORKSPACE", 4: "MSA_ERR_CUDA", 5: "MSA_ERR_DEVICE_TIMEOUT",
-                6: "MSA_ERR_DEVICE_INDEX"}
+                6: "MSA_ERR_DEVICE_INDEX", 7: "MSA_ERR_DEVICE_RANGE"}
 
 
 class MsaConfig(ctypes.Structure):

@@ -65,12 +65,14 @@ int sm_count() {
   return n;
 }
 
-// ---- prefill workspace for one chunk of `rows` query rows ------------------
+// ---- prefill workspace: the fp16 copy of V for all N tokens, then the
+// scratch of one chunk of `rows` query rows ---------------------------------
 struct PrefillLayout {
-  size_t ids, row_ptr, entries, unit_ptr, unit_list, csr, part_o, part_lse, total;
+  size_t v16, ids, row_ptr, entries, unit_ptr, unit_list, csr, part_o, part_lse, total;
 };
 
-PrefillLayout prefill_layout(const msa_config_t* c, int64_t rows, int64_t nb, bool own_ids) {
+PrefillLayout prefill_layout(const msa_config_t* c, int64_t N, int64_t rows, int64_t nb,
+                             bool own_ids) {
   const int64_t G = c->num_groups, k = c->top_k, HG = c->num_heads / c->num_groups;
   const int64_t slots = rows * G * k;
   const int64_t lists = G * nb;
@@ -78,6 +80,9 @@ PrefillLayout prefill_layout(const msa_config_t* c, int64_t rows, int64_t nb, bo
   const int64_t max_units = (slots + per_unit - 1) / per_unit + lists;
   PrefillLayout L;
   size_t off = kHeader;
+  // at a fixed offset for every chunk of the call: converted once, read by all
+  L.v16 = off;
+  off += align256(N * G * c->head_dim * 2);
   L.ids = off;
   off += own_ids ? align256(slots * 4) : 0;
   L.row_ptr = off;
@@ -103,12 +108,12 @@ PrefillLayout prefill_layout(const msa_config_t* c, int64_t rows, int64_t nb, bo
 // not even 128 rows fit.
 int64_t prefill_chunk(const msa_config_t* cfg, int64_t N, size_t ws_bytes, bool own_ids) {
   const int64_t nb = n_blocks(N);
-  if (prefill_layout(cfg, N, nb, own_ids).total <= ws_bytes) return N;
-  if (prefill_layout(cfg, kBlock, nb, own_ids).total > ws_bytes) return 0;
+  if (prefill_layout(cfg, N, N, nb, own_ids).total <= ws_bytes) return N;
+  if (prefill_layout(cfg, N, kBlock, nb, own_ids).total > ws_bytes) return 0;
   int64_t lo = 1, hi = nb;  // in blocks
   while (lo < hi) {
     const int64_t mid = (lo + hi + 1) / 2;
-    if (prefill_layout(cfg, mid * kBlock, nb, own_ids).total <= ws_bytes)
+    if (prefill_layout(cfg, N, mid * kBlock, nb, own_ids).total <= ws_bytes)
       lo = mid;
     else
       hi = mid - 1;
@@ -167,6 +172,7 @@ const char* msa_status_string(msa_status_t s) {
     case MSA_ERR_CUDA: return "CUDA runtime or launch error";
     case MSA_ERR_DEVICE_TIMEOUT: return "a device-side wait ran out";
     case MSA_ERR_DEVICE_INDEX: return "a device-side index was out of range";
+    case MSA_ERR_DEVICE_RANGE: return "an input value was outside the range it is computed in";
   }
   return "unknown status";
 }
@@ -203,7 +209,7 @@ msa_status_t msa_workspace_size(const msa_config_t* cfg, msa_op_t op, int64_t n_
       *bytes = kHeader + csr_scratch_bytes(n_tokens, cfg->num_groups, cfg->top_k, nb);
       return MSA_OK;
     case MSA_OP_PREFILL:
-      *bytes = prefill_layout(cfg, n_tokens, nb, true).total;
+      *bytes = prefill_layout(cfg, n_tokens, n_tokens, nb, true).total;
       return MSA_OK;
     case MSA_OP_DECODE:
       break;
@@ -217,7 +223,7 @@ msa_status_t msa_prefill_min_workspace(const msa_config_t* cfg, int64_t N, size_
   if (!bytes) return MSA_ERR_INVALID_ARG;
   if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
   const int64_t rows = N < kBlock ? N : kBlock;
-  *bytes = prefill_layout(cfg, rows, n_blocks(N), true).total;
+  *bytes = prefill_layout(cfg, N, rows, n_blocks(N), true).total;
   return MSA_OK;
 }
 
@@ -391,7 +397,6 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
                          bool events, int* launches_out, float* block_score = nullptr,
                          float* block_mass = nullptr, float* kl = nullptr) {
   const int64_t nb = n_blocks(N);
-  (void)nb;
   const bool own_ids = ids_out == nullptr;
   const int64_t chunk = prefill_chunk(cfg, N, ws_bytes, own_ids);
   if (chunk == 0) return MSA_ERR_WORKSPACE;
@@ -402,13 +407,15 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
   const int sms = sm_count();
   uint32_t* err = at<uint32_t>(ws, 0);
   int launches = 0;
+  // V in fp16 for the PV product (its offset is the same for every chunk)
+  void* v16 = at<void>(ws, prefill_layout(cfg, N, chunk, nb, own_ids).v16);
   for (int64_t t0 = 0, c = 0; t0 < N; t0 += chunk, ++c) {
     const int64_t t1 = t0 + chunk < N ? t0 + chunk : N;
     const int ev = (int)(5 * c);
     mark(ev, s);
     const int64_t rows = t1 - t0;
     const int64_t nbc = n_blocks(t1);
-    const PrefillLayout L = prefill_layout(cfg, rows, nbc, own_ids);
+    const PrefillLayout L = prefill_layout(cfg, N, rows, nbc, own_ids);
     int32_t* ids = own_ids ? at<int32_t>(ws, L.ids) : ids_out + t0 * G * kk;
 
     IndexLaunch ip{};
@@ -463,10 +470,15 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
     }
     mark(ev + 2, s);
 
+    if (c == 0) {  // converted once, before the first Main Branch launch
+      if (launch_v_to_fp16(v, v16, N * G * d, err, sms, s) != cudaSuccess)
+        return cuda_status(cudaErrorLaunchFailure);
+      ++launches;
+    }
     MainLaunch mp{};
     mp.q = q;
     mp.k = k;
-    mp.v = v;
+    mp.v = v16;
     mp.N = N;
     mp.H = H;
     mp.G = G;
@@ -683,6 +695,7 @@ msa_status_t msa_get_device_error(void* ws, msa_stream_t stream, uint32_t* code)
   *code = c;
   if (c == 0) return MSA_OK;
   if ((c & 0xF00u) == 0x100u) return MSA_ERR_DEVICE_TIMEOUT;
+  if ((c & 0xF00u) == 0x300u) return MSA_ERR_DEVICE_RANGE;
   return MSA_ERR_DEVICE_INDEX;
 }
 

@@ -48,7 +48,7 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches);
 struct MainLaunch {
   const void* q;  // [N][H][d] bf16
   const void* k;  // [N][G][d] bf16
-  const void* v;  // [N][G][d] bf16
+  const void* v;  // [N][G][d] fp16: V converted by launch_v_to_fp16
   int64_t N;
   int32_t H, G, d, top_k;
   float scale;
@@ -65,6 +65,11 @@ struct MainLaunch {
 };
 // query tokens per 128-row Main Branch tile
 int main_tile_tokens(int H, int G);
+// dst = fp16(src) for n bf16 values (n a multiple of 8, both pointers 16-byte
+// aligned): the V operand of the Main Branch's PV product.  A value beyond the
+// fp16 range (or NaN) is saturated and records kDevValueRange.
+cudaError_t launch_v_to_fp16(const void* src, void* dst, int64_t n, uint32_t* err, int sms,
+                             cudaStream_t s);
 cudaError_t launch_main(const MainLaunch& p, cudaStream_t s);
 
 // ---- merge (merge_kernel.cu) ----------------------------------------------

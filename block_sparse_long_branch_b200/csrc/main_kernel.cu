@@ -12,9 +12,9 @@
 // Per tile (128 rows = TT tokens x the H/G heads of group g):
 //   S = Q_tile K_j^T            tcgen05.mma M=128 N=128 K=d   (TMEM, fp32)
 //   P = exp(scale*(S - rowmax)) softmax warps, causal mask on the local block;
-//                               bf16 P overwrites the S columns already read
+//                               fp16 P overwrites the S columns already read
 //   O = P V_j                   tcgen05.mma M=128 N=d  K=128, A = P from TMEM,
-//                               B = V_j from shared memory (MN-major)
+//                               B = V_j (fp16) from shared memory (MN-major)
 // and the row's partial (o = O / rowsum in fp16, lse = scale*rowmax +
 // ln rowsum) goes to slot (t, g, r, head); the merge kernel combines the <= k
 // slots of a query with log-sum-exp weights.
@@ -37,6 +37,13 @@
 // columns), buffer w belonging to softmax group w.  Keeping P in TMEM halves
 // the shared-memory operand traffic of the PV product and leaves the P
 // stores off the shared-memory pipe.
+//
+// Precision of the PV product.  P in [0, 1] goes to the tensor cores in fp16
+// (11-bit significand) rather than bf16 (8 bits): with bf16 P a softmax over
+// a handful of keys (the first tokens of a sequence) can be off by 2^-9 of
+// |v| per weight, which together with the bf16 output rounding exceeds 1e-2
+// on outputs of magnitude 2 to 4.  The two operands of one MMA share a type,
+// so V is converted to fp16 once per call (v_to_fp16_kernel below).
 #include "kernels.h"
 #include "sm100.cuh"
 #include "tmap.h"
@@ -164,9 +171,10 @@ __device__ __forceinline__ bool read_entry(const MainArgs& a, int e, int64_t& t,
   return ok;
 }
 
-// exp2 of 32 scores of a row, packed two bf16 per word (the even column in
+// exp2 of 32 scores of a row, packed two fp16 per word (the even column in
 // the lower half, the layout of an A operand in TMEM), and the fp32 sum of the
 // rounded values.  MASK: keep columns <= lim (relative to the first of the 32).
+// p <= 1, so the fp16 conversion never overflows.
 template <bool MASK>
 __device__ __forceinline__ void softmax32(const uint32_t (&sv)[32], uint64_t k2, uint64_t nm2,
                                           int lim, uint32_t taddr, uint64_t& acc_a,
@@ -183,11 +191,11 @@ __device__ __forceinline__ void softmax32(const uint32_t (&sv)[32], uint64_t k2,
       p0 = col <= lim ? p0 : 0.f;
       p1 = col + 1 <= lim ? p1 : 0.f;
     }
-    w[x2] = pack_bf16x2(p0, p1);
+    w[x2] = pack_half2(p0, p1);
     if (x2 & 1)
-      acc_b = f2_add(acc_b, bf16x2_as_f2(w[x2]));
+      acc_b = f2_add(acc_b, half2_as_f2(w[x2]));
     else
-      acc_a = f2_add(acc_a, bf16x2_as_f2(w[x2]));
+      acc_a = f2_add(acc_a, half2_as_f2(w[x2]));
     if ((x2 & 7) == 7) tmem_st_32x32b_x8(taddr + (x2 - 7), &w[x2 - 7]);
   }
 }
@@ -394,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // TMEM, B = V_j from shared memory, into O buffer n%2 once the epilogue
     // of tile n-2 has read it.
     if (lane == 0) {
-      constexpr uint32_t idesc_o = idesc_bf16(kRows, D, false, true);
+      constexpr uint32_t idesc_o = idesc_f16(kRows, D, false, true);  // fp16 P and V
       TilePos pc = first_tile(a, n_units);
       int pb = 0;
       uint32_t vph = 0;
@@ -420,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // columns at offset 8*(kk%4) of that half's S columns
           const uint32_t a_tm = tmem + pb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
           const uint64_t bd = smem_desc_sw128(v_base + kk * 16 * 128, kKeys * 128, 1024);
-          umma_bf16_ts(d_tm, a_tm, bd, idesc_o, kk > 0 ? 1u : 0u);
+          umma_f16_ts(d_tm, a_tm, bd, idesc_o, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bar_s_empty[pb]);  // P read: the S/P buffer is free
         umma_commit(&bar_o_full[pb]);
@@ -656,6 +664,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// V (bf16) -> fp16, 16 bytes per thread and step; records kDevValueRange for
+// a value beyond the fp16 range or NaN (saturated to +-65504 / kept NaN)
+__global__ void __launch_bounds__(256) v_to_fp16_kernel(const uint4* __restrict__ src,
+                                                        uint4* __restrict__ dst, int64_t n8,
+                                                        uint32_t* err) {
+  bool bad = false;
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * 256) {
+    const uint4 w = __ldg(src + i);
+    uint4 o;
+    const uint32_t* wi = &w.x;
+    uint32_t* oi = &o.x;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float lo = __uint_as_float(wi[c] << 16), hi = __uint_as_float(wi[c] & 0xFFFF0000u);
+      bad |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
+      oi[c] = pack_half2_satfinite(lo, hi);
+    }
+    dst[i] = o;
+  }
+  if (bad) record_error(err, kDevValueRange);
+}
+
 template <int D>
 cudaError_t launch_main_impl(const MainLaunch& p, cudaStream_t s) {
   using Cfg = MainCfg<D>;
@@ -671,8 +702,8 @@ cudaError_t launch_main_impl(const MainLaunch& p, cudaStream_t s) {
                     64, box_rows, D / 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_bf16_3d(&mk, p.k, D, p.G, p.N, D, (uint64_t)p.G * D, 64, 1, kKeys,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_bf16_3d(&mv, p.v, D, p.G, p.N, D, (uint64_t)p.G * D, 64, 1, kKeys,
-                         CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_tmap_3d(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.v, D, p.G, p.N, D,
+                    (uint64_t)p.G * D, 64, 1, kKeys, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   MainArgs a;
   a.N = p.N;
@@ -707,6 +738,19 @@ cudaError_t launch_main_impl(const MainLaunch& p, cudaStream_t s) {
 int main_tile_tokens(int H, int G) {
   const int HG = H / G;
   return kRows / (HG < 8 ? 8 : HG);
+}
+
+cudaError_t launch_v_to_fp16(const void* src, void* dst, int64_t n, uint32_t* err, int sms,
+                             cudaStream_t s) {
+  if (n % 8 != 0 || (reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15)
+    return cudaErrorInvalidValue;
+  const int64_t n8 = n / 8;
+  const int64_t want = (n8 + 255) / 256;
+  const int64_t cap = (int64_t)sms * 8;
+  const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
+  v_to_fp16_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst),
+                                        n8, err);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_main(const MainLaunch& p, cudaStream_t s) {

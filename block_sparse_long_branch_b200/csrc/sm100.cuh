@@ -23,6 +23,7 @@ enum DeviceError : uint32_t {
   kDevTimeoutConsumer = 0x103, // an epilogue/softmax hand-off never arrived
   kDevSelfTest = 0x1FE,        // msa_selftest_wait_timeout: the planted wait ran out
   kDevBadIndex = 0x201,        // an id or list entry outside its range
+  kDevValueRange = 0x301,      // an input value outside the range it is computed in
 };
 
 // Upper bound on any single wait (ns).  Every wait in these kernels is for an
@@ -236,10 +237,11 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// Same with A read from tensor memory: a_tmem is the column of the first K
-// element, M rows in lanes 0..M-1, two 16-bit K elements per 32-bit column
-// (the lower half holds the even one).
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+// kind::f16 with A read from tensor memory: a_tmem is the column of the first
+// K element, M rows in lanes 0..M-1, two 16-bit K elements per 32-bit column
+// (the lower half holds the even one).  The operand type (fp16 or bf16, the
+// same for A and B) is the instruction descriptor's.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                              uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -347,6 +349,12 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Instruction descriptor, kind::f16 with fp16 A/B and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_f16(uint32_t M, uint32_t N, bool a_mn_major,
+                                                 bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((N >> 3) << 17) | ((M >> 4) << 24);
+}
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N, bool a_mn_major,
                                                   bool b_mn_major) {
@@ -406,6 +414,18 @@ __device__ __forceinline__ float sum_bf16x2(uint32_t v) {
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+// two fp32 -> packed fp16 pair (lo in the lower half), nearest even; values
+// beyond the fp16 range become +-65504
+__device__ __forceinline__ uint32_t pack_half2_satfinite(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+// packed fp16 pair -> packed fp32 pair (exact)
+__device__ __forceinline__ uint64_t half2_as_f2(uint32_t w) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+  return f2_pack(f.x, f.y);
 }
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }

@@ -29,9 +29,9 @@
  *    asynchronous and ordered on `stream`.
  *  - Errors: arguments are validated on the host before any launch; an
  *    invalid call returns a status and launches nothing.  A failed launch
- *    returns MSA_ERR_CUDA.  Kernels never trap: a wait that runs out or a bad
- *    index is recorded in a device error word inside the workspace and read
- *    back with msa_get_device_error.
+ *    returns MSA_ERR_CUDA.  Kernels never trap: a wait that runs out, a bad
+ *    index or an input value out of range is recorded in a device error word
+ *    inside the workspace and read back with msa_get_device_error.
  *  - Supported shapes: block_size 128; head_dim and index_dim 64 or 128;
  *    1 <= top_k <= 32; G divides 128; H/G is a power of two with
  *    (H/G) * head_dim <= 2048; 1 <= N < 2^26.  Others return
@@ -67,7 +67,9 @@ typedef enum {
   MSA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than required */
   MSA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
   MSA_ERR_DEVICE_TIMEOUT = 5, /* a kernel wait ran out (reported by msa_get_device_error) */
-  MSA_ERR_DEVICE_INDEX = 6    /* a kernel met an out-of-range id (msa_get_device_error) */
+  MSA_ERR_DEVICE_INDEX = 6,   /* a kernel met an out-of-range id (msa_get_device_error) */
+  MSA_ERR_DEVICE_RANGE = 7    /* an input value outside the range it is computed in
+                                 (msa_get_device_error) */
 } msa_status_t;
 
 typedef struct {
@@ -167,7 +169,10 @@ MSA_API msa_status_t msa_build_block_query_lists(const msa_config_t* cfg, const 
  *   q [N][H][d], k/v [N][G][d], q_idx [N][G][d_idx], k_idx [N][d_idx] bf16.
  *   out [N][H][d] bf16 out: softmax over the keys s <= t of the selected
  *       blocks of softmax_scale*<q[t][h], k[s][g]>, times v[s][g]; fp32
- *       accumulation, rounded to bf16 (nearest even).
+ *       accumulation, rounded to bf16 (nearest even).  The probabilities
+ *       and v meet on the tensor cores in fp16, so v must lie within the
+ *       fp16 range (|v| <= 65504): a value beyond it, or NaN, is saturated
+ *       and recorded as 0x301 (MSA_ERR_DEVICE_RANGE) in the device error word.
  *   ids_out [N][G][k] int32 out, nullable: the selection used.
  *   ws: at least msa_prefill_min_workspace(); with less than
  *       msa_workspace_size(PREFILL, N) the query axis is processed in chunks.
@@ -304,7 +309,8 @@ MSA_API msa_status_t msa_decode_static(const msa_config_t* cfg, const void* q, c
  * above.  Synchronises `stream` first.  *code = 0 when no kernel reported a
  * problem; otherwise the first code recorded (0x1xx: a wait ran out ->
  * returns MSA_ERR_DEVICE_TIMEOUT; 0x2xx: an out-of-range id ->
- * MSA_ERR_DEVICE_INDEX).
+ * MSA_ERR_DEVICE_INDEX; 0x301: a prefill V value beyond the fp16 range, or
+ * NaN -> MSA_ERR_DEVICE_RANGE).
  */
 MSA_API msa_status_t msa_get_device_error(void* ws, msa_stream_t stream, uint32_t* code);
 

@@ -196,6 +196,46 @@ def test_prefill_32k_sampled_rows(msa):
     assert torch.isfinite(out.float()).all()
 
 
+@pytest.mark.slow
+def test_prefill_32k_all_rows(msa):
+    """The 32K workload checked on every one of its 32,768 query rows (the
+    oracle walks the rows in chunks of 4,096; a few minutes of host time)."""
+    s = synth.PREFILL_CONFIGS["prefill_32k"]
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    ws = torch.empty(msa.msa_workspace_size(cfg, msa.OP_PREFILL, s.N), dtype=torch.uint8,
+                     device="cuda")
+    out, ids = msa.msa_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                               ids_out=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_error(ws) == 0
+    g_ids = ids.cpu().numpy()
+    g_out = out.float().cpu().numpy()
+    host = {name: inp[name].cpu() for name in ("q", "k", "v", "q_idx", "k_idx")}
+    del inp, out, ids, ws
+    ties, max_err, err_sum = [], 0.0, 0.0
+    for r0 in range(0, s.N, 4096):
+        rows = np.arange(r0, min(r0 + 4096, s.N))
+        ref = oracle.prefill(host["q"], host["k"], host["v"], host["q_idx"], host["k_idx"],
+                             block=s.block, top_k=s.top_k, scale=s.scale, rows=rows)
+        parity.check_id_rows_valid(g_ids[rows], rows, s.block, s.top_k)
+        t = parity.compare_ids(g_ids[rows], ref["ids"], ref["pooled"], rows, s.block, s.top_k)
+        ref_out = ref["out"]
+        if t:  # the oracle's Main Branch on the GPU's selection
+            ref_out = oracle.block_attention(oracle.as_bf16_bits(host["q"])[rows], rows,
+                                             host["k"], host["v"], g_ids[rows], s.scale,
+                                             s.block)
+        ties += t
+        err = np.abs(g_out[rows].astype(np.float64) - ref_out)
+        max_err = max(max_err, float(err.max()))
+        err_sum += float(err.sum())
+    mean_err = err_sum / g_out.size
+    assert np.isfinite(g_out).all()
+    assert max_err <= parity.OUT_MAX_ABS, max_err
+    assert mean_err <= parity.OUT_MEAN_ABS, mean_err
+    assert len(ties) <= 64, len(ties)
+
+
 def _check_sampled_large(msa, s, n_rows, ws_bytes, seed):
     """Prefill of a long workload in the benchmark's launch configuration
     (chunked query axis when the workspace is capped), checked on sampled rows
