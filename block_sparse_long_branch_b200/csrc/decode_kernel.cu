@@ -175,7 +175,8 @@ struct AttnSmem {
       int32_t cand_i[kCandCap];
     };
   };
-  __nv_bfloat16 p[NT * 8][kBlock + 8];  // P (heads x keys), padded rows
+  __nv_bfloat16 p[NT * 8][kBlock + 8];     // P (heads x keys), padded rows: bf16(p)
+  __nv_bfloat16 p_lo[NT * 8][kBlock + 8];  // and the rest, bf16(p - bf16(p))
   float red_m[kAttnWarps][NT * 8];
   float red_l[kAttnWarps][NT * 8];
   float m_run[NT * 8], l_run[NT * 8], alpha[NT * 8];
@@ -502,21 +503,28 @@ __global__ void __launch_bounds__(kAttnThreads)
       sm.m_run[tid] = mn;
     }
     __syncthreads();
-    // ---- P = exp2(S - m) in bf16 (heads x keys), row sums of the rounded values ----
+    // ---- P = exp2(S - m) (heads x keys) as two bf16 parts, hi = bf16(p) and
+    // lo = bf16(p - hi), so that the PV product sees p to about 16 significant
+    // bits (bf16 alone, 8 bits, is too coarse for a softmax over a handful of
+    // keys); row sums of the unrounded values ----
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int h0 = nt * 8 + 2 * tq, h1 = h0 + 1;
       const float mh0 = sm.m_run[h0], mh1 = sm.m_run[h1];
-      const __nv_bfloat16 p00 = __float2bfloat16_rn(fast_exp2(sacc[nt][0] - mh0));
-      const __nv_bfloat16 p01 = __float2bfloat16_rn(fast_exp2(sacc[nt][1] - mh1));
-      const __nv_bfloat16 p10 = __float2bfloat16_rn(fast_exp2(sacc[nt][2] - mh0));
-      const __nv_bfloat16 p11 = __float2bfloat16_rn(fast_exp2(sacc[nt][3] - mh1));
+      const float e00 = fast_exp2(sacc[nt][0] - mh0), e01 = fast_exp2(sacc[nt][1] - mh1);
+      const float e10 = fast_exp2(sacc[nt][2] - mh0), e11 = fast_exp2(sacc[nt][3] - mh1);
+      const __nv_bfloat16 p00 = __float2bfloat16_rn(e00), p01 = __float2bfloat16_rn(e01);
+      const __nv_bfloat16 p10 = __float2bfloat16_rn(e10), p11 = __float2bfloat16_rn(e11);
       sm.p[h0][k0] = p00;
       sm.p[h1][k0] = p01;
       sm.p[h0][k1] = p10;
       sm.p[h1][k1] = p11;
-      float l0 = __bfloat162float(p00) + __bfloat162float(p10);
-      float l1 = __bfloat162float(p01) + __bfloat162float(p11);
+      sm.p_lo[h0][k0] = __float2bfloat16_rn(e00 - __bfloat162float(p00));
+      sm.p_lo[h1][k0] = __float2bfloat16_rn(e01 - __bfloat162float(p01));
+      sm.p_lo[h0][k1] = __float2bfloat16_rn(e10 - __bfloat162float(p10));
+      sm.p_lo[h1][k1] = __float2bfloat16_rn(e11 - __bfloat162float(p11));
+      float l0 = e00 + e10;
+      float l1 = e01 + e11;
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
         l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -555,9 +563,11 @@ __global__ void __launch_bounds__(kAttnThreads)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const __nv_bfloat16* prow = &sm.p[nt * 8 + gq][kk * 16 + 2 * tq];
-          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(prow);
-          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(prow + 8);
-          mma_bf16_16816(oacc[nt], a0, a1, a2, a3, b0, b1);
+          const __nv_bfloat16* lrow = &sm.p_lo[nt * 8 + gq][kk * 16 + 2 * tq];
+          mma_bf16_16816(oacc[nt], a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(prow),
+                         *reinterpret_cast<const uint32_t*>(prow + 8));
+          mma_bf16_16816(oacc[nt], a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(lrow),
+                         *reinterpret_cast<const uint32_t*>(lrow + 8));
         }
       }
     }

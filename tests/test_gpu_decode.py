@@ -92,6 +92,16 @@ def _check(msa, s, inp):
     return n_ties
 
 
+def test_decode_short_sequences(msa):
+    """160 sequences of 2 to 5 tokens: softmaxes over a handful of keys, whose
+    outputs reach magnitude 2 to 4, where the bf16 output rounding alone takes
+    up to 0.0078 of the 1e-2 bound."""
+    s = synth.DecodeShape("dshort", seq_lens=(2, 3, 4, 5) * 40, H=64, G=8, d=128, d_idx=128,
+                          top_k=16, seed=17)
+    inp = synth.make_decode_inputs(s, device="cuda")
+    _check(msa, s, inp)
+
+
 def test_decode_small_mixed_lengths(msa):
     s = synth.DecodeShape("ds", seq_lens=(300, 5000, 128 * 20 + 7, 128, 1, 2049), H=16, G=2,
                           d=128, d_idx=64, top_k=4, needles_per_seq=(1, 2, 2, 0, 0, 1), seed=12)
