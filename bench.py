@@ -447,7 +447,8 @@ def run_ours(args, rank, world, local):
     dk = kernels[dominant]
     roofline = {"kernel": dominant, "bound": dk["bound"], "achieved": dk["achieved"],
                 "peak": dk["peak"], "unit": dk["unit"], "frac": dk["frac"],
-                "traffic": traffic_for(dominant), "peak_source": f"{peak_src} "
+                "traffic": traffic_for(dominant, shape.name if do_prefill else None),
+                "peak_source": f"{peak_src} "
                 f"({'hbm_gbs' if dk['unit'] == 'GB/s' else tc_name})"}
 
     # ---- end to end through the public API with host buffers ----
@@ -474,8 +475,9 @@ def run_ours(args, rank, world, local):
     return line
 
 
-def traffic_for(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if it is current."""
+def traffic_for(kernel: str, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it is current and
+    was taken on this workload (null otherwise)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -483,7 +485,7 @@ def traffic_for(kernel: str):
     except (OSError, ValueError):
         return None
     ent = table.get(kernel)
-    if not ent:
+    if not ent or table.get("workload") != workload:
         return None
     src = os.path.join(ROOT, "block_sparse_long_branch_b200", "csrc", ent.get("source", ""))
     try:
