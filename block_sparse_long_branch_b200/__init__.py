@@ -456,6 +456,6 @@ def msa_get_device_error(workspace: torch.Tensor, stream=None) -> int:
     code = ctypes.c_uint32(0)
     st = load_library().msa_get_device_error(_dev(workspace, torch.uint8, "workspace"),
                                              _stream(stream), ctypes.byref(code))
-    if st not in (0, 5, 6):
+    if st not in (0, 5, 6, 7):
         _check(st, "msa_get_device_error")
     return int(code.value)
