@@ -26,6 +26,7 @@ __all__ = [
     "msa_build_block_query_lists", "msa_prefill", "msa_decode", "msa_get_device_error",
     "msa_status_string", "msa_last_launch_count", "msa_set_phase_events", "msa_decode_static",
     "msa_selftest_wait_timeout", "msa_prefill_varlen", "msa_prefill_block_alignment",
+    "msa_prefill_fp8_index",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -98,6 +99,7 @@ def load_library():
     lib.msa_build_block_query_lists.argtypes = [C, P, I64, P, P, P, SZ, P]
     lib.msa_prefill.argtypes = [C, P, P, P, P, P, I64, P, P, P, SZ, P]
     lib.msa_prefill_varlen.argtypes = [C, P, P, P, P, P, P, I32, P, P, P, SZ, P]
+    lib.msa_prefill_fp8_index.argtypes = [C, P, P, P, P, P, P, I64, P, P, P, SZ, P]
     lib.msa_prefill_block_alignment.argtypes = [C, P, P, P, P, P, I64, P, P, P, P, P, P, SZ, P]
     lib.msa_decode.argtypes = [C, P, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
     lib.msa_decode_static.argtypes = [C, P, P, P, P, P, P, I32, I64, I64, P, P, I32, P]
@@ -113,7 +115,8 @@ def load_library():
                  "msa_index_scores",
                  "msa_select_topk", "msa_quantize_index_fp8", "msa_select_topk_fp8",
                  "msa_build_block_query_lists", "msa_prefill",
-                 "msa_prefill_varlen", "msa_prefill_block_alignment", "msa_decode",
+                 "msa_prefill_varlen", "msa_prefill_block_alignment", "msa_prefill_fp8_index",
+                 "msa_decode",
                  "msa_decode_static", "msa_get_device_error", "msa_selftest_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -304,6 +307,33 @@ def msa_prefill(cfg: MsaConfig, q, k, v, q_idx, k_idx, out: Optional[torch.Tenso
                          _dev(out, torch.bfloat16, "out", (N, H, d)), ids_ptr,
                          _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(st, "msa_prefill")
+    return out if ids_out is None else (out, ids_out)
+
+
+def msa_prefill_fp8_index(cfg: MsaConfig, q, k, v, q_idx8, k_idx8, k_scale,
+                          out: Optional[torch.Tensor] = None, ids_out=None,
+                          workspace: Optional[torch.Tensor] = None, stream=None):
+    """msa_prefill with the quantised Index Branch (e4m3 index tensors and
+    per-block key scales, as msa_quantize_index_fp8 returns them)."""
+    lib = load_library()
+    N = q.shape[0]
+    H, G, d, di, kk = cfg.num_heads, cfg.num_groups, cfg.head_dim, cfg.index_dim, cfg.top_k
+    nb = (N + cfg.block_size - 1) // cfg.block_size
+    if out is None:
+        out = torch.empty((N, H, d), dtype=torch.bfloat16, device=q.device)
+    if ids_out is True:
+        ids_out = torch.empty((N, G, kk), dtype=torch.int32, device=q.device)
+    ws = _workspace(workspace, msa_workspace_size(cfg, OP_PREFILL, N), q.device)
+    ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (N, G, kk))
+    st = lib.msa_prefill_fp8_index(ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (N, H, d)),
+                                   _dev(k, torch.bfloat16, "k", (N, G, d)),
+                                   _dev(v, torch.bfloat16, "v", (N, G, d)),
+                                   _dev(q_idx8, torch.uint8, "q_idx8", (N, G, di)),
+                                   _dev(k_idx8, torch.uint8, "k_idx8", (N, di)),
+                                   _dev(k_scale, torch.float32, "k_scale", (nb,)), N,
+                                   _dev(out, torch.bfloat16, "out", (N, H, d)), ids_ptr,
+                                   _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(st, "msa_prefill_fp8_index")
     return out if ids_out is None else (out, ids_out)
 
 

@@ -395,7 +395,10 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
                          const void* q_idx, const void* k_idx, int64_t N, void* out,
                          int32_t* ids_out, void* ws, size_t ws_bytes, cudaStream_t s,
                          bool events, int* launches_out, float* block_score = nullptr,
-                         float* block_mass = nullptr, float* kl = nullptr) {
+                         float* block_mass = nullptr, float* kl = nullptr,
+                         const float* k_scale = nullptr) {
+  // k_scale set: q_idx / k_idx are e4m3 bytes and the selection is the
+  // quantised one (d_idx 128); no alignment outputs in that case
   const int64_t nb = n_blocks(N);
   const bool own_ids = ids_out == nullptr;
   const int64_t chunk = prefill_chunk(cfg, N, ws_bytes, own_ids);
@@ -428,6 +431,7 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
     ip.row_begin = t0;
     ip.row_end = t1;
     ip.ids = ids;
+    ip.kscale = k_scale;
     ip.err = err;
     ip.num_sms = sms;
     if (launch_index_select(ip, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
@@ -551,6 +555,27 @@ msa_status_t msa_prefill(const msa_config_t* cfg, const void* q, const void* k, 
   if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
   int launches = 0;
   st = prefill_run(cfg, q, k, v, q_idx, k_idx, N, out, ids_out, ws, ws_bytes, s, true, &launches);
+  g_launches = launches;
+  return st;
+}
+
+msa_status_t msa_prefill_fp8_index(const msa_config_t* cfg, const void* q, const void* k,
+                                   const void* v, const void* q_idx8, const void* k_idx8,
+                                   const float* k_scale, int64_t N, void* out, int32_t* ids_out,
+                                   void* ws, size_t ws_bytes, msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  if (cfg->index_dim != 128) return MSA_ERR_UNSUPPORTED;
+  if ((st = check_prefill_ptrs(q, k, v, q_idx8, k_idx8, out, ids_out, ws)) != MSA_OK) return st;
+  if (!k_scale) return MSA_ERR_INVALID_ARG;
+  if (prefill_chunk(cfg, N, ws_bytes, ids_out == nullptr) == 0) return MSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  int launches = 0;
+  st = prefill_run(cfg, q, k, v, q_idx8, k_idx8, N, out, ids_out, ws, ws_bytes, s, true,
+                   &launches, nullptr, nullptr, nullptr, k_scale);
   g_launches = launches;
   return st;
 }

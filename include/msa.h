@@ -211,6 +211,21 @@ MSA_API msa_status_t msa_select_topk_fp8(const msa_config_t* cfg, const void* q_
                                          msa_stream_t stream);
 
 /*
+ * msa_prefill with the quantised Index Branch: the selection of
+ * msa_select_topk_fp8 on e4m3 index tensors (as msa_quantize_index_fp8
+ * writes them), then the same query lists, Main Branch and merge.
+ *   q [N][H][d], k/v [N][G][d] bf16; q_idx8 [N][G][128], k_idx8 [N][128] e4m3
+ *   bytes; k_scale [ceil(N/128)] fp32 (device, every entry finite and > 0).
+ *   Other arguments, the workspace and the chunking as for msa_prefill.
+ * d_idx other than 128 -> MSA_ERR_UNSUPPORTED.
+ */
+MSA_API msa_status_t msa_prefill_fp8_index(const msa_config_t* cfg, const void* q, const void* k,
+                                           const void* v, const void* q_idx8, const void* k_idx8,
+                                           const float* k_scale, int64_t N, void* out,
+                                           int32_t* ids_out, void* ws, size_t ws_bytes,
+                                           msa_stream_t stream);
+
+/*
  * msa_prefill plus the data of the Index Branch's KL alignment, forward only:
  * the Index Branch is trained to bring its distribution of block scores
  * close to the distribution of where the Main Branch's exact attention went

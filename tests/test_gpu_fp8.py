@@ -127,3 +127,42 @@ def test_fp8_rejects_other_index_dims(msa):
         msa.msa_quantize_index_fp8(cfg, torch.zeros((s.N, s.G, 64), dtype=torch.bfloat16,
                                                     device="cuda"),
                                    torch.zeros((s.N, 64), dtype=torch.bfloat16, device="cuda"))
+
+
+@pytest.mark.parametrize("chunked", [False, True])
+def test_prefill_fp8_index_matches_oracle(msa, chunked):
+    """Whole prefill on the quantised Index Branch: the selection of the oracle
+    on the dequantised index values, then its fp64 Main Branch; in one pass
+    and with a workspace small enough to chunk the query axis."""
+    s = synth.PrefillShape("pf8", N=4096 + 77, H=8, G=2, d=128, d_idx=128, top_k=16,
+                           n_needles=8, seed=64)
+    inp = synth.make_prefill_inputs(s, device="cpu")
+    q8, k8, ks = oracle.quantize_index_fp8(inp["q_idx"], inp["k_idx"])
+    cfg = _cfg(msa, s)
+    ws_bytes = msa.msa_workspace_size(cfg, msa.OP_PREFILL, s.N)
+    if chunked:
+        ws_bytes = msa.msa_prefill_min_workspace(cfg, s.N) + (ws_bytes >> 3)
+        assert msa.msa_prefill_chunk_tokens(cfg, s.N, ws_bytes) < s.N
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    dev = {n: inp[n].cuda() for n in ("q", "k", "v")}
+    out, ids = msa.msa_prefill_fp8_index(cfg, dev["q"], dev["k"], dev["v"],
+                                         torch.from_numpy(q8).cuda(),
+                                         torch.from_numpy(k8).cuda(),
+                                         torch.from_numpy(ks).cuda(), ids_out=True,
+                                         workspace=ws)
+    assert msa.msa_get_device_error(ws) == 0
+    g_ids = ids.cpu().numpy()
+    rows = np.arange(s.N)
+    pooled = oracle.pooled_scores_fp8(q8, rows, k8, ks, s.block, s.nb)
+    ref_ids = oracle.select_blocks(pooled, rows, s.block, s.top_k)
+    parity.check_id_rows_valid(g_ids, rows, s.block, s.top_k)
+    fin = pooled[np.isfinite(pooled)]
+    ties = parity.compare_ids(g_ids, ref_ids, pooled, rows, s.block, s.top_k,
+                              tol=1e-5 * float(np.abs(fin).max()))
+    assert len(ties) <= 8, ties
+    sel = g_ids if ties else ref_ids
+    ref_out = oracle.block_attention(oracle.as_bf16_bits(inp["q"]), rows, inp["k"], inp["v"],
+                                     sel, s.scale, s.block)
+    parity.check_output(out.float().cpu().numpy(), ref_out)
+    for (j, g, t) in inp["needles"]:
+        assert j in g_ids[t, g]
