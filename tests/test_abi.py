@@ -113,8 +113,9 @@ def test_missing_workspace_rejected():
 
 
 def test_status_strings():
-    for s in range(7):
+    for s in range(8):
         assert msa.msa_status_string(s)
+    assert msa.msa_status_string(7) != msa.msa_status_string(99)
 
 
 def test_selftest_arguments_checked_before_any_launch():
@@ -141,3 +142,26 @@ def test_varlen_offsets_checked_before_any_launch():
     assert call([0, 0, 0]) == 1     # nothing to do
     assert lib.msa_prefill_varlen(ctypes.byref(cfg), p, p, p, p, p, None, 1, p, None, ws, 1 << 30,
                                   None) == 1
+
+
+def test_fp8_entry_points_checked_before_any_launch():
+    lib = msa.load_library()
+    p = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 21)
+    cfg = msa.config(8, 2, 128, 128, top_k=16)
+    cfg64 = msa.config(8, 2, 128, 64, top_k=16)
+    # the key scales are required
+    assert lib.msa_prefill_fp8_index(ctypes.byref(cfg), p, p, p, p, p, None, 256, p, None, ws,
+                                     1 << 30, None) == 1
+    assert lib.msa_select_topk_fp8(ctypes.byref(cfg), p, p, None, 256, p, ws, 1 << 20,
+                                   None) == 1
+    assert lib.msa_quantize_index_fp8(ctypes.byref(cfg), p, p, 256, p, p, None, None) == 1
+    # e4m3 index tensors only with d_idx = 128
+    assert lib.msa_prefill_fp8_index(ctypes.byref(cfg64), p, p, p, p, p, p, 256, p, None, ws,
+                                     1 << 30, None) == 2
+    assert lib.msa_select_topk_fp8(ctypes.byref(cfg64), p, p, p, 256, p, ws, 1 << 20,
+                                   None) == 2
+    assert lib.msa_quantize_index_fp8(ctypes.byref(cfg64), p, p, 256, p, p, p, None) == 2
+    # no tokens
+    assert lib.msa_prefill_fp8_index(ctypes.byref(cfg), p, p, p, p, p, p, 0, p, None, ws,
+                                     1 << 30, None) == 1
