@@ -55,6 +55,9 @@ msa_status_t check_tokens(const msa_config_t* c, int64_t n) {
   return MSA_OK;
 }
 
+// decode attention tiles a group's heads in 8s, at most two tiles
+constexpr int kDecodeMaxHeadsPerGroup = 16;
+
 int64_t n_blocks(int64_t n) { return (n + kBlock - 1) / kBlock; }
 
 int sm_count() {
@@ -192,6 +195,7 @@ msa_status_t msa_workspace_size(const msa_config_t* cfg, msa_op_t op, int64_t n_
   if (st != MSA_OK) return st;
   if (!bytes) return MSA_ERR_INVALID_ARG;
   if (op == MSA_OP_DECODE) {
+    if (cfg->num_heads / cfg->num_groups > kDecodeMaxHeadsPerGroup) return MSA_ERR_UNSUPPORTED;
     // total cache rows over all sequences; only per-sequence lengths are bounded
     if (n_tokens < 1 || batch < 1 || batch > n_tokens || n_tokens >= (int64_t(1) << 40))
       return MSA_ERR_INVALID_ARG;
@@ -658,6 +662,7 @@ msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_id
   g_launches = 0;
   msa_status_t st = check_cfg(cfg);
   if (st != MSA_OK) return st;
+  if (cfg->num_heads / cfg->num_groups > kDecodeMaxHeadsPerGroup) return MSA_ERR_UNSUPPORTED;
   if (!q || !q_idx || !k_cache || !v_cache || !k_idx_cache || !cu_seqlens || !out)
     return MSA_ERR_INVALID_ARG;
   if (B < 1 || max_seqlen < 1) return MSA_ERR_INVALID_ARG;

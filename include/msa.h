@@ -288,6 +288,7 @@ MSA_API msa_status_t msa_prefill_varlen(const msa_config_t* cfg, const void* q, 
  *   max_seqlen: host value >= every L_b (sizes the grid);
  *   out [B][H][d] bf16 out; ids_out [B][G][k] int32 out, nullable.
  *   ws: at least msa_workspace_size(cfg, MSA_OP_DECODE, sum L, B).
+ * H/G above 16 -> MSA_ERR_UNSUPPORTED (here and in the decode workspace size).
  */
 MSA_API msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_idx,
                         const void* k_cache, const void* v_cache, const void* k_idx_cache,

@@ -165,3 +165,17 @@ def test_fp8_entry_points_checked_before_any_launch():
     # no tokens
     assert lib.msa_prefill_fp8_index(ctypes.byref(cfg), p, p, p, p, p, p, 0, p, None, ws,
                                      1 << 30, None) == 1
+
+
+def test_decode_heads_per_group_limit():
+    """Decode tiles a group's heads in 8s, at most 16; prefill takes up to 2048/d."""
+    lib = msa.load_library()
+    cfg32 = msa.config(32, 1, 64, 64, top_k=4)   # 32 heads per group, d = 64
+    n = ctypes.c_size_t(0)
+    assert lib.msa_workspace_size(ctypes.byref(cfg32), msa.OP_DECODE, 1024, 2, ctypes.byref(n)) == 2
+    assert lib.msa_workspace_size(ctypes.byref(cfg32), msa.OP_PREFILL, 1024, 0, ctypes.byref(n)) == 0
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.msa_decode(ctypes.byref(cfg32), p, p, p, p, p, p, 2, 512, p, None, p, 1 << 30,
+                          None) == 2
+    cfg16 = msa.config(32, 2, 128, 128, top_k=4)  # 16 heads per group: supported
+    assert lib.msa_workspace_size(ctypes.byref(cfg16), msa.OP_DECODE, 1024, 2, ctypes.byref(n)) == 0

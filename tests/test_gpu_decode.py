@@ -102,6 +102,14 @@ def test_decode_short_sequences(msa):
     _check(msa, s, inp)
 
 
+def test_decode_sixteen_heads_per_group(msa):
+    """16 query heads per group: the attention's two 8-head tiles."""
+    s = synth.DecodeShape("d16", seq_lens=(3, 300, 4097, 2, 128 * 9 + 1, 5000), H=32, G=2,
+                          d=128, d_idx=128, top_k=16, needles_per_seq=(0, 1, 2, 0, 1, 2), seed=19)
+    inp = synth.make_decode_inputs(s, device="cuda")
+    _check(msa, s, inp)
+
+
 def test_decode_small_mixed_lengths(msa):
     s = synth.DecodeShape("ds", seq_lens=(300, 5000, 128 * 20 + 7, 128, 1, 2049), H=16, G=2,
                           d=128, d_idx=64, top_k=4, needles_per_seq=(1, 2, 2, 0, 0, 1), seed=12)

@@ -153,7 +153,8 @@ def test_prefill_tiny_topk32_equals_dense(msa):
 
 
 @pytest.mark.parametrize("N,H,G,d,di,k", [(1000, 16, 2, 128, 128, 16), (1333, 8, 8, 64, 128, 3),
-                                         (777, 32, 4, 128, 64, 32), (129, 8, 1, 64, 64, 1)])
+                                         (777, 32, 4, 128, 64, 32), (129, 8, 1, 64, 64, 1),
+                                         (1500, 32, 2, 128, 128, 16), (700, 32, 1, 64, 64, 8)])
 def test_prefill_ragged_shapes(msa, N, H, G, d, di, k):
     s = synth.PrefillShape("r", N=N, H=H, G=G, d=d, d_idx=di, top_k=k, n_needles=3,
                            seed=N * 7 + H)
