@@ -115,7 +115,7 @@ __device__ __forceinline__ Unit make_unit(const IdxArgs& a, int v) {
 __device__ __forceinline__ void max_chains_ordered(float (&x)[8], const uint32_t (&r)[32]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i)
-    x[i & 7] = fmax3_ordered(x[i & 7], __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+    x[i & 7] = max3f_ordered(x[i & 7], __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
 }
 
 template <int DI, int MAXSEL, bool SCORES, bool FP8>
@@ -337,8 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c + 2 < 8) tmem_ld_32x32b_x32(col + (c + 2) * 32, ra);
             max_chains_ordered(x, rb);
             if ((c & 3) == 2)
-              m[c >> 2] = fmax3_ordered(fmax3_ordered(x[0], x[1], x[2]),
-                                        fmax3_ordered(x[3], x[4], x[5]), fmaxf(x[6], x[7]));
+              m[c >> 2] = max3f_ordered(max3f_ordered(x[0], x[1], x[2]),
+                                        max3f_ordered(x[3], x[4], x[5]), fmaxf(x[6], x[7]));
             if (c + 2 < 8) {
               tmem_wait();
               reg_fence(ra);

@@ -74,19 +74,6 @@ __device__ __forceinline__ bool mbar_test(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking probe of the phase with the given parity.
-__device__ __forceinline__ bool mbar_probe(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // if the CTA-wide abort flag is raised (by this or another thread) or the
 // time limit passes; in the latter case the abort flag and the error word are
@@ -287,17 +274,8 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
                : "memory");
 }
 
-// 32 TMEM lanes x 16 consecutive 32-bit columns from registers; thread i of the
+// 32 TMEM lanes x 8 consecutive 32-bit columns from registers; thread i of the
 // warp writes lane (lane base + i).  Complete only after tmem_wait_st().
-__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
 __device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
@@ -320,20 +298,6 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-// max(a, b, c) in one instruction (three-input max.f32, sm_100 and later);
-// a NaN operand is ignored as fmaxf ignores it.
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-// The same, kept in program order with the other volatile asm (TMEM loads and
-// waits), so a reduction is not deferred past the load that follows it.
-__device__ __forceinline__ float fmax3_ordered(float a, float b, float c) {
-  float d;
-  asm volatile("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
 
 // Shared-memory matrix descriptor for tcgen05.mma, 128-byte swizzle, sm_100
 // layout (version field = 1).  For a K-major operand the 8-row groups are
@@ -397,20 +361,21 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+// max(a, b, c) in one instruction (three-input max.f32, sm_100 and later);
+// a NaN operand is ignored as fmaxf ignores it.
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// the two bf16 halves of a packed pair as an fp32 pair (exact)
-__device__ __forceinline__ uint64_t bf16x2_as_f2(uint32_t w) {
-  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+// The same, kept in program order with the other volatile asm (TMEM loads and
+// waits), so a reduction is not deferred past the load that follows it.
+__device__ __forceinline__ float max3f_ordered(float a, float b, float c) {
+  float d;
+  asm volatile("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
-__device__ __forceinline__ float sum_bf16x2(uint32_t v) {
-  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
-  return f.x + f.y;
-}
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
