@@ -34,7 +34,9 @@ def _deps_hash() -> str:
             h.update(name.encode() + f.read())
     with open(HEADER, "rb") as f:
         h.update(f.read())
-    h.update(" ".join(FLAGS).encode())
+    # the flags without the include paths: those are absolute and differ between
+    # checkouts of the same sources
+    h.update(" ".join(f for f in FLAGS if not f.startswith("-I")).encode())
     return h.hexdigest()[:16]
 
 
