@@ -126,3 +126,86 @@ def test_group_range_splits_evenly():
     assert [shard.group_range(8, r, 4) for r in range(4)] == [(0, 2), (2, 4), (4, 6), (6, 8)]
     with pytest.raises(ValueError):
         shard.group_range(8, 0, 3)
+
+
+def _seq_shard_worker(rank, world, port, lens, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank), OMP_NUM_THREADS="2")
+    import torch
+    import torch.distributed as dist
+    import oracle
+    import synth
+    import block_sparse_long_branch_b200 as msa
+    from block_sparse_long_branch_b200 import shard
+    dist.init_process_group("gloo")
+    try:
+        s = synth.DecodeShape("dshard", seq_lens=tuple(lens), H=8, G=2, d=64, d_idx=64,
+                              top_k=4, seed=23)
+        inp = synth.make_decode_inputs(s, device="cpu")
+        cfg = msa.config(s.H, s.G, s.d, s.d_idx, top_k=s.top_k, scale=s.scale)
+
+        def oracle_shard(c, qq, qi, kc, vc, kic, cu):
+            r = oracle.decode(qq, qi, kc, vc, kic, cu.numpy(), block=c.block_size,
+                              top_k=c.top_k, scale=c.softmax_scale)
+            return (torch.from_numpy(r["out"]).to(torch.bfloat16),
+                    torch.from_numpy(r["ids"]))
+
+        cu = inp["cu_seqlens"].tolist()
+        out, ids = shard.sequence_sharded_decode(cfg, inp["q"], inp["q_idx"], inp["k_cache"],
+                                                 inp["v_cache"], inp["k_idx_cache"], cu,
+                                                 decode=oracle_shard)
+        mine = shard.sequence_range(cu, rank, world)
+        if rank == 0:
+            full = oracle.decode(inp["q"], inp["q_idx"], inp["k_cache"], inp["v_cache"],
+                                 inp["k_idx_cache"], cu, block=s.block, top_k=s.top_k,
+                                 scale=s.scale)
+            same = (torch.equal(out, torch.from_numpy(full["out"]).to(torch.bfloat16)) and
+                    torch.equal(ids, torch.from_numpy(full["ids"])))
+            q.put(("ok", same, tuple(out.shape), mine))
+        else:
+            q.put(("rank", None, None, mine))
+    except Exception as e:  # report instead of hanging the parent
+        q.put(("error", repr(e), None, None))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("lens", [[300, 700, 129, 2000, 50], [4000]])
+def test_sequence_sharded_decode_equals_one_rank(lens):
+    """Two gloo ranks split the batch by cached length (with one sequence, rank 0
+    has none); the gathered outputs equal the unsharded oracle's."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_seq_shard_worker, args=(r, world, port, lens, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=240) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+    errors = [g for g in got if g[0] == "error"]
+    assert not errors, errors
+    main = next(g for g in got if g[0] == "ok")
+    assert main[1] and main[2] == (len(lens), 8, 64)
+    ranges = sorted(g[3] for g in got)
+    assert ranges[0][0] == 0 and ranges[-1][1] == len(lens)
+    for p in procs:
+        assert p.exitcode == 0
+
+
+def test_sequence_range_balances_cached_length():
+    from block_sparse_long_branch_b200 import shard
+    cu = [0]
+    for L in [262144] * 16 + [1048576]:
+        cu.append(cu[-1] + L)
+    assert [shard.sequence_range(cu, r, 2) for r in range(2)] == [(0, 10), (10, 17)]
+    parts = [shard.sequence_range(cu, r, 8) for r in range(8)]
+    assert parts[0][0] == 0 and parts[-1] == (16, 17)
+    assert all(a[1] == b[0] for a, b in zip(parts, parts[1:]))
+    # one sequence: its middle lies in rank 1's half, rank 0 has none
+    assert shard.sequence_range([0, 4000], 0, 2) == (0, 0)
+    assert shard.sequence_range([0, 4000], 1, 2) == (0, 1)

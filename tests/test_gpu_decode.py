@@ -169,3 +169,30 @@ def test_decode_clustered_high_scores(msa):
                 r0 = cu[b] + j * s.block
                 kic[r0:r0 + s.block] = (u * (1.0 + 1e-3 * j)).to(torch.bfloat16)
     _check(msa, s, inp)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_shards_equal_whole_decode(msa, world):
+    """The sequence-sharded decode's per-rank calls on one GPU: shards run with
+    the library's msa_decode and concatenated in rank order give the whole
+    batch's ids exactly, and its outputs up to the order of the split merge."""
+    from block_sparse_long_branch_b200 import shard
+    s = synth.DecodeShape("dsh", seq_lens=(3000, 129, 70000, 4096, 1, 20000, 640), H=16, G=2,
+                          d=128, d_idx=128, top_k=16, seed=29)
+    inp = synth.make_decode_inputs(s, device="cuda")
+    whole_out, whole_ids = _run(msa, s, inp)
+    cu = inp["cu_seqlens"].tolist()
+    cfg = _cfg(msa, s)
+    outs, ids = [], []
+    for r in range(world):
+        qq, qi, kc, vc, kic, cu_r = shard.shard_decode_inputs(
+            inp["q"], inp["q_idx"], inp["k_cache"], inp["v_cache"], inp["k_idx_cache"], cu, r,
+            world)
+        if qq.shape[0] == 0:
+            continue
+        lens = (cu_r[1:] - cu_r[:-1]).tolist()
+        o, i = msa.msa_decode(cfg, qq, qi, kc, vc, kic, cu_r.cuda(), max(lens), ids_out=True)
+        outs.append(o.float().cpu().numpy())
+        ids.append(i.cpu().numpy())
+    np.testing.assert_array_equal(np.concatenate(ids), whole_ids)
+    np.testing.assert_allclose(np.concatenate(outs), whole_out, atol=2e-3, rtol=0)
