@@ -26,7 +26,7 @@ __all__ = [
     "msa_build_block_query_lists", "msa_prefill", "msa_decode", "msa_get_device_error",
     "msa_status_string", "msa_last_launch_count", "msa_set_phase_events", "msa_decode_static",
     "msa_selftest_wait_timeout", "msa_prefill_varlen", "msa_prefill_block_alignment",
-    "msa_prefill_fp8_index",
+    "msa_prefill_fp8_index", "msa_prefill_varlen_workspace_size",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -99,6 +99,7 @@ def load_library():
     lib.msa_build_block_query_lists.argtypes = [C, P, I64, P, P, P, SZ, P]
     lib.msa_prefill.argtypes = [C, P, P, P, P, P, I64, P, P, P, SZ, P]
     lib.msa_prefill_varlen.argtypes = [C, P, P, P, P, P, P, I32, P, P, P, SZ, P]
+    lib.msa_prefill_varlen_workspace_size.argtypes = [C, P, I32, ctypes.POINTER(SZ)]
     lib.msa_prefill_fp8_index.argtypes = [C, P, P, P, P, P, P, I64, P, P, P, SZ, P]
     lib.msa_prefill_block_alignment.argtypes = [C, P, P, P, P, P, I64, P, P, P, P, P, P, SZ, P]
     lib.msa_decode.argtypes = [C, P, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
@@ -115,7 +116,8 @@ def load_library():
                  "msa_index_scores",
                  "msa_select_topk", "msa_quantize_index_fp8", "msa_select_topk_fp8",
                  "msa_build_block_query_lists", "msa_prefill",
-                 "msa_prefill_varlen", "msa_prefill_block_alignment", "msa_prefill_fp8_index",
+                 "msa_prefill_varlen", "msa_prefill_varlen_workspace_size",
+                 "msa_prefill_block_alignment", "msa_prefill_fp8_index",
                  "msa_decode",
                  "msa_decode_static", "msa_get_device_error", "msa_selftest_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
@@ -364,6 +366,20 @@ def msa_prefill_block_alignment(cfg: MsaConfig, q, k, v, q_idx, k_idx,
     return out, ids, score, mass, kl
 
 
+def msa_prefill_varlen_workspace_size(cfg: MsaConfig, cu_seqlens) -> int:
+    """Bytes of workspace with which msa_prefill_varlen runs the batch in one
+    pass (or, beyond 1024 sequences, each sequence without chunking)."""
+    import numpy as _np
+    cu = _np.ascontiguousarray(_np.asarray(
+        cu_seqlens.cpu() if isinstance(cu_seqlens, torch.Tensor) else cu_seqlens,
+        dtype=_np.int64))
+    out = ctypes.c_size_t(0)
+    _check(load_library().msa_prefill_varlen_workspace_size(
+        ctypes.byref(cfg), cu.ctypes.data_as(ctypes.c_void_p), len(cu) - 1, ctypes.byref(out)),
+        "msa_prefill_varlen_workspace_size")
+    return int(out.value)
+
+
 def msa_prefill_varlen(cfg: MsaConfig, q, k, v, q_idx, k_idx, cu_seqlens,
                        out: Optional[torch.Tensor] = None, ids_out=None,
                        workspace: Optional[torch.Tensor] = None, stream=None):
@@ -383,8 +399,7 @@ def msa_prefill_varlen(cfg: MsaConfig, q, k, v, q_idx, k_idx, cu_seqlens,
         out = torch.empty((T, H, d), dtype=torch.bfloat16, device=q.device)
     if ids_out is True:
         ids_out = torch.empty((T, G, kk), dtype=torch.int32, device=q.device)
-    max_len = int(_np.max(_np.diff(cu)))
-    ws = _workspace(workspace, msa_workspace_size(cfg, OP_PREFILL, max(max_len, 1)), q.device)
+    ws = _workspace(workspace, msa_prefill_varlen_workspace_size(cfg, cu), q.device)
     ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (T, G, kk))
     st = lib.msa_prefill_varlen(ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (T, H, d)),
                                 _dev(k, torch.bfloat16, "k", (T, G, d)),

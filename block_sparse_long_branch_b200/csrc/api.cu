@@ -531,6 +531,162 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
   return MSA_OK;
 }
 
+// ---- a batch of packed sequences in one pass --------------------------------
+// Every kernel runs once over the whole batch: the Index Branch walks a table
+// of (sequence, query block) tiles with keys offset to the sequence's first
+// row, the query lists number key blocks globally (blk_base[b] + local id), and
+// the Main Branch reads each block's K/V from its sequence's rows.  A
+// sequence's last block may be partial; it is only ever its own tokens' local
+// block, so the causal mask already hides the next sequence's rows behind it.
+struct PackedLayout {
+  PrefillLayout base;
+  size_t nbs, blk_base, level, units, blk_row0, row_base, total;
+};
+
+PackedLayout packed_layout(const msa_config_t* c, int64_t N, int32_t B, int32_t NB,
+                           int32_t max_nb, bool own_ids) {
+  PackedLayout P;
+  P.base = prefill_layout(c, N, N, NB, own_ids);
+  size_t off = P.base.total;
+  P.nbs = off;
+  off += align256((size_t)B * 4);
+  P.blk_base = off;
+  off += align256((size_t)(B + 1) * 4);
+  P.level = off;
+  off += align256((size_t)(max_nb + 1) * 4);
+  P.units = off;
+  off += align256((size_t)NB * 16);
+  P.blk_row0 = off;
+  off += align256((size_t)NB * 4);
+  P.row_base = off;
+  off += align256((size_t)N * 4);
+  P.total = off;
+  return P;
+}
+
+// Runs the batch in one pass if it fits `ws_bytes` (and has at most
+// kVarlenMaxSeqs sequences); *ran = false leaves it to the per-sequence path.
+msa_status_t prefill_packed(const msa_config_t* cfg, const void* q, const void* k, const void* v,
+                            const void* q_idx, const void* k_idx, const int64_t* cu, int32_t B,
+                            void* out, int32_t* ids_out, void* ws, size_t ws_bytes,
+                            cudaStream_t s, int* launches_out, bool* ran) {
+  *ran = false;
+  if (B > kVarlenMaxSeqs) return MSA_OK;
+  const int64_t N = cu[B];
+  int64_t NB = 0, max_nb = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    const int64_t nb = (cu[b + 1] - cu[b] + kBlock - 1) / kBlock;
+    NB += nb;
+    if (nb > max_nb) max_nb = nb;
+  }
+  if (check_tokens(cfg, N) != MSA_OK || NB >= (int64_t(1) << 30)) return MSA_OK;
+  const bool own_ids = ids_out == nullptr;
+  const PackedLayout P = packed_layout(cfg, N, B, (int32_t)NB, (int32_t)max_nb, own_ids);
+  if (P.total > ws_bytes) return MSA_OK;
+  *ran = true;
+  const PrefillLayout& L = P.base;
+  const int G = cfg->num_groups, H = cfg->num_heads, d = cfg->head_dim, kk = cfg->top_k;
+  const int sms = sm_count();
+  uint32_t* err = at<uint32_t>(ws, 0);
+  int launches = 0;
+
+  VarlenOffsets offs;
+  offs.B = B;
+  for (int32_t b = 0; b <= B; ++b) offs.cu[b] = cu[b];
+  VarlenPlan pl{};
+  pl.N = N;
+  pl.NB = (int32_t)NB;
+  pl.max_nb = (int32_t)max_nb;
+  pl.nbs = at<int32_t>(ws, P.nbs);
+  pl.blk_base = at<int32_t>(ws, P.blk_base);
+  pl.level = at<int32_t>(ws, P.level);
+  pl.units = at<int4>(ws, P.units);
+  pl.blk_row0 = at<int32_t>(ws, P.blk_row0);
+  pl.row_base = at<int32_t>(ws, P.row_base);
+  if (launch_varlen_plan(offs, pl, s, &launches) != cudaSuccess)
+    return cuda_status(cudaErrorLaunchFailure);
+
+  int32_t* ids = own_ids ? at<int32_t>(ws, L.ids) : ids_out;
+  IndexLaunch ip{};
+  ip.q_idx = q_idx;
+  ip.k_idx = k_idx;
+  ip.N = N;
+  ip.G = G;
+  ip.d_idx = cfg->index_dim;
+  ip.top_k = kk;
+  ip.row_begin = 0;
+  ip.row_end = N;
+  ip.ids = ids;
+  ip.units = pl.units;
+  ip.n_units = (int32_t)NB;
+  ip.err = err;
+  ip.num_sms = sms;
+  if (launch_index_select(ip, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
+  ++launches;
+
+  CsrLaunch cp{};
+  cp.ids = ids;
+  cp.row_begin = 0;
+  cp.rows = N;
+  cp.G = G;
+  cp.top_k = kk;
+  cp.nb = NB;
+  cp.row_base = pl.row_base;
+  cp.row_ptr = at<int32_t>(ws, L.row_ptr);
+  cp.entries = at<int32_t>(ws, L.entries);
+  cp.scratch = at<void>(ws, L.csr);
+  cp.err = err;
+  cp.unit_ptr = at<int32_t>(ws, L.unit_ptr);
+  cp.unit_desc = at<int4>(ws, L.unit_list);
+  cp.tile_tokens = main_tile_tokens(H, G);
+  cp.unit_tiles = kUnitTiles;
+  if (launch_csr(cp, s, &launches) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
+
+  void* v16 = at<void>(ws, L.v16);
+  if (launch_v_to_fp16(v, v16, N * G * d, err, sms, s) != cudaSuccess)
+    return cuda_status(cudaErrorLaunchFailure);
+  ++launches;
+  MainLaunch mp{};
+  mp.q = q;
+  mp.k = k;
+  mp.v = v16;
+  mp.N = N;
+  mp.H = H;
+  mp.G = G;
+  mp.d = d;
+  mp.top_k = kk;
+  mp.scale = cfg->softmax_scale;
+  mp.row_begin = 0;
+  mp.rows = N;
+  mp.nb = NB;
+  mp.row_ptr = cp.row_ptr;
+  mp.entries = cp.entries;
+  mp.unit_ptr = cp.unit_ptr;
+  mp.unit_desc = cp.unit_desc;
+  mp.blk_row0 = pl.blk_row0;
+  mp.part_o = at<__half>(ws, L.part_o);
+  mp.part_lse = at<float>(ws, L.part_lse);
+  mp.err = err;
+  mp.grid = sms;
+  if (launch_main(mp, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
+  ++launches;
+
+  MergeLaunch gp{};
+  gp.part_o = mp.part_o;
+  gp.part_lse = mp.part_lse;
+  gp.ids = ids;
+  gp.rows = N;
+  gp.H = H;
+  gp.G = G;
+  gp.d = d;
+  gp.top_k = kk;
+  gp.out = out;
+  if (launch_merge(gp, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
+  ++launches;
+  *launches_out += launches;
+  return MSA_OK;
+}
+
 msa_status_t check_prefill_ptrs(const void* q, const void* k, const void* v, const void* q_idx,
                                 const void* k_idx, const void* out, const int32_t* ids_out,
                                 const void* ws) {
@@ -607,6 +763,30 @@ msa_status_t msa_prefill_block_alignment(const msa_config_t* cfg, const void* q,
   return st;
 }
 
+msa_status_t msa_prefill_varlen_workspace_size(const msa_config_t* cfg, const int64_t* cu_seqlens,
+                                               int32_t B, size_t* bytes) {
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if (!bytes || !cu_seqlens || B < 1 || cu_seqlens[0] != 0) return MSA_ERR_INVALID_ARG;
+  int64_t max_len = 0, NB = 0, max_nb = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    const int64_t L = cu_seqlens[b + 1] - cu_seqlens[b];
+    if (L < 0) return MSA_ERR_INVALID_ARG;
+    if (L > max_len) max_len = L;
+    const int64_t nb = (L + kBlock - 1) / kBlock;
+    NB += nb;
+    if (nb > max_nb) max_nb = nb;
+  }
+  if (max_len == 0) return MSA_ERR_INVALID_ARG;
+  if ((st = check_tokens(cfg, max_len)) != MSA_OK) return st;
+  const int64_t N = cu_seqlens[B];
+  if (B <= kVarlenMaxSeqs && check_tokens(cfg, N) == MSA_OK && NB < (int64_t(1) << 30))
+    *bytes = packed_layout(cfg, N, B, (int32_t)NB, (int32_t)max_nb, true).total;
+  else  // one sequence after another
+    *bytes = prefill_layout(cfg, max_len, max_len, n_blocks(max_len), true).total;
+  return MSA_OK;
+}
+
 msa_status_t msa_prefill_varlen(const msa_config_t* cfg, const void* q, const void* k,
                                 const void* v, const void* q_idx, const void* k_idx,
                                 const int64_t* cu_seqlens, int32_t B, void* out,
@@ -636,6 +816,14 @@ msa_status_t msa_prefill_varlen(const msa_config_t* cfg, const void* q, const vo
   const int64_t H = cfg->num_heads, G = cfg->num_groups, d = cfg->head_dim;
   const int64_t di = cfg->index_dim, kk = cfg->top_k;
   int launches = 0;
+  bool ran = false;
+  st = prefill_packed(cfg, q, k, v, q_idx, k_idx, cu_seqlens, B, out, ids_out, ws, ws_bytes, s,
+                      &launches, &ran);
+  if (st != MSA_OK || ran) {
+    g_launches = launches;
+    return st;
+  }
+  // too large for one pass: one sequence after another, each chunked to fit
   for (int32_t b = 0; b < B; ++b) {
     const int64_t r0 = cu_seqlens[b], L = cu_seqlens[b + 1] - r0;
     if (L == 0) continue;

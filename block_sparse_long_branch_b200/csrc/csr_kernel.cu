@@ -27,9 +27,17 @@ constexpr int kScanThreads = 1024;
 constexpr int kScanPer = 4;
 constexpr int kScanChunk = kScanThreads * kScanPer;
 
+// Packed sequences: ids are local to each sequence and row_base[row] (the
+// global number of the row's sequence's first block) turns them into the list
+// key; without it the id is the key.
+__device__ __forceinline__ int32_t list_key(const int32_t* row_base, int64_t row, int32_t j) {
+  return (row_base && j >= 0) ? __ldg(row_base + row) + j : j;
+}
+
 __global__ void __launch_bounds__(256) csr_hist_kernel(const int32_t* __restrict__ ids, int64_t rows,
                                                        int32_t G, int32_t top_k, int64_t nb,
                                                        int32_t ntiles, int32_t* __restrict__ cnt,
+                                                       const int32_t* __restrict__ row_base,
                                                        uint32_t* err) {
   extern __shared__ int32_t bins[];
   const int tile = blockIdx.x, g = blockIdx.y;
@@ -43,7 +51,7 @@ __global__ void __launch_bounds__(256) csr_hist_kernel(const int32_t* __restrict
     for (int64_t e = threadIdx.x; e < n_el; e += blockDim.x) {
       const int64_t row = r0 + e / top_k;
       const int r = (int)(e % top_k);
-      const int32_t j = ids[(row * G + g) * top_k + r];
+      const int32_t j = list_key(row_base, row, ids[(row * G + g) * top_k + r]);
       if (j < -1 || j >= nb) {
         if (s0 == 0) record_error(err, kDevBadIndex);
         continue;
@@ -147,6 +155,7 @@ __global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restri
                                                          int32_t G, int32_t top_k, int64_t nb,
                                                          int32_t ntiles,
                                                          const int32_t* __restrict__ scanned,
+                                                         const int32_t* __restrict__ row_base,
                                                          int32_t* __restrict__ entries) {
   extern __shared__ int32_t run[];
   const int tile = blockIdx.x, g = blockIdx.y;
@@ -167,7 +176,7 @@ __global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restri
       if (e < n_el) {
         row = r0 + e / top_k;
         r = (int)(e % top_k);
-        j = ids[(row * G + g) * top_k + r];
+        j = list_key(row_base, row, ids[(row * G + g) * top_k + r]);
       }
       const bool mine = j >= s0 && j < s0 + width;
       const int key = mine ? (int)(j - s0) : -1;
@@ -209,6 +218,94 @@ __global__ void unit_count_kernel(const int32_t* __restrict__ row_ptr, int64_t n
   }
 }
 
+// ---- schedule of a batch of packed sequences --------------------------------
+// One CTA: blocks per sequence, their exclusive prefix (blk_base), and the
+// first unit of every local block level b when the units are ordered by b
+// descending (the longest rows of the Index Branch first), then by sequence.
+__global__ void __launch_bounds__(1024) varlen_levels_kernel(const VarlenOffsets off,
+                                                             int32_t max_nb,
+                                                             int32_t* __restrict__ nbs,
+                                                             int32_t* __restrict__ blk_base,
+                                                             int32_t* __restrict__ level) {
+  __shared__ int32_t sh_nb[kVarlenMaxSeqs];
+  __shared__ int32_t sh_scan[1024];
+  const int tid = threadIdx.x, B = off.B;
+  for (int b = tid; b < B; b += 1024) {
+    const int32_t n = (int32_t)((off.cu[b + 1] - off.cu[b] + 127) / 128);
+    sh_nb[b] = n;
+    nbs[b] = n;
+  }
+  __syncthreads();
+  if (tid == 0) {  // B <= 1024: a serial prefix is cheap next to the kernels it plans
+    int32_t acc = 0;
+    for (int b = 0; b < B; ++b) {
+      blk_base[b] = acc;
+      acc += sh_nb[b];
+    }
+    blk_base[B] = acc;
+  }
+  // units of level b: the sequences with more than b blocks; levels from the
+  // top down, scanned in chunks of 1024 with a carry
+  int32_t carry = 0;
+  for (int32_t c0 = 0; c0 < max_nb; c0 += 1024) {
+    const int32_t b = max_nb - 1 - (c0 + tid);  // descending
+    int32_t cnt = 0;
+    if (b >= 0)
+      for (int x = 0; x < B; ++x) cnt += sh_nb[x] > b;
+    sh_scan[tid] = cnt;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan
+      const int32_t v = tid >= o ? sh_scan[tid - o] : 0;
+      __syncthreads();
+      sh_scan[tid] += v;
+      __syncthreads();
+    }
+    if (b >= 0) level[b] = carry + sh_scan[tid] - cnt;
+    carry += sh_scan[1023];
+    __syncthreads();
+  }
+  if (tid == 0) level[max_nb] = carry;
+}
+
+// largest s < B with key[s] <= x (key non-decreasing): the owner of x
+template <typename T>
+__device__ __forceinline__ int owner_of(const T* key, int B, int64_t x) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)key[mid] <= x)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+// Grid-stride: the unit table and first K/V row of every global block, and
+// the block base of every packed row.
+__global__ void __launch_bounds__(256) varlen_tables_kernel(const VarlenOffsets off, int32_t NB,
+                                                            int64_t N,
+                                                            const int32_t* __restrict__ nbs,
+                                                            const int32_t* __restrict__ blk_base,
+                                                            const int32_t* __restrict__ level,
+                                                            int4* __restrict__ units,
+                                                            int32_t* __restrict__ blk_row0,
+                                                            int32_t* __restrict__ row_base) {
+  const int B = off.B;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t J = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; J < NB; J += stride) {
+    const int s = owner_of(blk_base, B, J);
+    const int32_t b = (int32_t)(J - blk_base[s]);
+    int32_t rank = 0;  // earlier sequences on the same level
+    for (int x = 0; x < s; ++x) rank += __ldg(nbs + x) > b;
+    const int64_t r0 = off.cu[s] + (int64_t)b * 128;
+    units[level[b] + rank] = make_int4((int32_t)r0, (int32_t)off.cu[s], b, (int32_t)off.cu[s + 1]);
+    blk_row0[J] = (int32_t)r0;
+  }
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < N; t += stride)
+    row_base[t] = __ldg(blk_base + owner_of(off.cu, B, t));
+}
+
 }  // namespace
 
 size_t csr_scratch_bytes(int64_t rows, int32_t G, int32_t top_k, int64_t nb) {
@@ -242,7 +339,7 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
       return e;
   }
   csr_hist_kernel<<<grid, 256, bins * sizeof(int32_t), s>>>(p.ids, p.rows, p.G, p.top_k, p.nb,
-                                                           (int32_t)ntiles, cnt, p.err);
+                                                           (int32_t)ntiles, cnt, p.row_base, p.err);
   ++*launches;
   if ((e = cudaMemcpyAsync(last, cnt + table - 1, sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) !=
       cudaSuccess)
@@ -255,7 +352,7 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
   ++*launches;
   csr_scatter_kernel<<<grid, 32, bins * sizeof(int32_t), s>>>(p.ids, p.row_begin, p.rows, p.G,
                                                              p.top_k, p.nb, (int32_t)ntiles, cnt,
-                                                             p.entries);
+                                                             p.row_base, p.entries);
   ++*launches;
   if (p.unit_ptr) {
     unit_count_kernel<<<(unsigned)((n_lists + 255) / 256), 256, 0, s>>>(
@@ -268,6 +365,21 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
         p.unit_ptr, p.row_ptr, n_lists, p.nb, p.tile_tokens * p.unit_tiles, p.unit_desc);
     ++*launches;
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_varlen_plan(const VarlenOffsets& off, const VarlenPlan& p, cudaStream_t s,
+                               int* launches) {
+  if (off.B < 1 || off.B > kVarlenMaxSeqs || p.max_nb < 1) return cudaErrorInvalidValue;
+  varlen_levels_kernel<<<1, 1024, 0, s>>>(off, p.max_nb, p.nbs, p.blk_base, p.level);
+  ++*launches;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t work = p.N > p.NB ? p.N : p.NB;
+  const unsigned grid = (unsigned)((work + 255) / 256 < 1184 ? (work + 255) / 256 : 1184);
+  varlen_tables_kernel<<<grid, 256, 0, s>>>(off, p.NB, p.N, p.nbs, p.blk_base, p.level, p.units,
+                                             p.blk_row0, p.row_base);
+  ++*launches;
   return cudaGetLastError();
 }
 

@@ -82,29 +82,46 @@ struct IdxArgs {
   int32_t* ids;
   float* scores;
   const float* kscale;  // FP8 only: [nb] scale of each key block
+  const int4* units;    // packed sequences: {first token, key row 0, local block, end}
+  int32_t n_ublocks;    // entries of `units`
   uint32_t* err;
 };
 
 struct Unit {
-  int32_t b;        // query block
+  int32_t b;        // query block (local to its sequence)
   int64_t tok0;     // first token of the tile
   int64_t row0;     // first q_idx row ([N*G] view)
+  int64_t key0;     // first row of the sequence's keys
+  int64_t end;      // end of the sequence (one past its last token)
   int32_t nblk;     // key blocks scored
   int32_t pairs;    // MMAs of N=256
   bool valid;
 };
 
+// Tile v: query block v / G (latest first) and its sub-tile v % G.  With
+// packed sequences the query blocks come from a table, ordered the same way
+// across sequences, and every offset is relative to the sequence's first row.
 template <bool SCORES>
 __device__ __forceinline__ Unit make_unit(const IdxArgs& a, int v) {
   Unit u;
   const int T = kRows >> a.log2G;
-  u.b = a.qb_lo + (a.n_qblocks - 1 - (v >> a.log2G));
   const int sub = v & (a.G - 1);
-  u.tok0 = (int64_t)u.b * kBlock + (int64_t)sub * T;
+  if (a.units) {
+    const int4 e = __ldg(a.units + (v >> a.log2G));
+    u.b = e.z;
+    u.tok0 = (int64_t)e.x + (int64_t)sub * T;
+    u.key0 = e.y;
+    u.end = e.w;
+  } else {
+    u.b = a.qb_lo + (a.n_qblocks - 1 - (v >> a.log2G));
+    u.tok0 = (int64_t)u.b * kBlock + (int64_t)sub * T;
+    u.key0 = 0;
+    u.end = a.N;
+  }
   u.row0 = u.tok0 * a.G;
   u.nblk = SCORES ? u.b + 1 : u.b;
   u.pairs = (u.nblk + 1) >> 1;
-  u.valid = u.tok0 < a.row_end && u.tok0 + T > a.row_begin;
+  u.valid = u.tok0 < u.end && u.tok0 < a.row_end && u.tok0 + T > a.row_begin;
   return u;
 }
 
@@ -160,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
   volatile int* abort_flag = &abort_s;
-  const int n_units = a.n_qblocks << a.log2G;
+  const int n_units = (a.units ? a.n_ublocks : a.n_qblocks) << a.log2G;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -196,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int r = 0; r < Cfg::kRegions; ++r)
             tma_load_2d(sB + stage * Cfg::kBBytes + r * kPairKeys * 128, &map_k, &bar_b_full[stage],
-                        r * Cfg::kRegionElems, p * kPairKeys);
+                        r * Cfg::kRegionElems, (int32_t)(u.key0 + p * kPairKeys));
           b_issued[stage] = true;
           b_last[stage] = sphase;
           if (++stage == S) stage = 0, sphase ^= 1;
@@ -280,13 +297,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit u = make_unit<SCORES>(a, v);
       if (!u.valid) continue;
       const int64_t t = u.tok0 + tl;
-      const bool row_out = t >= a.row_begin && t < a.row_end && t < a.N;
+      const bool row_out = t >= a.row_begin && t < a.row_end && t < u.end;
       float sc[MAXSEL > 0 ? MAXSEL : 1];
       int32_t id[MAXSEL > 0 ? MAXSEL : 1];
 #pragma unroll
       for (int i = 0; i < (MAXSEL > 0 ? MAXSEL : 1); ++i) sc[i] = -INFINITY, id[i] = -1;
       // local-block mask (scores mode only): keys s = 128*b + c with c <= lim
-      const int lim = static_cast<int>(t - (int64_t)u.b * kBlock);
+      const int lim = static_cast<int>(t - u.key0 - (int64_t)u.b * kBlock);
       float* srow = nullptr;
       if (SCORES && row_out) srow = a.scores + ((t - a.row_begin) * a.G + g) * a.nb;
 
@@ -435,8 +452,11 @@ cudaError_t launch_impl(const IndexLaunch& p, cudaStream_t s) {
   a.ids = p.ids;
   a.scores = p.scores;
   a.kscale = p.kscale;
+  a.units = p.units;
+  a.n_ublocks = p.n_units;
   a.err = p.err;
-  const int n_units = a.n_qblocks * p.G;
+  const int n_units = (p.units ? p.n_units : a.n_qblocks) * p.G;
+  if (n_units < 1) return cudaSuccess;
   const int grid = n_units < p.num_sms ? n_units : p.num_sms;
   auto kern = index_kernel<DI, MAXSEL, SCORES, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);

@@ -13,6 +13,11 @@ namespace msa {
 struct IndexLaunch {
   const void* q_idx;  // [N][G][d_idx] bf16, or e4m3 when kscale is set
   const void* k_idx;  // [N][d_idx] bf16, or e4m3 when kscale is set
+  // optional, packed sequences (selection only): one entry per (sequence, query
+  // block) {first token, first row of the sequence, local block, end of the
+  // sequence}, longest first; ids are then local to each sequence
+  const int4* units;
+  int32_t n_units;
   int64_t N;
   int32_t G, d_idx, top_k;
   int64_t row_begin, row_end;  // query rows processed: [row_begin, row_end)
@@ -31,6 +36,9 @@ struct CsrLaunch {
   int64_t row_begin, rows;
   int32_t G, top_k;
   int64_t nb;          // key blocks (lists per group)
+  // optional, packed sequences: per query row, the global number of its
+  // sequence's first key block (ids are local: list = row_base[row] + id)
+  const int32_t* row_base;
   int32_t* row_ptr;    // [G*nb+1]
   int32_t* entries;    // [rows*G*top_k]
   void* scratch;       // csr_scratch_bytes()
@@ -43,6 +51,29 @@ struct CsrLaunch {
 };
 size_t csr_scratch_bytes(int64_t rows, int32_t G, int32_t top_k, int64_t nb);
 cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches);
+
+// ---- schedule of a batch of packed sequences (csr_kernel.cu) ---------------
+// Sequence b owns packed rows cu[b] .. cu[b+1]-1 and key blocks blk_base[b] ..
+// blk_base[b+1]-1 of the global numbering (nb_b = ceil(L_b / 128) each).
+constexpr int kVarlenMaxSeqs = 1024;  // sequences whose offsets travel as a kernel parameter
+struct VarlenOffsets {
+  int32_t B;
+  int64_t cu[kVarlenMaxSeqs + 1];
+};
+struct VarlenPlan {
+  int64_t N;         // packed rows (cu[B])
+  int32_t NB;        // global key blocks
+  int32_t max_nb;    // blocks of the longest sequence
+  // workspace outputs
+  int32_t* nbs;      // [B] blocks per sequence
+  int32_t* blk_base; // [B+1]
+  int32_t* level;    // [max_nb + 1]: first unit of local block b (longest first)
+  int4* units;       // [NB] {first token, first row of the sequence, local block, end}
+  int32_t* blk_row0; // [NB] first K/V row of each global block
+  int32_t* row_base; // [N] blk_base of each row's sequence
+};
+cudaError_t launch_varlen_plan(const VarlenOffsets& off, const VarlenPlan& p, cudaStream_t s,
+                               int* launches);
 
 // ---- Main Branch (main_kernel.cu) -----------------------------------------
 struct MainLaunch {
@@ -58,6 +89,7 @@ struct MainLaunch {
   const int32_t* entries;
   const int32_t* unit_ptr;   // [G*nb+1]
   const int4* unit_desc;     // [units] {g, j, first entry, end entry}
+  const int32_t* blk_row0;   // optional, packed sequences: first K/V row of key block j
   __half* part_o;   // [rows][G][top_k][H/G][d] fp16
   float* part_lse;  // [rows][G][top_k][H/G] fp32
   uint32_t* err;

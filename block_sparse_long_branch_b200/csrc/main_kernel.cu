@@ -90,6 +90,7 @@ struct MainArgs {
   const int32_t* entries;
   const int32_t* unit_ptr;
   const int4* unit_desc;
+  const int32_t* blk_row0;  // packed sequences: first K/V row of key block j (else j*128)
   __half* part_o;
   float* part_lse;
   uint32_t* err;
@@ -97,6 +98,7 @@ struct MainArgs {
 
 struct MUnit {
   int32_t g, j, e0, e1, ntiles;
+  int32_t row0;  // first K/V row of the unit's key block
 };
 
 __device__ __forceinline__ MUnit decode_unit(const MainArgs& a, int u) {
@@ -107,6 +109,7 @@ __device__ __forceinline__ MUnit decode_unit(const MainArgs& a, int u) {
   m.e0 = d.z;
   m.e1 = d.w;
   m.ntiles = (m.e1 - m.e0 + a.TT - 1) / a.TT;
+  m.row0 = a.blk_row0 ? __ldg(a.blk_row0 + m.j) : m.j * kKeys;
   return m;
 }
 
@@ -321,15 +324,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const MUnit nx = decode_unit(a, u + gridDim.x);
 #pragma unroll
           for (int ri = 0; ri < Cfg::kRegions; ++ri) {
-            tma_prefetch_l2_3d(&map_k, ri * 64, nx.g, nx.j * kKeys);
-            tma_prefetch_l2_3d(&map_v, ri * 64, nx.g, nx.j * kKeys);
+            tma_prefetch_l2_3d(&map_k, ri * 64, nx.g, nx.row0);
+            tma_prefetch_l2_3d(&map_v, ri * 64, nx.g, nx.row0);
           }
         }
         if (!mbar_wait(&bar_k_empty, kph ^ 1, abort_flag, a.err, kDevTimeoutMma)) break;
         mbar_arrive_expect_tx(&bar_k_full, Cfg::kKVBytes);
 #pragma unroll
         for (int ri = 0; ri < Cfg::kRegions; ++ri)
-          tma_load_3d(sK + ri * kKeys * 128, &map_k, &bar_k_full, ri * 64, m.g, m.j * kKeys);
+          tma_load_3d(sK + ri * kKeys * 128, &map_k, &bar_k_full, ri * 64, m.g, m.row0);
         k_any = true;
         k_last = kph;
         kph ^= 1;
@@ -337,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bar_v_full, Cfg::kKVBytes);
 #pragma unroll
         for (int ri = 0; ri < Cfg::kRegions; ++ri)
-          tma_load_3d(sV + ri * kKeys * 128, &map_v, &bar_v_full, ri * 64, m.g, m.j * kKeys);
+          tma_load_3d(sV + ri * kKeys * 128, &map_v, &bar_v_full, ri * 64, m.g, m.row0);
         v_any = true;
         v_last = vph;
         vph ^= 1;
@@ -568,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool good = false;
       if (row_valid) good = check_entry(a, cur_ent, t, r);
       // last visible column of this half (keys s <= t on the local block)
-      const int lim = (row_valid ? (int)min64(t - (int64_t)m.j * kKeys, kKeys - 1) : kKeys - 1) -
+      const int lim = (row_valid ? (int)min64(t - (int64_t)m.row0, kKeys - 1) : kKeys - 1) -
                       hc * 64;
       const bool unmasked = __all_sync(0xffffffffu, lim >= 63);
 
@@ -722,6 +725,7 @@ cudaError_t launch_main_impl(const MainLaunch& p, cudaStream_t s) {
   a.entries = p.entries;
   a.unit_ptr = p.unit_ptr;
   a.unit_desc = p.unit_desc;
+  a.blk_row0 = p.blk_row0;
   a.part_o = p.part_o;
   a.part_lse = p.part_lse;
   a.err = p.err;

@@ -255,8 +255,11 @@ MSA_API msa_status_t msa_prefill_block_alignment(const msa_config_t* cfg, const 
  * Prefill of B independent sequences packed along the token axis (no
  * attention across sequences); each is the causal prefill msa_prefill
  * computes.  The pages serve MSA to batched requests but describe no batched
- * kernel; this entry point runs the same kernels once per sequence, in
- * order, on `stream` and `ws`.
+ * kernel.  When the workspace holds the whole batch (at least
+ * msa_prefill_varlen_workspace_size()) and B <= 1024, the batch runs in one
+ * pass: every kernel runs once, over tiles of all sequences, with key blocks
+ * numbered across the batch.  Otherwise the sequences run one after another,
+ * each as msa_prefill, on `stream` and `ws`.
  *   q [T][H][d], k/v [T][G][d], q_idx [T][G][d_idx], k_idx [T][d_idx] bf16,
  *     T = cu_seqlens[B]; sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1
  *     and its token i is position i of that sequence.
@@ -265,10 +268,14 @@ MSA_API msa_status_t msa_prefill_block_alignment(const msa_config_t* cfg, const 
  *   out [T][H][d] bf16 out; ids_out [T][G][k] int32 out, nullable (ids are
  *     block numbers within the token's own sequence; every sequence's rows
  *     must start 16-byte aligned, else MSA_ERR_UNSUPPORTED).
- *   ws: at least msa_prefill_min_workspace() for the longest sequence; every
- *     sequence then runs in query chunks that fit, as in msa_prefill.
+ *   ws: at least msa_prefill_min_workspace() for the longest sequence; with
+ *     less than msa_prefill_varlen_workspace_size() every sequence runs in
+ *     query chunks that fit, as in msa_prefill.
  * Phase events (msa_set_phase_events) are not recorded by this call.
  */
+MSA_API msa_status_t msa_prefill_varlen_workspace_size(const msa_config_t* cfg,
+                                                       const int64_t* cu_seqlens, int32_t B,
+                                                       size_t* bytes);
 MSA_API msa_status_t msa_prefill_varlen(const msa_config_t* cfg, const void* q, const void* k,
                                         const void* v, const void* q_idx, const void* k_idx,
                                         const int64_t* cu_seqlens, int32_t B, void* out,

@@ -5,10 +5,23 @@ import numpy as np
 
 # Acceptance bars: selected ids bit-exact except near-ties within 1e-3 (raw
 # dot-product units) of the boundary score; bf16 outputs within 1e-2 max-abs
-# and 2e-3 mean-abs of the fp64 oracle.
+# and 2e-3 mean-abs of the fp64 oracle.  An output of magnitude 4 or more is
+# beyond that bound by its own bf16 rounding (half a spacing there is 2^-6 >
+# 1e-2, even for the correctly rounded exact value): such an output may be off
+# by its bf16 half-spacing plus the arithmetic budget the bound leaves at
+# magnitudes 2 to 4 (1e-2 - 2^-7).
 NEAR_TIE = 1e-3
 OUT_MAX_ABS = 1e-2
 OUT_MEAN_ABS = 2e-3
+
+
+def bf16_half_spacing(x):
+    """Half the distance between neighbouring bf16 values at |x| (normal range)."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
+    return 2.0 ** (e - 8)
+
+
+OUT_ARITH = OUT_MAX_ABS - 2.0 ** -7
 
 
 def check_id_rows_valid(ids: np.ndarray, rows: np.ndarray, block: int, top_k: int):
@@ -49,6 +62,9 @@ def check_output(gpu_out: np.ndarray, ref_out: np.ndarray, max_abs: float = OUT_
                  mean_abs: float = OUT_MEAN_ABS):
     err = np.abs(gpu_out.astype(np.float64) - ref_out)
     assert np.isfinite(gpu_out).all()
-    assert err.max() <= max_abs, f"max abs err {err.max():.3g}"
+    bound = np.maximum(max_abs, bf16_half_spacing(ref_out) + OUT_ARITH)
+    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    assert (err <= bound).all(), (f"max abs err {err.max():.3g}; worst over its bound: "
+                                  f"{err[worst]:.3g} at |ref| {abs(ref_out[worst]):.3g}")
     assert err.mean() <= mean_abs, f"mean abs err {err.mean():.3g}"
     return float(err.max()), float(err.mean())

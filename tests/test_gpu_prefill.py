@@ -292,19 +292,8 @@ def test_prefill_1m_sampled_rows_chunked(msa):
     assert n_ties <= 64
 
 
-def test_prefill_varlen_matches_per_sequence_oracle(msa):
-    """Packed sequences of mixed lengths (one empty, one of a single token):
-    each must equal its own causal prefill, ids counted within the sequence."""
-    lens = [700, 0, 4096 + 5, 128, 1, 2049]
+def _check_varlen(msa, s, inp, lens, out, ids):
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
-    s = synth.PrefillShape("varlen", N=int(cu[-1]), H=16, G=2, d=128, d_idx=64, top_k=8,
-                           n_needles=6, seed=41)
-    inp = synth.make_prefill_inputs(s, device="cuda")
-    cfg = _cfg(msa, s)
-    out, ids = msa.msa_prefill_varlen(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"],
-                                      inp["k_idx"], cu, ids_out=True)
-    torch.cuda.synchronize()
-    assert msa.msa_last_launch_count() > 0
     for b, L in enumerate(lens):
         if L == 0:
             continue
@@ -322,6 +311,45 @@ def test_prefill_varlen_matches_per_sequence_oracle(msa):
                                              inp["k"][s0:s1], inp["v"][s0:s1], g_ids, s.scale,
                                              s.block)
         parity.check_output(out[s0:s1].float().cpu().numpy(), ref_out)
+
+
+def test_prefill_varlen_matches_per_sequence_oracle(msa):
+    """Packed sequences of mixed lengths (one empty, one of a single token), run
+    as one batch: each must equal its own causal prefill, ids counted within
+    the sequence."""
+    lens = [700, 0, 4096 + 5, 128, 1, 2049]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    s = synth.PrefillShape("varlen", N=int(cu[-1]), H=16, G=2, d=128, d_idx=64, top_k=8,
+                           n_needles=6, seed=41)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    out, ids = msa.msa_prefill_varlen(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"],
+                                      inp["k_idx"], cu, ids_out=True)
+    torch.cuda.synchronize()
+    # one pass over the batch: the plan, the five prefill stages, not six sequences
+    assert 0 < msa.msa_last_launch_count() < 20
+    _check_varlen(msa, s, inp, lens, out, ids)
+
+
+def test_prefill_varlen_many_short_sequences(msa):
+    """96 sequences of 1 to 600 tokens (most end in a partial block, followed
+    directly by the next sequence's rows) with the benchmark's head layout."""
+    rng = np.random.default_rng(43)
+    lens = [int(x) for x in rng.integers(1, 601, 96)]
+    lens[5] = 128
+    lens[6] = 256
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    s = synth.PrefillShape("varlen_many", N=int(cu[-1]), H=64, G=8, d=128, d_idx=128,
+                           top_k=16, n_needles=0, seed=44)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    ws = torch.empty(msa.msa_prefill_varlen_workspace_size(cfg, cu), dtype=torch.uint8,
+                     device="cuda")
+    out, ids = msa.msa_prefill_varlen(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"],
+                                      inp["k_idx"], cu, ids_out=True, workspace=ws)
+    assert msa.msa_get_device_error(ws) == 0
+    assert msa.msa_last_launch_count() < 20
+    _check_varlen(msa, s, inp, lens, out, ids)
 
 
 def test_prefill_varlen_small_workspace_chunks_each_sequence(msa):
