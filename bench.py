@@ -652,6 +652,62 @@ def _e2e_decode(args, msa, dec, dcfg, dws, dev, world):
             "ms_per_step": dms}
 
 
+def run_varlen(args, rank, world, local):
+    """A packed batch of equal-length sequences: the one-pass varlen prefill
+    against one msa_prefill per sequence, both timed with CUDA events."""
+    import block_sparse_long_branch_b200 as msa
+    B, L = (int(x) for x in args.varlen.lower().split("x"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    msa.load_library()
+    cu = np.arange(B + 1, dtype=np.int64) * L
+    shape = synth.PrefillShape(f"varlen_{B}x{L}", N=B * L, H=64, G=8, d=128, d_idx=128,
+                               top_k=16, seed=synth.SEED_BASE + 40)
+    inp = synth.make_prefill_inputs(shape, device=dev, seed=shape.seed + rank)
+    cfg = msa.config(shape.H, shape.G, shape.d, shape.d_idx, top_k=shape.top_k,
+                     scale=shape.scale)
+    ws = torch.empty(msa.msa_prefill_varlen_workspace_size(cfg, cu), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((shape.N, shape.H, shape.d), dtype=torch.bfloat16, device=dev)
+    ref = torch.empty_like(out)
+
+    def one_pass():
+        msa.msa_prefill_varlen(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], cu,
+                               out=out, workspace=ws)
+
+    def per_sequence():
+        for b in range(B):
+            r = slice(b * L, (b + 1) * L)
+            msa.msa_prefill(cfg, inp["q"][r], inp["k"][r], inp["v"][r], inp["q_idx"][r],
+                            inp["k_idx"][r], out=ref[r], workspace=ws)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        return reduce_max(e0.elapsed_time(e1), world) / args.steps
+
+    ms_one = timed(one_pass)
+    ms_seq = timed(per_sequence)
+    assert torch.equal(out, ref), "one pass and per-sequence prefill differ"
+    value, _ = replica_rate(shape.N, ms_one, world)
+    return {"metric": "MSA varlen prefill tokens/s (one pass over the packed batch)",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_one, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": shape.name, "B": B, "L": L, "H": shape.H, "G": shape.G,
+                       "d": shape.d, "d_idx": shape.d_idx, "top_k": shape.top_k},
+            "per_sequence_ms": ms_seq, "speedup_vs_per_sequence": ms_seq / ms_one}
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -674,6 +730,10 @@ def parse_args(argv=None):
                     help="cap on the prefill workspace; above it the query axis is chunked")
     ap.add_argument("--ref-rows", type=int, default=32,
                     help="query rows per step in the reference arm")
+    ap.add_argument("--varlen", metavar="BxL",
+                    help="time only a packed batch of B sequences of L tokens (64 heads, 8 "
+                         "groups, d 128): one msa_prefill_varlen pass vs one msa_prefill "
+                         "per sequence")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
@@ -688,6 +748,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             line = run_reference(args, rank, world)
+        elif args.varlen:
+            line = run_varlen(args, rank, world, local)
         else:
             line = run_ours(args, rank, world, local)
         if rank == 0 and line is not None:
