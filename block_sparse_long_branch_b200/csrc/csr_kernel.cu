@@ -15,6 +15,12 @@
 //                a shared-memory running count carries the rank across batches
 //   5. units   : per list, number of Main Branch work units; exclusive prefix
 // HBM-bound integer work: each id is read twice, each entry written once.
+//
+// For a batch of packed sequences the ids are local to each sequence; the key
+// is row_base[row] + id, a global block number.  The plan kernels at the end
+// of the anonymous namespace build row_base and the other tables of that
+// schedule (the Index Branch's tiles, each block's first K/V row) on the
+// device.
 #include "kernels.h"
 #include "sm100.cuh"
 
