@@ -10,9 +10,10 @@
 //   2. scan    : exclusive prefix over that table (flattened g, j, tile), so
 //                the entry gives where tile `tile`'s hits on (g, j) start
 //   3. row_ptr : row_ptr[g*nb+j] = scanned[(g*nb+j)*ntiles]
-//   4. scatter : one warp per (tile, group) walks its hits in (t, slot) order;
-//                equal keys inside a 32-hit batch are ranked with match.any,
-//                a shared-memory running count carries the rank across batches
+//   4. scatter : one warp per (tile, group) loads its start offsets into
+//                shared memory, then walks its hits in (t, slot) order; equal
+//                keys inside a 32-hit batch are ranked with match.any, and the
+//                shared-memory offset of a key advances by its batch count
 //   5. units   : per list, number of Main Branch work units; exclusive prefix
 // HBM-bound integer work: each id is read twice, each entry written once.
 //
@@ -172,7 +173,10 @@ __global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restri
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int64_t s0 = 0; s0 < nb; s0 += kBinSlice) {
     const int width = (int)min64(kBinSlice, nb - s0);
-    for (int i = lane; i < width; i += 32) run[i] = 0;
+    // where this tile's hits on each key of the slice start (independent
+    // loads here keep them off the per-batch chain below)
+    for (int i = lane; i < width; i += 32)
+      run[i] = __ldg(scanned + ((int64_t)g * nb + s0 + i) * ntiles + tile);
     __syncwarp();
     for (int64_t e0 = 0; e0 < n_el; e0 += 32) {
       const int64_t e = e0 + lane;
@@ -191,8 +195,7 @@ __global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restri
       if (mine) {
         base = run[key];
         const int rank = __popc(peers & lt_mask);
-        const int64_t pos = (int64_t)scanned[((int64_t)g * nb + j) * ntiles + tile] + base + rank;
-        entries[pos] = (int32_t)(((row_begin + row) << 5) | r);
+        entries[(int64_t)base + rank] = (int32_t)(((row_begin + row) << 5) | r);
       }
       __syncwarp();
       if (mine && (peers & lt_mask) == 0) run[key] = base + __popc(peers);
