@@ -352,6 +352,33 @@ def test_prefill_varlen_many_short_sequences(msa):
     _check_varlen(msa, s, inp, lens, out, ids)
 
 
+@pytest.mark.parametrize("B", [1024, 1100])
+def test_prefill_varlen_batch_size_limit(msa, B):
+    """1024 sequences is the largest batch the one-pass plan takes (its offsets
+    travel as a kernel parameter); 1100 run one after another.  Both match the
+    oracle on a spread of sequences."""
+    rng = np.random.default_rng(B)
+    lens = [int(x) for x in rng.integers(1, 5, B)]
+    lens[B // 2] = 300
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    s = synth.PrefillShape("varlen_b", N=int(cu[-1]), H=8, G=2, d=64, d_idx=64, top_k=4,
+                           seed=45)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = _cfg(msa, s)
+    out, ids = msa.msa_prefill_varlen(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"],
+                                      inp["k_idx"], cu, ids_out=True)
+    torch.cuda.synchronize()
+    one_pass = msa.msa_last_launch_count() < 20
+    assert one_pass == (B <= 1024)
+    pick = sorted({0, 1, B // 2, B - 1} | set(int(x) for x in rng.integers(0, B, 8)))
+    sub = [lens[b] for b in pick]
+    rows = np.concatenate([np.arange(cu[b], cu[b + 1]) for b in pick])
+    sub_inp = {n: inp[n][torch.from_numpy(rows).cuda()] for n in ("q", "k", "v", "q_idx",
+                                                                    "k_idx")}
+    _check_varlen(msa, s, sub_inp, sub, out[torch.from_numpy(rows).cuda()],
+                  ids[torch.from_numpy(rows).cuda()])
+
+
 def test_prefill_varlen_small_workspace_chunks_each_sequence(msa):
     """With the minimum workspace every sequence runs in query chunks; the
     result equals the one-shot call bit for bit."""
