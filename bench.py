@@ -145,6 +145,12 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
+        return self.parse_samples(out)
+
+    @staticmethod
+    def parse_samples(out: str) -> dict:
+        """Median SM clock of the loaded samples (above half the highest seen), the
+        maximum clock, and every throttle reason seen active in any sample."""
         sm, mx, reasons = [], [], set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for line in out.strip().splitlines():
