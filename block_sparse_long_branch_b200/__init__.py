@@ -384,7 +384,11 @@ def msa_prefill_varlen(cfg: MsaConfig, q, k, v, q_idx, k_idx, cu_seqlens,
                        out: Optional[torch.Tensor] = None, ids_out=None,
                        workspace: Optional[torch.Tensor] = None, stream=None):
     """Prefill of sequences packed along the token axis (host ``cu_seqlens``,
-    any int sequence of B+1 offsets).  Returns ``out`` or ``(out, ids)``."""
+    any int sequence of B+1 offsets).  Returns ``out`` or ``(out, ids)``.
+
+    Without ``workspace`` one is allocated: the one-pass size when it takes at
+    most half of the device's free memory, else the size for the longest
+    sequence (the sequences then run one after another)."""
     lib = load_library()
     import numpy as _np
     cu = _np.ascontiguousarray(_np.asarray(
@@ -399,7 +403,13 @@ def msa_prefill_varlen(cfg: MsaConfig, q, k, v, q_idx, k_idx, cu_seqlens,
         out = torch.empty((T, H, d), dtype=torch.bfloat16, device=q.device)
     if ids_out is True:
         ids_out = torch.empty((T, G, kk), dtype=torch.int32, device=q.device)
-    ws = _workspace(workspace, msa_prefill_varlen_workspace_size(cfg, cu), q.device)
+    need = msa_prefill_varlen_workspace_size(cfg, cu)
+    if workspace is None:
+        # one pass over the batch if it fits comfortably, else one sequence at a time
+        free, _ = torch.cuda.mem_get_info(q.device)
+        if need > free // 2:
+            need = msa_workspace_size(cfg, OP_PREFILL, max(int(_np.max(_np.diff(cu))), 1))
+    ws = _workspace(workspace, need, q.device)
     ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (T, G, kk))
     st = lib.msa_prefill_varlen(ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (T, H, d)),
                                 _dev(k, torch.bfloat16, "k", (T, G, d)),
