@@ -11,12 +11,17 @@
 //      contiguous bytes of a key row straight from global memory.
 //      Writes the pooled (max) score of every non-local block, [G][nb] per
 //      sequence so that each group's scores are contiguous.
-//   2. decode_topk_kernel  : per (sequence, group), the best k-1 non-local
-//      blocks under (score desc, id asc), plus the local block, ascending.
-//   3. decode_attn_kernel  : per (sequence, group, slot), softmax of the
-//      group's heads over the slot's block (causal on the local block), the
-//      partial (o, lse) in the same layout as the prefill partials.
-//   4. the prefill merge kernel combines the slots.
+//   2. decode_attend_kernel : n_split CTAs per (sequence, group).  Each one
+//      selects, exactly and identically to its siblings, the best k-1
+//      non-local blocks under (score desc, id asc) plus the local block (a
+//      threshold from per-warp bests, then an exact ranking of the candidates
+//      by counting; sorted per-thread lists and warp tournaments when the
+//      scores cluster), then attends over its share of them (selected blocks
+//      z, z + n_split, ...) with an online softmax: S^T = K Q^T on mma.sync
+//      with K rows loaded one block ahead, P carried as two bf16 parts (hi and
+//      lo) into O^T += V^T P^T with V double-buffered by cp.async.  Split CTAs
+//      leave (o, m, l) partials; the last to finish (a ticket per (sequence,
+//      group)) merges them and writes the output.
 #include "kernels.h"
 #include "sm100.cuh"
 
