@@ -179,3 +179,10 @@ def test_decode_heads_per_group_limit():
                           None) == 2
     cfg16 = msa.config(32, 2, 128, 128, top_k=4)  # 16 heads per group: supported
     assert lib.msa_workspace_size(ctypes.byref(cfg16), msa.OP_DECODE, 1024, 2, ctypes.byref(n)) == 0
+
+
+def test_binding_offers_every_declared_function():
+    """The Python layer has a function of the same name for every C entry point."""
+    missing = [name for name in _declared() if not callable(getattr(msa, name, None))]
+    assert not missing, missing
+    assert set(_declared()) <= set(msa.__all__) | {"msa_last_launch_count"}
