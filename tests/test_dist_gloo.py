@@ -209,3 +209,31 @@ def test_sequence_range_balances_cached_length():
     # one sequence: its middle lies in rank 1's half, rank 0 has none
     assert shard.sequence_range([0, 4000], 0, 2) == (0, 0)
     assert shard.sequence_range([0, 4000], 1, 2) == (0, 1)
+
+
+@pytest.mark.parametrize("world", [1, 3, 4, 6])
+def test_decode_shards_cover_the_batch_exactly(world):
+    """Every rank's slice, concatenated in rank order, gives back the batch; each
+    slice's offsets start at 0 and keep the sequence lengths."""
+    import torch
+    from block_sparse_long_branch_b200 import shard
+    lens = [5, 1, 300, 2, 40, 7]
+    cu = [0]
+    for L in lens:
+        cu.append(cu[-1] + L)
+    B, T = len(lens), cu[-1]
+    q = torch.arange(B * 3, dtype=torch.float32).reshape(B, 3)
+    qi = q + 1000
+    kc = torch.arange(T * 2, dtype=torch.float32).reshape(T, 2)
+    parts = [shard.shard_decode_inputs(q, qi, kc, kc + 1, kc + 2, cu, r, world)
+             for r in range(world)]
+    assert torch.equal(torch.cat([p[0] for p in parts]), q)
+    assert torch.equal(torch.cat([p[1] for p in parts]), qi)
+    assert torch.equal(torch.cat([p[2] for p in parts]), kc)
+    assert torch.equal(torch.cat([p[4] for p in parts]), kc + 2)
+    got_lens = []
+    for p in parts:
+        c = p[5].tolist()
+        assert c[0] == 0 and len(c) == p[0].shape[0] + 1 and c[-1] == p[2].shape[0]
+        got_lens += [b - a for a, b in zip(c, c[1:])]
+    assert got_lens == lens
