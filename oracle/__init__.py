@@ -153,6 +153,59 @@ def block_query_lists(ids: np.ndarray, nb: int):
     return row_ptr, entries[:total].copy()
 
 
+def block_alignment(pooled: np.ndarray, ids: np.ndarray, lse: np.ndarray):
+    """Index-vs-Main alignment of the selected blocks of every (query, group).
+
+    ai-tool-zukan MiniMax MSA guide, section "非微分的な選択をどう学習させるか
+    （KLダイバージェンス）" (subsection "選択を学習可能にするKL損失"): the Index
+    Branch's distribution of scores over the blocks is brought close, by a KL
+    divergence, to the distribution of which blocks really mattered to the Main
+    Branch's exact attention.  The pages give no formulas; the reading used:
+      index side  q_r = softmax over the filled slots of the pooled raw-dot
+                  scores (temperature 1);
+      main side   p_r = mean over the group's heads of exp(lse[h, r] - L_h),
+                  the share of head h's exact softmax on slot r's keys
+                  (L_h = logsumexp_r lse[h, r]);
+      KL(p || q) = sum_r p_r (ln p_r - ln q_r), in nats, terms with p_r = 0
+                  contributing 0.
+    pooled [n,G,nb] (as from pooled_scores), ids [n,G,k] (-1 = empty slot),
+    lse [n,H,k] (as from block_attention with partials) ->
+    (score [n,G,k] with -inf in empty slots, mass [n,G,k] with 0 there, kl [n,G]).
+    """
+    pooled = np.asarray(pooled, dtype=np.float64)
+    ids = np.asarray(ids)
+    lse = np.asarray(lse, dtype=np.float64)
+    n, G, k = ids.shape
+    H = lse.shape[1]
+    assert lse.shape == (n, H, k) and H % G == 0
+    HG = H // G
+    filled = ids >= 0
+    score = np.full((n, G, k), -np.inf)
+    mass = np.zeros((n, G, k))
+    kl = np.zeros((n, G))
+    for t in range(n):
+        for g in range(G):
+            f = filled[t, g]
+            if not f.any():
+                continue
+            sc = pooled[t, g, ids[t, g, f]]
+            score[t, g, f] = sc
+            # index side: softmax of the scores over the filled slots
+            lq = sc - sc.max()
+            lq = lq - np.log(np.exp(lq).sum())
+            # main side: each head's softmax mass per slot, averaged over heads
+            p = np.zeros(int(f.sum()))
+            for h in range(g * HG, (g + 1) * HG):
+                lh = lse[t, h, f]
+                w = np.exp(lh - lh.max())
+                p += w / w.sum()
+            p /= HG
+            mass[t, g, f] = p
+            pos = p > 0
+            kl[t, g] = float(np.sum(p[pos] * (np.log(p[pos]) - lq[pos])))
+    return score, mass, kl
+
+
 # ---------------------------------------------------------------------------
 # Whole-path helpers (composition of the steps above, nothing more).
 # ---------------------------------------------------------------------------

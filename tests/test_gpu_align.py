@@ -1,8 +1,8 @@
 """GPU parity: the block-alignment outputs of msa_prefill_block_alignment.
 
 The expected values come from the oracle only: its pooled index scores of
-every visible block, and its per-slot partial softmax (lse) of the Main
-Branch on the same selection, combined as the header describes (head-mean
+every visible block and its per-slot partial softmax (lse) of the Main Branch
+on the same selection, combined by oracle.block_alignment (head-mean
 attention mass per slot; KL of that mass from the softmax of the slots'
 scores).
 """
@@ -26,26 +26,12 @@ def msa(cuda_device):
 
 def _expected(inp, s, ids):
     """Oracle block scores, head-mean block mass and KL for the given selection."""
-    N = s.N
-    rows = np.arange(N)
+    rows = np.arange(s.N)
     pooled = oracle.pooled_scores(oracle.as_bf16_bits(inp["q_idx"]), rows, inp["k_idx"], s.block,
                                   s.nb)
     _, lse, _ = oracle.block_attention(oracle.as_bf16_bits(inp["q"]), rows, inp["k"], inp["v"],
                                        ids, s.scale, s.block, partials=True)
-    HG = s.H // s.G
-    filled = ids >= 0
-    score = np.where(filled, np.take_along_axis(pooled, np.maximum(ids, 0), axis=2), -np.inf)
-    lse = lse.reshape(N, s.G, HG, s.top_k)
-    lse = np.where(filled[:, :, None, :], lse, -np.inf)
-    w = np.exp(lse - np.max(lse, axis=3, keepdims=True))
-    w /= w.sum(axis=3, keepdims=True)
-    mass = w.mean(axis=2)
-    sc = np.where(filled, score, -np.inf)
-    logq = sc - np.max(sc, axis=2, keepdims=True)
-    logq -= np.log(np.exp(logq).sum(axis=2, keepdims=True))
-    with np.errstate(divide="ignore", invalid="ignore"):
-        terms = np.where(filled & (mass > 0), mass * (np.log(mass) - logq), 0.0)
-    return score, mass, terms.sum(axis=2)
+    return oracle.block_alignment(pooled, ids, lse)
 
 
 @pytest.mark.parametrize("d_idx", [128, 64])
