@@ -10,11 +10,13 @@
 //   2. scan    : exclusive prefix over that table (flattened g, j, tile), so
 //                the entry gives where tile `tile`'s hits on (g, j) start
 //   3. row_ptr : row_ptr[g*nb+j] = scanned[(g*nb+j)*ntiles]
-//   4. scatter : one warp per (tile, group) loads its start offsets into
-//                shared memory, then walks its hits in (t, slot) order; equal
-//                keys inside a 32-hit batch are ranked with match.any, and the
-//                shared-memory offset of a key advances by its batch count
-//   5. units   : per list, number of Main Branch work units; exclusive prefix
+//   4. scatter : one warp per (tile, group) copies its tile's keys and its
+//                start offsets into shared memory, then walks its hits in
+//                (t, slot) order; equal keys inside a 32-hit batch are ranked
+//                with match.any, and the shared-memory offset of a key
+//                advances by its batch count
+//   5. units   : one CTA: per list, the number of Main Branch work units, their
+//                exclusive prefix and the unit table
 // HBM-bound integer work: each id is read twice, each entry written once.
 //
 // For a batch of packed sequences the ids are local to each sequence; the key
@@ -119,12 +121,6 @@ __global__ void add_offsets_kernel(int32_t* __restrict__ data, int64_t n,
   if (i < n) data[i] += offs[i / kScanChunk];
 }
 
-// total = last exclusive value + last count (read before the scan)
-__global__ void store_total_kernel(const int32_t* scanned, const int32_t* last_count, int64_t n,
-                                   int32_t* total) {
-  *total = scanned[n - 1] + *last_count;
-}
-
 size_t scan_scratch_elems(int64_t n) {
   size_t s = 0;
   while (n > kScanChunk) {
@@ -149,45 +145,48 @@ cudaError_t exclusive_scan(int32_t* data, int64_t n, int32_t* tmp, cudaStream_t 
   return cudaGetLastError();
 }
 
+// row_ptr[x] = scanned[x * ntiles]; the end, row_ptr[n_lists], is the last
+// exclusive value plus the last count (saved before the in-place scan)
 __global__ void csr_rowptr_kernel(const int32_t* __restrict__ scanned, int64_t n_lists,
-                                  int32_t ntiles, const int32_t* __restrict__ total,
+                                  int32_t ntiles, const int32_t* __restrict__ last_count,
                                   int32_t* __restrict__ row_ptr) {
   const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (x < n_lists) row_ptr[x] = scanned[x * ntiles];
-  if (x == n_lists) row_ptr[x] = *total;
+  if (x == n_lists) row_ptr[x] = scanned[n_lists * ntiles - 1] + *last_count;
 }
 
+// One warp per (tile, group).  The tile's list keys are first copied to
+// shared memory with independent, coalesced loads, so the ranking loop below
+// only waits on shared memory.
 __global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restrict__ ids,
                                                          int64_t row_begin, int64_t rows,
                                                          int32_t G, int32_t top_k, int64_t nb,
-                                                         int32_t ntiles,
+                                                         int32_t ntiles, int32_t bins,
                                                          const int32_t* __restrict__ scanned,
                                                          const int32_t* __restrict__ row_base,
                                                          int32_t* __restrict__ entries) {
-  extern __shared__ int32_t run[];
+  extern __shared__ int32_t sm[];
+  int32_t* run = sm;          // [bins]: next free entry of each key of the slice
+  int32_t* keys = sm + bins;  // [kTileTok * top_k]: the tile's keys of group g
   const int tile = blockIdx.x, g = blockIdx.y;
   const int lane = threadIdx.x;
   const int64_t r0 = (int64_t)tile * kTileTok;
   const int64_t r1 = min(rows, r0 + kTileTok);
-  const int64_t n_el = (r1 - r0) * top_k;
+  const int n_el = (int)((r1 - r0) * top_k);
+  for (int e = lane; e < n_el; e += 32) {
+    const int64_t row = r0 + e / top_k;
+    keys[e] = list_key(row_base, row, __ldg(ids + (row * G + g) * top_k + e % top_k));
+  }
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int64_t s0 = 0; s0 < nb; s0 += kBinSlice) {
     const int width = (int)min64(kBinSlice, nb - s0);
-    // where this tile's hits on each key of the slice start (independent
-    // loads here keep them off the per-batch chain below)
+    // where this tile's hits on each key of the slice start
     for (int i = lane; i < width; i += 32)
       run[i] = __ldg(scanned + ((int64_t)g * nb + s0 + i) * ntiles + tile);
     __syncwarp();
-    for (int64_t e0 = 0; e0 < n_el; e0 += 32) {
-      const int64_t e = e0 + lane;
-      int32_t j = -1;
-      int64_t row = 0;
-      int r = 0;
-      if (e < n_el) {
-        row = r0 + e / top_k;
-        r = (int)(e % top_k);
-        j = list_key(row_base, row, ids[(row * G + g) * top_k + r]);
-      }
+    for (int e0 = 0; e0 < n_el; e0 += 32) {
+      const int e = e0 + lane;
+      const int32_t j = e < n_el ? keys[e] : -1;
       const bool mine = j >= s0 && j < s0 + width;
       const int key = mine ? (int)(j - s0) : -1;
       const unsigned peers = __match_any_sync(0xffffffffu, key);
@@ -195,7 +194,8 @@ __global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restri
       if (mine) {
         base = run[key];
         const int rank = __popc(peers & lt_mask);
-        entries[(int64_t)base + rank] = (int32_t)(((row_begin + row) << 5) | r);
+        const int64_t row = r0 + e / top_k;
+        entries[(int64_t)base + rank] = (int32_t)(((row_begin + row) << 5) | (e % top_k));
       }
       __syncwarp();
       if (mine && (peers & lt_mask) == 0) run[key] = base + __popc(peers);
@@ -205,26 +205,38 @@ __global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restri
 }
 
 // Work units of the Main Branch: list x = g*nb + j is cut into runs of at
-// most `per_unit` entries; unit u gets {g, j, first entry, end entry}.
-__global__ void unit_fill_kernel(const int32_t* __restrict__ unit_ptr,
-                                 const int32_t* __restrict__ row_ptr, int64_t n_lists, int64_t nb,
-                                 int32_t per_unit, int4* __restrict__ unit_desc) {
-  const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (x >= n_lists) return;
-  const int32_t beg = row_ptr[x], end = row_ptr[x + 1];
-  const int g = (int)(x / nb), j = (int)(x - (int64_t)g * nb);
-  int32_t e0 = beg;
-  for (int32_t u = unit_ptr[x]; u < unit_ptr[x + 1]; ++u, e0 += per_unit)
-    unit_desc[u] = make_int4(g, j, e0, min(end, e0 + per_unit));
-}
-
-__global__ void unit_count_kernel(const int32_t* __restrict__ row_ptr, int64_t n_lists,
-                                  int32_t per_unit, int32_t* __restrict__ units) {
-  const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (x < n_lists) {
-    const int32_t len = row_ptr[x + 1] - row_ptr[x];
-    units[x] = (len + per_unit - 1) / per_unit;
+// most `per_unit` entries; unit_ptr[x] is the exclusive prefix of the unit
+// counts (unit_ptr[n_lists] the total) and unit u gets {g, j, first entry,
+// end entry}.  One CTA: each thread counts a contiguous range of lists, the
+// CTA scans the per-thread sums, and each thread fills its range.
+constexpr int kUnitThreads = 1024;
+__global__ void __launch_bounds__(kUnitThreads)
+    units_kernel(const int32_t* __restrict__ row_ptr, int64_t n_lists, int64_t nb,
+                 int32_t per_unit, int32_t* __restrict__ unit_ptr, int4* __restrict__ unit_desc) {
+  __shared__ int32_t warp_tot[32];
+  const int64_t per = (n_lists + kUnitThreads - 1) / kUnitThreads;
+  const int64_t x0 = min64((int64_t)threadIdx.x * per, n_lists);
+  const int64_t x1 = min64(x0 + per, n_lists);
+  int32_t mine = 0;
+  for (int64_t x = x0; x < x1; ++x) mine += (row_ptr[x + 1] - row_ptr[x] + per_unit - 1) / per_unit;
+  const int32_t incl = warp_incl_scan(mine);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int32_t t = warp_tot[l];
+    warp_tot[l] = warp_incl_scan(t) - t;
   }
+  __syncthreads();
+  int32_t u = warp_tot[w] + incl - mine;
+  for (int64_t x = x0; x < x1; ++x) {
+    unit_ptr[x] = u;
+    const int32_t beg = row_ptr[x], end = row_ptr[x + 1];
+    const int g = (int)(x / nb), j = (int)(x - (int64_t)g * nb);
+    for (int32_t e0 = beg; e0 < end; e0 += per_unit, ++u)
+      unit_desc[u] = make_int4(g, j, e0, min(end, e0 + per_unit));
+  }
+  if (threadIdx.x == kUnitThreads - 1) unit_ptr[n_lists] = u;
 }
 
 // ---- schedule of a batch of packed sequences --------------------------------
@@ -332,46 +344,39 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
   const int64_t table = n_lists * ntiles;
   int32_t* cnt = static_cast<int32_t*>(p.scratch);
   int32_t* scan_tmp = cnt + table;
-  int32_t* total = scan_tmp + scan_scratch_elems(table);
-  int32_t* last = total + 1;
-  int32_t* tmp2 = last + 1;
+  int32_t* last = scan_tmp + scan_scratch_elems(table) + 1;  // the table's last count
   const int bins = (int)(p.nb < kBinSlice ? p.nb : kBinSlice);
   cudaError_t e;
 
   dim3 grid((unsigned)ntiles, (unsigned)p.G);
   const size_t bin_bytes = (size_t)bins * sizeof(int32_t);
-  if (bin_bytes > 48 * 1024) {
-    if ((e = cudaFuncSetAttribute(csr_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)bin_bytes)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(csr_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)bin_bytes)) != cudaSuccess)
-      return e;
-  }
-  csr_hist_kernel<<<grid, 256, bins * sizeof(int32_t), s>>>(p.ids, p.rows, p.G, p.top_k, p.nb,
-                                                           (int32_t)ntiles, cnt, p.row_base, p.err);
+  const size_t scatter_bytes = bin_bytes + (size_t)kTileTok * p.top_k * sizeof(int32_t);
+  if (bin_bytes > 48 * 1024 &&
+      (e = cudaFuncSetAttribute(csr_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)bin_bytes)) != cudaSuccess)
+    return e;
+  if (scatter_bytes > 48 * 1024 &&
+      (e = cudaFuncSetAttribute(csr_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)scatter_bytes)) != cudaSuccess)
+    return e;
+  csr_hist_kernel<<<grid, 256, bin_bytes, s>>>(p.ids, p.rows, p.G, p.top_k, p.nb,
+                                               (int32_t)ntiles, cnt, p.row_base, p.err);
   ++*launches;
   if ((e = cudaMemcpyAsync(last, cnt + table - 1, sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) !=
       cudaSuccess)
     return e;
   if ((e = exclusive_scan(cnt, table, scan_tmp, s, launches)) != cudaSuccess) return e;
-  store_total_kernel<<<1, 1, 0, s>>>(cnt, last, table, total);
-  ++*launches;
   csr_rowptr_kernel<<<(unsigned)((n_lists + 1 + 255) / 256), 256, 0, s>>>(
-      cnt, n_lists, (int32_t)ntiles, total, p.row_ptr);
+      cnt, n_lists, (int32_t)ntiles, last, p.row_ptr);
   ++*launches;
-  csr_scatter_kernel<<<grid, 32, bins * sizeof(int32_t), s>>>(p.ids, p.row_begin, p.rows, p.G,
-                                                             p.top_k, p.nb, (int32_t)ntiles, cnt,
-                                                             p.row_base, p.entries);
+  csr_scatter_kernel<<<grid, 32, scatter_bytes, s>>>(p.ids, p.row_begin, p.rows, p.G, p.top_k,
+                                                     p.nb, (int32_t)ntiles, bins, cnt,
+                                                     p.row_base, p.entries);
   ++*launches;
   if (p.unit_ptr) {
-    unit_count_kernel<<<(unsigned)((n_lists + 255) / 256), 256, 0, s>>>(
-        p.row_ptr, n_lists, p.tile_tokens * p.unit_tiles, p.unit_ptr);
-    ++*launches;
-    // unit_ptr[n_lists] = total units: scan n_lists+1 values with a trailing 0
-    if ((e = cudaMemsetAsync(p.unit_ptr + n_lists, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
-    if ((e = exclusive_scan(p.unit_ptr, n_lists + 1, tmp2, s, launches)) != cudaSuccess) return e;
-    unit_fill_kernel<<<(unsigned)((n_lists + 255) / 256), 256, 0, s>>>(
-        p.unit_ptr, p.row_ptr, n_lists, p.nb, p.tile_tokens * p.unit_tiles, p.unit_desc);
+    units_kernel<<<1, kUnitThreads, 0, s>>>(p.row_ptr, n_lists, p.nb,
+                                            p.tile_tokens * p.unit_tiles, p.unit_ptr,
+                                            p.unit_desc);
     ++*launches;
   }
   return cudaGetLastError();
