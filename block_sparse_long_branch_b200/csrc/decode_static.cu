@@ -11,15 +11,15 @@
 //
 // The array occupies kStaticScratchBytes on every GPU that loads this library
 // (when the module is loaded) until the process exits.  Its device address is
-// looked up once per device, on the first call made with that device current;
-// make that first call before any stream capture.  All calls share the array
-// and it keeps the previous call's contents: the decode path clears its error
-// word at the start of every call and writes every other scratch value before
-// reading it.  Calls whose work overlaps on the GPU (different streams, or
-// different host threads) race on the array and must be serialised by the
-// caller.
-#include <mutex>
-
+// looked up with cudaGetSymbolAddress on every call, with the caller's device
+// current: the first call on a device may load the module there, so make it
+// before any stream capture; later calls only look the address up, which also
+// stays right after a cudaDeviceReset recreates the context.  All calls share
+// the array and it keeps the previous call's contents: the decode path clears
+// its error word at the start of every call and writes every other scratch
+// value before reading it.  Calls whose work overlaps on the GPU (different
+// streams, or different host threads) race on the array and must be
+// serialised by the caller.
 #include "../../include/msa.h"
 #include "kernels.h"
 
@@ -30,24 +30,12 @@ constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 128;
-void* g_scratch_ptr[kMaxDevices];
-std::mutex g_scratch_mu;
-
-// Device address of g_decode_scratch on the current device (looked up once).
+// Device address of g_decode_scratch on the current device.
 cudaError_t static_scratch(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return cudaSuccess;
 }
 
