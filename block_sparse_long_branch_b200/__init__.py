@@ -26,7 +26,8 @@ __all__ = [
     "msa_build_block_query_lists", "msa_prefill", "msa_decode", "msa_get_device_error",
     "msa_status_string", "msa_last_launch_count", "msa_set_phase_events", "msa_decode_static",
     "msa_selftest_wait_timeout", "msa_prefill_varlen", "msa_prefill_block_alignment",
-    "msa_prefill_fp8_index", "msa_prefill_varlen_workspace_size",
+    "msa_prefill_fp8_index", "msa_prefill_varlen_workspace_size", "msa_decode_fp8_index",
+    "msa_quantize_rows_fp8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -104,6 +105,8 @@ def load_library():
     lib.msa_prefill_block_alignment.argtypes = [C, P, P, P, P, P, I64, P, P, P, P, P, P, SZ, P]
     lib.msa_decode.argtypes = [C, P, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
     lib.msa_decode_static.argtypes = [C, P, P, P, P, P, P, I32, I64, I64, P, P, I32, P]
+    lib.msa_decode_fp8_index.argtypes = [C, P, P, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
+    lib.msa_quantize_rows_fp8.argtypes = [P, I64, P, P, P]
     lib.msa_get_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
     lib.msa_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
     lib.msa_status_string.argtypes = [ctypes.c_int]
@@ -446,6 +449,51 @@ def msa_decode(cfg: MsaConfig, q, q_idx, k_cache, v_cache, k_idx_cache, cu_seqle
                         _dev(out, torch.bfloat16, "out", (B, H, d)), ids_ptr,
                         _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(st, "msa_decode")
+    return out if ids_out is None else (out, ids_out)
+
+
+def msa_quantize_rows_fp8(x: torch.Tensor, stream=None):
+    """x [..., 128] bf16 -> (x8 uint8 e4m3 bytes of the same shape, scale [...] float32):
+    one scale per row of 128 values."""
+    lib = load_library()
+    rows = x.numel() // 128
+    x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    sc = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    if x.shape[-1] != 128:
+        raise MsaError("msa_quantize_rows_fp8: rows of 128 values expected")
+    st = lib.msa_quantize_rows_fp8(_dev(x, torch.bfloat16, "x"), rows,
+                                   _dev(x8, torch.uint8, "x8"), _dev(sc, torch.float32, "scale"),
+                                   _stream(stream))
+    _check(st, "msa_quantize_rows_fp8")
+    return x8, sc
+
+
+def msa_decode_fp8_index(cfg: MsaConfig, q, q_idx8, k_cache, v_cache, k_idx8_cache, k_idx_scale,
+                         cu_seqlens, max_seqlen: int, out: Optional[torch.Tensor] = None,
+                         ids_out=None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """msa_decode with the e4m3 Index Branch: q_idx8 [B,G,128] and k_idx8_cache
+    [sum L,128] e4m3 bytes, k_idx_scale [sum L] float32 (one scale per key row)."""
+    lib = load_library()
+    B = q.shape[0]
+    H, G, d, di, kk = cfg.num_heads, cfg.num_groups, cfg.head_dim, cfg.index_dim, cfg.top_k
+    total = k_cache.shape[0]
+    if out is None:
+        out = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
+    if ids_out is True:
+        ids_out = torch.empty((B, G, kk), dtype=torch.int32, device=q.device)
+    ws = _workspace(workspace, msa_workspace_size(cfg, OP_DECODE, total, B), q.device)
+    ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (B, G, kk))
+    st = lib.msa_decode_fp8_index(
+        ctypes.byref(cfg), _dev(q, torch.bfloat16, "q", (B, H, d)),
+        _dev(q_idx8, torch.uint8, "q_idx8", (B, G, di)),
+        _dev(k_cache, torch.bfloat16, "k_cache", (total, G, d)),
+        _dev(v_cache, torch.bfloat16, "v_cache", (total, G, d)),
+        _dev(k_idx8_cache, torch.uint8, "k_idx8_cache", (total, di)),
+        _dev(k_idx_scale, torch.float32, "k_idx_scale", (total,)),
+        _dev(cu_seqlens, torch.int64, "cu_seqlens", (B + 1,)), B, max_seqlen,
+        _dev(out, torch.bfloat16, "out", (B, H, d)), ids_ptr,
+        _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(st, "msa_decode_fp8_index")
     return out if ids_out is None else (out, ids_out)
 
 

@@ -71,7 +71,7 @@ int sm_count() {
 // ---- prefill workspace: the fp16 copy of V for all N tokens, then the
 // scratch of one chunk of `rows` query rows ---------------------------------
 struct PrefillLayout {
-  size_t v16, ids, row_ptr, entries, unit_ptr, unit_list, csr, part_o, part_lse, total;
+  size_t v16, vexp, ids, row_ptr, entries, unit_ptr, unit_list, csr, part_o, part_ml, total;
 };
 
 PrefillLayout prefill_layout(const msa_config_t* c, int64_t N, int64_t rows, int64_t nb,
@@ -84,8 +84,13 @@ PrefillLayout prefill_layout(const msa_config_t* c, int64_t N, int64_t rows, int
   PrefillLayout L;
   size_t off = kHeader;
   // at a fixed offset for every chunk of the call: converted once, read by all
+  // (the scale exponents cover every key block: nb is the call's block count
+  // for a packed batch, at most n_blocks(N) for a chunk of one sequence)
+  const int64_t nb_all = nb > n_blocks(N) ? nb : n_blocks(N);
   L.v16 = off;
   off += align256(N * G * c->head_dim * 2);
+  L.vexp = off;
+  off += align256(nb_all * G * 4);
   L.ids = off;
   off += own_ids ? align256(slots * 4) : 0;
   L.row_ptr = off;
@@ -100,8 +105,8 @@ PrefillLayout prefill_layout(const msa_config_t* c, int64_t N, int64_t rows, int
   off += csr_scratch_bytes(rows, (int32_t)G, (int32_t)k, nb);
   L.part_o = off;
   off += align256(slots * HG * c->head_dim * 2);
-  L.part_lse = off;
-  off += align256(slots * HG * 4);
+  L.part_ml = off;
+  off += align256(slots * HG * 8);
   L.total = off;
   return L;
 }
@@ -414,8 +419,10 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
   const int sms = sm_count();
   uint32_t* err = at<uint32_t>(ws, 0);
   int launches = 0;
-  // V in fp16 for the PV product (its offset is the same for every chunk)
-  void* v16 = at<void>(ws, prefill_layout(cfg, N, chunk, nb, own_ids).v16);
+  // V' in fp16 for the PV product (its offset is the same for every chunk)
+  const PrefillLayout L0 = prefill_layout(cfg, N, chunk, nb, own_ids);
+  void* v16 = at<void>(ws, L0.v16);
+  int32_t* vexp = at<int32_t>(ws, L0.vexp);
   for (int64_t t0 = 0, c = 0; t0 < N; t0 += chunk, ++c) {
     const int64_t t1 = t0 + chunk < N ? t0 + chunk : N;
     const int ev = (int)(5 * c);
@@ -479,7 +486,7 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
     mark(ev + 2, s);
 
     if (c == 0) {  // converted once, before the first Main Branch launch
-      if (launch_v_to_fp16(v, v16, N * G * d, err, sms, s) != cudaSuccess)
+      if (launch_v_to_fp16(v, v16, vexp, N, G, d, nb, nullptr, err, sms, s) != cudaSuccess)
         return cuda_status(cudaErrorLaunchFailure);
       ++launches;
     }
@@ -500,8 +507,9 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
     mp.entries = cp.entries;
     mp.unit_ptr = cp.unit_ptr;
     mp.unit_desc = cp.unit_desc;
+    mp.vexp = vexp;
     mp.part_o = at<__half>(ws, L.part_o);
-    mp.part_lse = at<float>(ws, L.part_lse);
+    mp.part_ml = at<float2>(ws, L.part_ml);
     mp.err = err;
     mp.grid = sms;
     if (launch_main(mp, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
@@ -510,7 +518,7 @@ msa_status_t prefill_run(const msa_config_t* cfg, const void* q, const void* k, 
 
     MergeLaunch gp{};
     gp.part_o = mp.part_o;
-    gp.part_lse = mp.part_lse;
+    gp.part_ml = mp.part_ml;
     gp.ids = ids;
     gp.rows = rows;
     gp.H = H;
@@ -643,7 +651,8 @@ msa_status_t prefill_packed(const msa_config_t* cfg, const void* q, const void* 
   if (launch_csr(cp, s, &launches) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
 
   void* v16 = at<void>(ws, L.v16);
-  if (launch_v_to_fp16(v, v16, N * G * d, err, sms, s) != cudaSuccess)
+  int32_t* vexp = at<int32_t>(ws, L.vexp);
+  if (launch_v_to_fp16(v, v16, vexp, N, G, d, NB, pl.blk_row0, err, sms, s) != cudaSuccess)
     return cuda_status(cudaErrorLaunchFailure);
   ++launches;
   MainLaunch mp{};
@@ -664,8 +673,9 @@ msa_status_t prefill_packed(const msa_config_t* cfg, const void* q, const void* 
   mp.unit_ptr = cp.unit_ptr;
   mp.unit_desc = cp.unit_desc;
   mp.blk_row0 = pl.blk_row0;
+  mp.vexp = vexp;
   mp.part_o = at<__half>(ws, L.part_o);
-  mp.part_lse = at<float>(ws, L.part_lse);
+  mp.part_ml = at<float2>(ws, L.part_ml);
   mp.err = err;
   mp.grid = sms;
   if (launch_main(mp, s) != cudaSuccess) return cuda_status(cudaErrorLaunchFailure);
@@ -673,7 +683,7 @@ msa_status_t prefill_packed(const msa_config_t* cfg, const void* q, const void* 
 
   MergeLaunch gp{};
   gp.part_o = mp.part_o;
-  gp.part_lse = mp.part_lse;
+  gp.part_ml = mp.part_ml;
   gp.ids = ids;
   gp.rows = N;
   gp.H = H;
@@ -843,10 +853,13 @@ msa_status_t msa_prefill_varlen(const msa_config_t* cfg, const void* q, const vo
   return MSA_OK;
 }
 
-msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_idx,
+namespace {
+// msa_decode, or with k_idx_scale set its e4m3-index variant
+msa_status_t decode_run(const msa_config_t* cfg, const void* q, const void* q_idx,
                         const void* k_cache, const void* v_cache, const void* k_idx_cache,
-                        const int64_t* cu_seqlens, int32_t B, int64_t max_seqlen, void* out,
-                        int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream) {
+                        const float* k_idx_scale, const int64_t* cu_seqlens, int32_t B,
+                        int64_t max_seqlen, void* out, int32_t* ids_out, void* ws,
+                        size_t ws_bytes, msa_stream_t stream) {
   g_launches = 0;
   msa_status_t st = check_cfg(cfg);
   if (st != MSA_OK) return st;
@@ -872,6 +885,7 @@ msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_id
   p.k_cache = k_cache;
   p.v_cache = v_cache;
   p.k_idx_cache = k_idx_cache;
+  p.k_idx_scale = k_idx_scale;
   p.cu_seqlens = cu_seqlens;
   p.B = B;
   p.H = cfg->num_heads;
@@ -900,6 +914,43 @@ msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_id
   int launches = 0;
   st = cuda_status(launch_decode(p, s, &launches));
   g_launches = launches;
+  return st;
+}
+}  // namespace
+
+msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const void* q_idx,
+                        const void* k_cache, const void* v_cache, const void* k_idx_cache,
+                        const int64_t* cu_seqlens, int32_t B, int64_t max_seqlen, void* out,
+                        int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream) {
+  return decode_run(cfg, q, q_idx, k_cache, v_cache, k_idx_cache, nullptr, cu_seqlens, B,
+                    max_seqlen, out, ids_out, ws, ws_bytes, stream);
+}
+
+msa_status_t msa_decode_fp8_index(const msa_config_t* cfg, const void* q, const void* q_idx8,
+                                  const void* k_cache, const void* v_cache,
+                                  const void* k_idx8_cache, const float* k_idx_scale,
+                                  const int64_t* cu_seqlens, int32_t B, int64_t max_seqlen,
+                                  void* out, int32_t* ids_out, void* ws, size_t ws_bytes,
+                                  msa_stream_t stream) {
+  g_launches = 0;
+  const msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if (cfg->index_dim != 128) return MSA_ERR_UNSUPPORTED;
+  if (!k_idx_scale || !aligned16(k_idx_scale)) return MSA_ERR_INVALID_ARG;
+  return decode_run(cfg, q, q_idx8, k_cache, v_cache, k_idx8_cache, k_idx_scale, cu_seqlens, B,
+                    max_seqlen, out, ids_out, ws, ws_bytes, stream);
+}
+
+msa_status_t msa_quantize_rows_fp8(const void* x, int64_t rows, void* x8, float* scale,
+                                   msa_stream_t stream) {
+  g_launches = 0;
+  if (rows < 0) return MSA_ERR_INVALID_ARG;
+  if (rows == 0) return MSA_OK;
+  if (!x || !x8 || !scale || !aligned16(x) || !aligned16(x8) || !aligned16(scale))
+    return MSA_ERR_INVALID_ARG;
+  const msa_status_t st = cuda_status(
+      launch_quantize_rows(x, rows, x8, scale, reinterpret_cast<cudaStream_t>(stream)));
+  if (st == MSA_OK) g_launches = 1;
   return st;
 }
 

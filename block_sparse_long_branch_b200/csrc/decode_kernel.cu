@@ -8,7 +8,9 @@
 //      scores a 128-key block against the sequence's G index queries with
 //      mma.sync m16n8k16 (keys as M, groups as N).  The reduction axis is
 //      permuted identically for both operands so that every lane reads 16
-//      contiguous bytes of a key row straight from global memory.
+//      contiguous bytes of a key row straight from global memory.  With an
+//      e4m3 cache (one fp32 scale per key row), decode_index_fp8_kernel does
+//      the same on mma.sync m16n8k32 e4m3 over half the bytes.
 //      Writes the pooled (max) score of every non-local block, [G][nb] per
 //      sequence so that each group's scores are contiguous.
 //   2. decode_attend_kernel : n_split CTAs per (sequence, group).  Each one
@@ -111,6 +113,102 @@ __global__ void __launch_bounds__(kIdxWarps * 32)
                          qw[2 * kk + 1]);
         m0 = fmaxf(m0, fmaxf(acc[0], acc[2]));
         m1 = fmaxf(m1, fmaxf(acc[1], acc[3]));
+      }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      }
+      if (gq == 0) {
+        const int g0 = nt * 8 + 2 * tq;
+        if (g0 < G) pout[(int64_t)g0 * nb + j] = m0;
+        if (g0 + 1 < G) pout[(int64_t)(g0 + 1) * nb + j] = m1;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void mma_e4m3_16832(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The same scan over an e4m3 index-key cache with one fp32 scale per cached
+// key row (index dim 128): the score of key s is kscale[s] * <q8, k8[s]> (the
+// query's own scale, a positive constant of the (sequence, group), is left
+// out: it cannot change the ranking).  Lane (g = lane/4, t = lane%4) owns bytes
+// [32t, 32t+32) of key rows g and g+8 of each 16-key tile; in k-step kk its mma
+// positions (4t..4t+3 | 16+4t..16+4t+3) hold physical bytes 32t + 8kk + (0..3 |
+// 4..7), and q8 uses the same map, so the dot products are unchanged.
+__global__ void __launch_bounds__(kIdxWarps * 32)
+    decode_index_fp8_kernel(const uint8_t* __restrict__ q_idx8, const uint8_t* __restrict__ k_idx8,
+                            const float* __restrict__ kscale, const int64_t* __restrict__ cu,
+                            int32_t G, float* __restrict__ pooled, int64_t pooled_cap,
+                            uint32_t* err) {
+  constexpr int DI = 128;
+  constexpr int WPR = DI / 16;  // 32-bit words per lane per key row (32 bytes)
+  constexpr int STEPS = DI / 32;
+  const int b = blockIdx.y;
+  const int64_t s0 = cu[b];
+  const int64_t L = cu[b + 1] - s0;
+  const int64_t nb = (L + kBlock - 1) / kBlock;
+  const int64_t j_lo = (int64_t)blockIdx.x * kBlocksPerCta;
+  const int64_t j_hi = min64(j_lo + kBlocksPerCta, nb - 1);  // non-local blocks only
+  if (j_lo >= j_hi) return;
+  if (pooled_offset(cu, b) + nb > pooled_cap) {  // workspace sized for fewer cache rows
+    if (threadIdx.x == 0) record_error(err, kDevBadIndex);
+    return;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int n_tiles = (G + 7) / 8;
+  float* pout = pooled + pooled_offset(cu, b) * G;
+
+  for (int nt = 0; nt < n_tiles; ++nt) {
+    uint32_t qw[WPR];
+    const int grp = nt * 8 + gq;
+    if (grp < G) {
+      const uint4* src =
+          reinterpret_cast<const uint4*>(q_idx8 + ((int64_t)b * G + grp) * DI + tq * (DI / 4));
+#pragma unroll
+      for (int i = 0; i < WPR / 4; ++i) {
+        const uint4 v = __ldg(src + i);
+        qw[4 * i] = v.x, qw[4 * i + 1] = v.y, qw[4 * i + 2] = v.z, qw[4 * i + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < WPR; ++i) qw[i] = 0;
+    }
+    for (int64_t j = j_lo + warp; j < j_hi; j += kIdxWarps) {
+      const int64_t row0 = s0 + j * kBlock;
+      const uint8_t* blk = k_idx8 + row0 * DI;
+      float m0 = -INFINITY, m1 = -INFINITY;  // groups nt*8 + 2tq, +1
+#pragma unroll 2
+      for (int mt = 0; mt < kBlock / 16; ++mt) {
+        uint32_t w0[WPR], w1[WPR];
+        const uint4* r0 = reinterpret_cast<const uint4*>(blk + (mt * 16 + gq) * DI + tq * (DI / 4));
+        const uint4* r1 =
+            reinterpret_cast<const uint4*>(blk + (mt * 16 + gq + 8) * DI + tq * (DI / 4));
+#pragma unroll
+        for (int i = 0; i < WPR / 4; ++i) {
+          const uint4 a = __ldg(r0 + i), c = __ldg(r1 + i);
+          w0[4 * i] = a.x, w0[4 * i + 1] = a.y, w0[4 * i + 2] = a.z, w0[4 * i + 3] = a.w;
+          w1[4 * i] = c.x, w1[4 * i + 1] = c.y, w1[4 * i + 2] = c.z, w1[4 * i + 3] = c.w;
+        }
+        const float sc0 = __ldg(kscale + row0 + mt * 16 + gq);
+        const float sc1 = __ldg(kscale + row0 + mt * 16 + gq + 8);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < STEPS; ++kk)
+          mma_e4m3_16832(acc, w0[2 * kk], w1[2 * kk], w0[2 * kk + 1], w1[2 * kk + 1], qw[2 * kk],
+                         qw[2 * kk + 1]);
+        m0 = fmaxf(m0, fmaxf(acc[0] * sc0, acc[2] * sc1));
+        m1 = fmaxf(m1, fmaxf(acc[1] * sc0, acc[3] * sc1));
       }
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
@@ -707,7 +805,12 @@ cudaError_t launch_decode(const DecodeLaunch& p, cudaStream_t s, int* launches) 
   dim3 gi((unsigned)(chunks > 0 ? chunks : 1), (unsigned)p.B);
   const auto* qi = static_cast<const __nv_bfloat16*>(p.q_idx);
   const auto* ki = static_cast<const __nv_bfloat16*>(p.k_idx_cache);
-  if (p.d_idx == 128)
+  if (p.k_idx_scale) {
+    if (p.d_idx != 128) return cudaErrorInvalidValue;
+    decode_index_fp8_kernel<<<gi, kIdxWarps * 32, 0, s>>>(
+        static_cast<const uint8_t*>(p.q_idx), static_cast<const uint8_t*>(p.k_idx_cache),
+        p.k_idx_scale, p.cu_seqlens, p.G, p.pooled, p.pooled_cap, p.err);
+  } else if (p.d_idx == 128)
     decode_index_kernel<128><<<gi, kIdxWarps * 32, 0, s>>>(qi, ki, p.cu_seqlens, p.G, p.pooled,
                                                             p.pooled_cap, p.err);
   else

@@ -90,24 +90,28 @@ struct MainLaunch {
   const int32_t* unit_ptr;   // [G*nb+1]
   const int4* unit_desc;     // [units] {g, j, first entry, end entry}
   const int32_t* blk_row0;   // optional, packed sequences: first K/V row of key block j
-  __half* part_o;   // [rows][G][top_k][H/G][d] fp16
-  float* part_lse;  // [rows][G][top_k][H/G] fp32
+  const int32_t* vexp;       // [nb][G] from launch_v_to_fp16
+  __half* part_o;   // [rows][G][top_k][H/G][d] fp16, unnormalised o'
+  float2* part_ml;  // [rows][G][top_k][H/G] (m~, l~)
   uint32_t* err;
   int grid;
 };
 // query tokens per 128-row Main Branch tile
 int main_tile_tokens(int H, int G);
-// dst = fp16(src) for n bf16 values (n a multiple of 8, both pointers 16-byte
-// aligned): the V operand of the Main Branch's PV product.  A value beyond the
-// fp16 range (or NaN) is saturated and records kDevValueRange.
-cudaError_t launch_v_to_fp16(const void* src, void* dst, int64_t n, uint32_t* err, int sms,
-                             cudaStream_t s);
+// V' = fp16(V * 2^-e) for the PV product of the Main Branch: V [N][G][d] bf16,
+// V' the same layout (both 16-byte aligned, d a multiple of 8, G <= 128).  Key
+// block j (rows blk_row0[j] .. blk_row0[j+1]-1, or 128j .. 128j+127) and group
+// g take the smallest e >= 0 with max|v| * 2^-e <= 511.75, written to
+// vexp[j*G + g].  A NaN or infinite value records kDevValueRange.
+cudaError_t launch_v_to_fp16(const void* src, void* dst, int32_t* vexp, int64_t N, int32_t G,
+                             int32_t d, int64_t nb, const int32_t* blk_row0, uint32_t* err,
+                             int sms, cudaStream_t s);
 cudaError_t launch_main(const MainLaunch& p, cudaStream_t s);
 
 // ---- merge (merge_kernel.cu) ----------------------------------------------
 struct MergeLaunch {
   const __half* part_o;
-  const float* part_lse;
+  const float2* part_ml;
   const int32_t* ids;  // [rows][G][top_k]
   int64_t rows;
   int32_t H, G, d, top_k;
@@ -132,6 +136,10 @@ struct QuantLaunch {
   float* kscale;
 };
 cudaError_t launch_quantize_index(const QuantLaunch& p, cudaStream_t s);
+// rows x 128 bf16 -> e4m3 with one fp32 scale per row (the same rule as the
+// index-query rows above): x8 [rows][128], scale [rows]
+cudaError_t launch_quantize_rows(const void* x, int64_t rows, void* x8, float* scale,
+                                 cudaStream_t s);
 
 // Block-alignment diagnostic: pooled index score of every listed (t, r).
 struct BlockScoreLaunch {
@@ -153,7 +161,10 @@ struct DecodeLaunch {
   const void* q_idx;        // [B][G][d_idx]
   const void* k_cache;      // [sumL][G][d]
   const void* v_cache;      // [sumL][G][d]
-  const void* k_idx_cache;  // [sumL][d_idx]
+  const void* k_idx_cache;  // [sumL][d_idx] bf16, or e4m3 when k_idx_scale is set
+  // optional: e4m3 index cache -- q_idx [B][G][128] and k_idx_cache [sumL][128]
+  // are e4m3 bytes and key row s scores k_idx_scale[s] * <q8, k8[s]>
+  const float* k_idx_scale;
   const int64_t* cu_seqlens;
   int32_t B, H, G, d, d_idx, top_k;
   int64_t max_seqlen;

@@ -2,10 +2,12 @@
 //
 // The Main Branch is one exact softmax over all selected keys (ai-tool-zukan
 // "MiniMax MSA guide", section "Index BranchとMain Branchの役割分担").  The
-// key-block-outer kernel produces it in pieces, one per selected block r:
-// o_r (normalised over block r) and lse_r = log sum_{s in r} exp(logit_s).
-// The exact result is  out = sum_r exp(lse_r - L) o_r  with  L = log sum_r
-// exp(lse_r),  i.e. the standard log-sum-exp split of a softmax.
+// key-block-outer kernel produces it in pieces, one per selected block r: the
+// unnormalised o'_r = sum_{s in r} exp(logit_s - m_r) v'_s, where v' is the
+// value row scaled by 2^-e_r, with m~_r = m_r + e_r ln2 and l~_r = 2^-e_r
+// sum_{s in r} exp(logit_s - m_r).  With M = max_r m~_r and w_r = exp(m~_r - M)
+// the exact result is  out = sum_r w_r o'_r / sum_r w_r l~_r,  the standard
+// max-shifted split of a softmax (the 2^e_r factors cancel).
 //
 // One warp per (query t, group g).  The group's H/G heads x d values of one
 // slot are contiguous (2 KiB for 8 heads of 128): lane l owns CPL consecutive
@@ -24,7 +26,7 @@ constexpr int kWarps = 8;
 // of that mass from the softmax of the slots' pooled index scores.
 template <int CPL, int KMAX, bool ALIGN>
 __global__ void __launch_bounds__(kWarps * 32)
-    merge_kernel(const __half* __restrict__ part_o, const float* __restrict__ part_lse,
+    merge_kernel(const __half* __restrict__ part_o, const float2* __restrict__ part_ml,
                  const int32_t* __restrict__ ids, int64_t rows, int32_t G, int32_t HG, int32_t d,
                  int32_t top_k, __nv_bfloat16* __restrict__ out, float* __restrict__ block_score,
                  float* __restrict__ block_mass, float* __restrict__ kl) {
@@ -40,27 +42,37 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int h = active ? (c0 * 8) / d : 0;
   const int64_t slot_elems = (int64_t)HG * d;
   const __half* o_tg = part_o + tg * top_k * slot_elems + (int64_t)c0 * 8;
-  const float* l_tg = part_lse + tg * top_k * HG + h;
+  const float2* l_tg = part_ml + tg * top_k * HG + h;
 
-  float lse[KMAX];
+  // slot r's weight w_r = exp(m~_r - M) (in wt[r], 0 for empty slots) and the
+  // normaliser sum_r w_r l~_r; l~ is not kept past this point
+  float wt[KMAX], lt[KMAX];
   float m = -INFINITY;
 #pragma unroll
   for (int r = 0; r < KMAX; ++r) {
-    lse[r] = (active && r < top_k && (valid >> r & 1u)) ? __ldg(l_tg + r * HG) : -INFINITY;
-    m = fmaxf(m, lse[r]);
+    const bool use = active && r < top_k && (valid >> r & 1u);
+    const float2 ml = use ? __ldg(l_tg + r * HG) : make_float2(-INFINITY, 0.f);
+    wt[r] = ml.x;
+    lt[r] = ml.y;
+    m = fmaxf(m, wt[r]);
+  }
+  float wsum = 0.f;
+#pragma unroll
+  for (int r = 0; r < KMAX; ++r) {
+    wt[r] = (r < top_k && (valid >> r & 1u)) ? __expf(wt[r] - m) : 0.f;
+    // explicit roundings: the same sum whether or not the products are kept
+    // for the alignment outputs (no fused multiply-add in one variant only)
+    lt[r] = __fmul_rn(lt[r], wt[r]);
+    wsum = __fadd_rn(wsum, lt[r]);
   }
   if (ALIGN) {
     // per slot: this head's softmax weight; summed over the head leaders
     // (the first lane of each head) and divided by H/G
-    float ws = 0.f;
-#pragma unroll
-    for (int r = 0; r < KMAX; ++r)
-      if (r < top_k && (valid >> r & 1u)) ws += __expf(lse[r] - m);
     const bool leader = active && (c0 * 8) % d == 0;
     float mass[KMAX];
 #pragma unroll
     for (int r = 0; r < KMAX; ++r) {
-      float w = (leader && r < top_k && (valid >> r & 1u)) ? __expf(lse[r] - m) / ws : 0.f;
+      float w = (leader && r < top_k && (valid >> r & 1u)) ? lt[r] / wsum : 0.f;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
       mass[r] = w / (float)HG;
@@ -93,12 +105,10 @@ __global__ void __launch_bounds__(kWarps * 32)
   float acc[CPL * 8];
 #pragma unroll
   for (int x = 0; x < CPL * 8; ++x) acc[x] = 0.f;
-  float wsum = 0.f;
 #pragma unroll
   for (int r = 0; r < KMAX; ++r) {
     if (r >= top_k || !(valid >> r & 1u)) continue;
-    const float w = __expf(lse[r] - m);
-    wsum += w;
+    const float w = wt[r];
     const uint4* src = reinterpret_cast<const uint4*>(o_tg + r * slot_elems);
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
@@ -132,7 +142,7 @@ cudaError_t launch_k(const MergeLaunch& p, cudaStream_t s, unsigned grid) {
   const int HG = p.H / p.G;
 #define MSA_MERGE(CPL)                                                                       \
   merge_kernel<CPL, KMAX, ALIGN><<<grid, kWarps * 32, 0, s>>>(                               \
-      p.part_o, p.part_lse, p.ids, p.rows, p.G, HG, p.d, p.top_k, o, p.block_score,          \
+      p.part_o, p.part_ml, p.ids, p.rows, p.G, HG, p.d, p.top_k, o, p.block_score,          \
       p.block_mass, p.kl)
   if (chunks >= 256)
     MSA_MERGE(8);

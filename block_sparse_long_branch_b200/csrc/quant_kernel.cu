@@ -29,10 +29,12 @@ __device__ __forceinline__ float scale_of(float amax) {
   return amax > 0.f ? __fdiv_rn(amax, kE4m3Max) : 1.f;
 }
 
-// one warp per index-query row of DI values (DI / 32 per lane)
+// one warp per row of DI values (DI / 32 per lane); the row's scale is written
+// to `scale` when it is given
 template <int DI>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16* __restrict__ x,
-                                                         int64_t rows, uint8_t* __restrict__ x8) {
+                                                         int64_t rows, uint8_t* __restrict__ x8,
+                                                         float* __restrict__ scale) {
   constexpr int PER = DI / 32;
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (r >= rows) return;
@@ -48,6 +50,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16* __
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const float s = scale_of(amax);
+  if (scale && lane == 0) scale[r] = s;
 #pragma unroll
   for (int i = 0; i < PER; ++i) x8[r * DI + lane * PER + i] = to_e4m3(__fdiv_rn(v[i], s));
 }
@@ -87,11 +90,19 @@ cudaError_t launch_quantize_index(const QuantLaunch& p, cudaStream_t s) {
   const auto* q = static_cast<const __nv_bfloat16*>(p.q_idx);
   const auto* k = static_cast<const __nv_bfloat16*>(p.k_idx);
   quant_rows_kernel<128><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
-      q, rows, static_cast<uint8_t*>(p.q_idx8));
+      q, rows, static_cast<uint8_t*>(p.q_idx8), nullptr);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   quant_blocks_kernel<128><<<(unsigned)nb, 256, 0, s>>>(k, p.N, static_cast<uint8_t*>(p.k_idx8),
                                                         p.kscale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rows(const void* x, int64_t rows, void* x8, float* scale,
+                                 cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  quant_rows_kernel<128><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, static_cast<uint8_t*>(x8), scale);
   return cudaGetLastError();
 }
 

@@ -170,9 +170,13 @@ MSA_API msa_status_t msa_build_block_query_lists(const msa_config_t* cfg, const 
  *   out [N][H][d] bf16 out: softmax over the keys s <= t of the selected
  *       blocks of softmax_scale*<q[t][h], k[s][g]>, times v[s][g]; fp32
  *       accumulation, rounded to bf16 (nearest even).  The probabilities
- *       and v meet on the tensor cores in fp16, so v must lie within the
- *       fp16 range (|v| <= 65504): a value beyond it, or NaN, is saturated
- *       and recorded as 0x301 (MSA_ERR_DEVICE_RANGE) in the device error word.
+ *       and v meet on the tensor cores in fp16: each key block's v (per
+ *       group) is first scaled by the power of two 2^-e that brings its
+ *       largest |v| to at most 511.75 (e = 0 when it already is), so any
+ *       finite bf16 v is accepted; within a block scaled this way, values
+ *       below 2^(e-14) are held to an absolute 2^(e-25).  A NaN or infinite
+ *       v is recorded as 0x301 (MSA_ERR_DEVICE_RANGE) in the device error
+ *       word.
  *   ids_out [N][G][k] int32 out, nullable: the selection used.
  *   ws: at least msa_prefill_min_workspace(); with less than
  *       msa_workspace_size(PREFILL, N) the query axis is processed in chunks.
@@ -303,6 +307,41 @@ MSA_API msa_status_t msa_decode(const msa_config_t* cfg, const void* q, const vo
                         int32_t* ids_out, void* ws, size_t ws_bytes, msa_stream_t stream);
 
 /*
+ * msa_decode with the quantised (e4m3) Index Branch over an e4m3 index-key
+ * cache: the "Q8" indexer of the model card's Q8KV8 -> Q8KV4 move (dot-ai
+ * "MiniMax M3.1 Flashとは？428BのMoEモデルがウェイト公開", the passage on the
+ * ModelScope model card's quantisation), read as e4m3 with one fp32 scale per
+ * index-key row: a decode cache grows by one token at a time, and a per-row
+ * scale lets each token be quantised once, when it is appended.
+ *   q_idx8 [B][G][128] e4m3 bytes (per-row scales, as msa_quantize_rows_fp8
+ *     writes them; the query scales are not needed: a positive constant of a
+ *     (sequence, group) cannot change its ranking);
+ *   k_idx8_cache [sum L][128] e4m3 bytes, k_idx_scale [sum L] fp32 (device,
+ *     every entry finite and > 0; not checked on the device): key row s
+ *     scores k_idx_scale[s] * <q_idx8[b][g], k_idx8_cache[s]> (fp32
+ *     accumulation of exact e4m3 products), max-pooled per block.
+ *   Everything else (q, k/v caches, cu_seqlens, outputs, workspace, H/G
+ *   limit) as for msa_decode.  d_idx other than 128 -> MSA_ERR_UNSUPPORTED.
+ */
+MSA_API msa_status_t msa_decode_fp8_index(const msa_config_t* cfg, const void* q,
+                                          const void* q_idx8, const void* k_cache,
+                                          const void* v_cache, const void* k_idx8_cache,
+                                          const float* k_idx_scale, const int64_t* cu_seqlens,
+                                          int32_t B, int64_t max_seqlen, void* out,
+                                          int32_t* ids_out, void* ws, size_t ws_bytes,
+                                          msa_stream_t stream);
+
+/*
+ * Per-row e4m3 quantiser for the decode index tensors (same passage and
+ * reading as above): x [rows][128] bf16 -> x8 [rows][128] e4m3 bytes and
+ * scale [rows] fp32, s = max|x| / 448 (fp32, nearest; 1 for an all-zero row),
+ * x8 = e4m3(x / s) (fp32 division, nearest even, saturating at +-448).  All
+ * pointers device, 16-byte aligned.  rows = 0 is a no-op.
+ */
+MSA_API msa_status_t msa_quantize_rows_fp8(const void* x, int64_t rows, void* x8, float* scale,
+                                           msa_stream_t stream);
+
+/*
  * msa_decode without a workspace argument, for callers that cannot allocate
  * device memory (a serving loop whose memory another runtime reserved up
  * front, a thread that must not enter the allocator, an embedding that only
@@ -332,8 +371,8 @@ MSA_API msa_status_t msa_decode_static(const msa_config_t* cfg, const void* q, c
  * above.  Synchronises `stream` first.  *code = 0 when no kernel reported a
  * problem; otherwise the first code recorded (0x1xx: a wait ran out ->
  * returns MSA_ERR_DEVICE_TIMEOUT; 0x2xx: an out-of-range id ->
- * MSA_ERR_DEVICE_INDEX; 0x301: a prefill V value beyond the fp16 range, or
- * NaN -> MSA_ERR_DEVICE_RANGE).
+ * MSA_ERR_DEVICE_INDEX; 0x301: a prefill V value that is NaN or infinite ->
+ * MSA_ERR_DEVICE_RANGE).
  */
 MSA_API msa_status_t msa_get_device_error(void* ws, msa_stream_t stream, uint32_t* code);
 

@@ -349,3 +349,34 @@ def pooled_scores_fp8(q8_rows, pos, k8, k_scale, block: int, nb_out: int) -> np.
     lib.msa_oracle_pooled_scores_f64(_ptr(qv), _ptr(pos), n, _ptr(kv), G, di, block, nb_out,
                                      _ptr(out))
     return out
+
+
+# ---------------------------------------------------------------------------
+# Quantised Index Branch over a decode cache: the same e4m3 reading with one
+# fp32 scale per index-key row (a cache grows one token at a time, and each
+# token is quantised once, when it is appended); the query rows as above.
+# ---------------------------------------------------------------------------
+
+def quantize_rows_fp8(x):
+    """x [..., d] bf16 -> (x8 [..., d] u8, scale [...] f32): per row of d values,
+    s = max|x| / 448 in fp32 (1 when the max is 0), x8 = e4m3(x / s)."""
+    xf = bf16_bits_to_f64(as_bf16_bits(x)).astype(np.float32)
+    s = _scale(np.abs(xf).max(axis=-1))
+    return e4m3_encode(xf / s[..., None]), s
+
+
+def pooled_scores_fp8_rows(q8_rows, pos, k8, k_row_scale, block: int, nb_out: int) -> np.ndarray:
+    """Pooled scores of the quantised Index Branch with per-key-row scales: the
+    max over visible keys s of <e4m3(q8), e4m3(k8[s]) * k_row_scale[s]> (fp64)."""
+    lib = _load()
+    qv = np.ascontiguousarray(e4m3_decode(q8_rows), dtype=np.float64)
+    kv = e4m3_decode(k8) * np.asarray(k_row_scale, dtype=np.float64)[:, None]
+    kv = np.ascontiguousarray(kv, dtype=np.float64)
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int64))
+    n, G, di = qv.shape
+    assert kv.shape[1] == di and pos.shape == (n,)
+    assert n == 0 or kv.shape[0] > int(pos.max())
+    out = np.empty((n, G, nb_out), dtype=np.float64)
+    lib.msa_oracle_pooled_scores_f64(_ptr(qv), _ptr(pos), n, _ptr(kv), G, di, block, nb_out,
+                                     _ptr(out))
+    return out

@@ -61,16 +61,53 @@ def test_context_usable_after_timeout(msa):
     assert (ids[:, :, 0] >= 0).all()
 
 
-def test_v_beyond_fp16_range_is_reported(msa):
-    """The PV product runs in fp16: a V value beyond 65504 is saturated and
-    recorded as 0x301 in the device error word; the prefill completes, other
-    rows are unaffected and the next read finds the word cleared."""
+def test_v_beyond_fp16_range_is_computed(msa):
+    """The PV product runs in fp16 on V scaled, per key block and group, by a
+    power of two: values far beyond the fp16 range are computed like any other,
+    with no error recorded.  Block 1 of group 0 is scaled by 300 (|v| up to
+    about 1.3e3) and one value of block 2, group 1 is 1e5."""
     import oracle
-    import synth
     from tests import parity
     s = synth.PrefillShape("vrange", N=512, H=8, G=2, d=64, d_idx=64, top_k=4, seed=71)
     inp = synth.make_prefill_inputs(s, device="cuda")
+    inp["v"][128:256, 0, :] = (inp["v"][128:256, 0, :].float() * 300.0).to(torch.bfloat16)
     inp["v"][300, 1, 5] = 1.0e5
+    cfg = msa.config(s.H, s.G, s.d, s.d_idx, top_k=s.top_k, scale=s.scale)
+    ws = torch.empty(msa.msa_workspace_size(cfg, msa.OP_PREFILL, s.N), dtype=torch.uint8,
+                     device="cuda")
+    out = msa.msa_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                          workspace=ws)
+    assert msa.msa_get_device_error(ws) == 0
+    ref = oracle.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], block=s.block,
+                         top_k=s.top_k, scale=s.scale)
+    got = out.float().cpu().numpy().astype(np.float64)
+    want = ref["out"]
+    assert np.isfinite(got).all()
+    # the same weights on |v|: sum_s p_s |v_s|, the size of the terms each
+    # output is summed from (the oracle on |V|)
+    mag = oracle.prefill(inp["q"], inp["k"], inp["v"].abs(), inp["q_idx"], inp["k_idx"],
+                         block=s.block, top_k=s.top_k, scale=s.scale)["out"]
+    # outputs summed from ordinary values meet the usual bar; where large values
+    # enter, fp16 P and fp16 partials add up to 2^-9 of the terms' size
+    err = np.abs(got - want)
+    bound = np.maximum(parity.OUT_MAX_ABS, parity.bf16_half_spacing(want) + parity.OUT_ARITH)
+    bound = bound + np.where(mag > 4.0, 2.0 ** -9 * mag, 0.0)
+    assert (err <= bound).all(), float((err - bound).max())
+    assert np.abs(want).max() > 1.0e3  # the large values reached the outputs
+    plain = mag <= 4.0
+    assert plain.mean() > 0.5 and err[plain].max() <= parity.OUT_MAX_ABS
+
+
+@pytest.mark.parametrize("bad", [float("nan"), float("inf")])
+def test_v_not_finite_is_reported(msa, bad):
+    """A NaN or infinite V value is recorded as 0x301 in the device error word;
+    the prefill completes, rows that cannot see that key are exact as usual,
+    and the next read finds the word cleared."""
+    import oracle
+    from tests import parity
+    s = synth.PrefillShape("vbad", N=512, H=8, G=2, d=64, d_idx=64, top_k=4, seed=71)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    inp["v"][300, 1, 5] = bad
     cfg = msa.config(s.H, s.G, s.d, s.d_idx, top_k=s.top_k, scale=s.scale)
     ws = torch.empty(msa.msa_workspace_size(cfg, msa.OP_PREFILL, s.N), dtype=torch.uint8,
                      device="cuda")

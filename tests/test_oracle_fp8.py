@@ -136,3 +136,55 @@ def test_quantised_selection_keeps_planted_block():
     pooled = oracle.pooled_scores_fp8(q8, np.arange(N), k8, ks, block, nb)
     ids = oracle.select_blocks(pooled, np.arange(N), block, top_k)
     assert 2 in ids[900, 0]
+
+
+def test_row_quantizer_equals_query_rows_of_index_quantizer():
+    """Per-row quantisation of the decode tensors follows the same rule as the
+    index-query rows of quantize_index_fp8 (pinned above): identical bytes."""
+    q_idx = _bf16((300, 4, 128), 21, 2.5)
+    k_idx = _bf16((300, 128), 22)
+    q_idx[7, 2] = 0
+    q8, _, _ = oracle.quantize_index_fp8(q_idx, k_idx)
+    r8, rs = oracle.quantize_rows_fp8(q_idx)
+    np.testing.assert_array_equal(r8, q8)
+    assert rs.shape == (300, 4) and rs[7, 2] == 1.0
+    # every non-zero row's largest magnitude lands on code +-448
+    dec = oracle.e4m3_decode(r8)
+    amax = np.abs(dec).max(axis=2)
+    assert np.all((amax == 448.0) | ((rs == 1.0) & (amax == 0)))
+
+
+def test_row_scaled_pooled_equals_block_scaled_when_scales_agree():
+    """With each row's scale equal to its block's, the per-row pooled score is
+    the pinned per-block one."""
+    N, block = 700, 128
+    q8, k8, ks = oracle.quantize_index_fp8(_bf16((N, 2, 128), 31), _bf16((N, 128), 32))
+    rows = np.arange(0, N, 7)
+    nb = (N + block - 1) // block
+    a = oracle.pooled_scores_fp8(q8[rows], rows, k8, ks, block, nb)
+    b = oracle.pooled_scores_fp8_rows(q8[rows], rows, k8, np.repeat(ks, block)[:N], block, nb)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_row_scaled_pooled_equals_dense_masked_max():
+    """Random codes and power-of-two row scales (every product and sum exact):
+    the pooled score equals a dense masked score matrix reduced by a library max."""
+    rng = np.random.default_rng(9)
+    N, G, block = 300, 2, 32
+    q8 = rng.integers(0, 0x7E, (N, G, 128)).astype(np.uint8) & 0xBF
+    k8 = rng.integers(0, 0x7E, (N, 128)).astype(np.uint8) & 0xBF
+    sc = (2.0 ** rng.integers(-3, 4, N)).astype(np.float32)
+    rows = np.arange(N)
+    nb = (N + block - 1) // block
+    got = oracle.pooled_scores_fp8_rows(q8, rows, k8, sc, block, nb)
+    qv = torch.from_numpy(oracle.e4m3_decode(q8))
+    kv = torch.from_numpy(oracle.e4m3_decode(k8) * sc[:, None].astype(np.float64))
+    dense = torch.einsum("tgc,sc->tgs", qv, kv)
+    vis = torch.arange(N)[None, :] <= torch.arange(N)[:, None]
+    dense = dense.masked_fill(~vis[:, None, :], -torch.inf)
+    want = dense.view(N, G, nb, block).amax(dim=3).numpy() if N % block == 0 else None
+    if want is None:
+        pad = nb * block - N
+        dense = torch.nn.functional.pad(dense, (0, pad), value=-torch.inf)
+        want = dense.view(N, G, nb, block).amax(dim=3).numpy()
+    np.testing.assert_array_equal(got, want)
