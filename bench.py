@@ -2,12 +2,15 @@
 """MSA hot-path benchmark on B200: prefill tokens/s and decode tokens/s.
 
 One step = one msa_prefill over the prefill workload (index branch, query
-lists, Main Branch, merge) plus one msa_decode step over the decode workload
-(16 sequences of 256K cached tokens and one of 1M).  Inputs are seeded
-synthetic tensors (``synth``) resident in HBM; each is larger than the 126 MB
-L2 (Q at 32K is 512 MiB, the decode caches 21 GiB), so no flush is needed
-between steps.  Kernel times come from CUDA events that the library records
-on its own stream at kernel boundaries (msa_set_phase_events).
+lists, Main Branch, merge; by default the 1M-token workload, its query axis
+processed in chunks that fit a 96 GiB workspace) plus one msa_decode step over
+the decode workload (16 sequences of 256K cached tokens and one of 1M).  The
+32K and 128K prefill workloads are then measured the same way, prefill only,
+and reported under "extra".  Inputs are seeded synthetic tensors (``synth``)
+resident in HBM; each is larger than the 126 MB L2 (Q is 512 MiB at 32K and
+16 GiB at 1M, the decode caches 21 GiB), so no flush is needed between steps.
+Kernel times come from CUDA events that the library records on its own
+stream at kernel boundaries (msa_set_phase_events).
 
 Prints exactly one JSON line on rank 0.  ``--impl reference`` times the fp64
 CPU oracle on bounded samples of the same workload instead.
@@ -36,6 +39,11 @@ import synth  # noqa: E402
 
 METRIC = "MSA prefill tokens/s & decode tokens/s on 1 B200; % of tensor/HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures, reported beside the measured fractions (the targets
+# are judged on the measured peaks)
+NOMINAL_PEAKS = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
+DEFAULT_WORKLOAD = "prefill_1m"
+DEFAULT_EXTRA = "prefill_32k,prefill_128k"
 PREFILL_PHASES = ("index_select", "block_query_lists", "main_branch", "merge")
 DECODE_PHASES = ("decode_index", "decode_select_attend")
 
@@ -75,9 +83,9 @@ def prefill_work(ids: np.ndarray, H: int, d: int, block: int = 128) -> dict:
     slots = int(valid.sum())
     pairs = slots * HG
     main_flops = 4.0 * d * HG * float(keys.sum())
-    # gathered q row (2d) + partial o (2d fp16) + lse (4) per (token, head, block)
-    main_bytes = pairs * (2 * d + 2 * d + 4.0)
-    merge_bytes = pairs * (2 * d + 4.0) + N * H * 2.0 * d + N * G * k * 4.0
+    # gathered q row (2d) + partial o (2d fp16) + its (m, l) (8) per (token, head, block)
+    main_bytes = pairs * (2 * d + 2 * d + 8.0)
+    merge_bytes = pairs * (2 * d + 8.0) + N * H * 2.0 * d + N * G * k * 4.0
     csr_bytes = 3.0 * N * G * k * 4.0
     return dict(slots=slots, pairs=pairs, main_flops=main_flops, main_bytes=main_bytes,
                 merge_bytes=merge_bytes, csr_bytes=csr_bytes,
@@ -85,11 +93,18 @@ def prefill_work(ids: np.ndarray, H: int, d: int, block: int = 128) -> dict:
 
 
 def decode_work(seq_lens, H: int, G: int, d: int, d_idx: int, ids: np.ndarray,
-                block: int = 128) -> dict:
+                block: int = 128, fp8_index: bool = False) -> dict:
+    """Bytes and FLOPs of one decode step.  The index scan reads every non-local
+    cached key once (bf16: 2 bytes a value; e4m3: 1 byte a value plus its row's
+    4-byte scale) and each sequence's G index queries; the attention reads the
+    K and V rows of the selected blocks."""
     lens = np.asarray(seq_lens, dtype=np.int64)
     nb = (lens + block - 1) // block
     scan_keys = float(((nb - 1) * block).sum())
-    idx_bytes = scan_keys * d_idx * 2.0 + len(lens) * G * d_idx * 2.0
+    if fp8_index:
+        idx_bytes = scan_keys * (d_idx + 4.0) + len(lens) * G * d_idx * 1.0
+    else:
+        idx_bytes = scan_keys * d_idx * 2.0 + len(lens) * G * d_idx * 2.0
     idx_flops = 2.0 * d_idx * G * scan_keys
     keys = 0.0
     for b, L in enumerate(lens):
@@ -214,17 +229,40 @@ def replica_rate(units_per_rank: float, ms_local: float, world: int):
 # CPU oracle timing (the baseline arm)
 # --------------------------------------------------------------------------
 
+class OracleRows:
+    """The oracle on sampled query rows of a prefill workload: the rows of q and
+    q_idx are gathered where the inputs live and copied to the host, the key
+    side (k, v, k_idx) is copied once."""
+
+    def __init__(self, inp, shape):
+        self.inp, self.shape = inp, shape
+        self.key_side = {k: inp[k].cpu() for k in ("k", "v", "k_idx")}
+        self.nb = (shape.N + shape.block - 1) // shape.block
+
+    def gather(self, rows):
+        ridx = torch.as_tensor(rows, device=self.inp["q"].device)
+        return (self.inp["q"].index_select(0, ridx).cpu(),
+                self.inp["q_idx"].index_select(0, ridx).cpu())
+
+    def run(self, rows, q_rows, qi_rows):
+        import oracle
+        sh, ks = self.shape, self.key_side
+        pooled = oracle.pooled_scores(qi_rows, rows, ks["k_idx"], sh.block, self.nb)
+        ids = oracle.select_blocks(pooled, rows, sh.block, sh.top_k)
+        return oracle.block_attention(q_rows, rows, ks["k"], ks["v"], ids, sh.scale, sh.block)
+
+
 def oracle_prefill_rate(inp, shape, budget_s: float, max_rows: int = 4096, seed: int = 0):
     """Tokens/s of the oracle over a uniform sample of query rows."""
-    import oracle
+    orc = OracleRows(inp, shape)
     rows_done, elapsed, n = 0, 0.0, 16
     rng_seed = seed
     while elapsed < budget_s and rows_done < max_rows:
         rows = synth.sample_rows(shape.N, n, seed=rng_seed)[:n]
         rng_seed += 1
+        q_rows, qi_rows = orc.gather(rows)
         t0 = time.perf_counter()
-        oracle.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
-                       block=shape.block, top_k=shape.top_k, scale=shape.scale, rows=rows)
+        orc.run(rows, q_rows, qi_rows)
         elapsed += time.perf_counter() - t0
         rows_done += len(rows)
         n = min(4 * n, max_rows - rows_done) if elapsed < budget_s / 4 else n
@@ -240,11 +278,6 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def host_inputs(shape):
-    """The same seeded inputs, drawn on the host (the oracle's arrays)."""
-    return synth.make_prefill_inputs(shape, device="cpu")
-
-
 # --------------------------------------------------------------------------
 # arms
 # --------------------------------------------------------------------------
@@ -254,15 +287,17 @@ def run_reference(args, rank, world):
         return None
     os.environ.setdefault("OMP_NUM_THREADS", str(cpu_cores()))
     shape = synth.PREFILL_CONFIGS[args.workload]
-    inp = host_inputs(shape)
-    import oracle
+    # the seeded inputs are drawn where they are cheapest to draw (the device, if
+    # any); only the sampled rows and the key side reach the oracle on the host
+    inp = synth.make_prefill_inputs(shape, device="cuda" if torch.cuda.is_available() else "cpu")
+    orc = OracleRows(inp, shape)
     rows_per_step = args.ref_rows
     step_times = []
     for i in range(args.warmup + args.steps):
         rows = synth.sample_rows(shape.N, rows_per_step, seed=1000 + i)[:rows_per_step]
+        q_rows, qi_rows = orc.gather(rows)
         t0 = time.perf_counter()
-        oracle.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
-                       block=shape.block, top_k=shape.top_k, scale=shape.scale, rows=rows)
+        orc.run(rows, q_rows, qi_rows)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             step_times.append((dt, len(rows)))
@@ -311,24 +346,205 @@ def _phase_ms(evs, n_phases):
     return [evs[i].elapsed_time(evs[i + 1]) for i in range(n_phases)]
 
 
+class KernelTable:
+    """Per-phase figures: mean event-timed ms, algorithmic work per launch, the
+    achieved rate, and its fraction of the measured and of the nominal peak."""
+
+    def __init__(self, peaks, tc_name, step_ms):
+        self.peaks, self.tc_name, self.step_ms = peaks, tc_name, step_ms
+        self.rows = {}
+
+    def add(self, name, ms_arr, bound, work, peak_scale=1.0):
+        ms = float(np.mean(ms_arr))
+        if bound == "hbm":
+            ach = work / (ms * 1e-3) / 1e9
+            peak, nominal, unit = self.peaks["hbm_gbs"], NOMINAL_PEAKS["hbm_gbs"], "GB/s"
+        else:
+            ach = work / (ms * 1e-3) / 1e12
+            peak = self.peaks[self.tc_name] * peak_scale
+            nominal, unit = NOMINAL_PEAKS["bf16_tflops"] * peak_scale, "TFLOP/s"
+        self.rows[name] = {"ms": ms, "ms_median": float(np.median(ms_arr)),
+                           "ms_min": float(np.min(ms_arr)), "bound": bound, "achieved": ach,
+                           "peak": peak, "unit": unit, "frac": ach / peak,
+                           "frac_nominal": ach / nominal, "work_per_launch": work,
+                           "share": ms / self.step_ms}
+        return self.rows[name]
+
+
+class PrefillRun:
+    """One prefill workload on the device: inputs, workspace (capped; above the
+    cap the query axis is processed in chunks) and the timed call."""
+
+    def __init__(self, msa, shape, dev, rank, args):
+        self.msa, self.shape, self.args = msa, shape, args
+        N = shape.N
+        self.cfg = msa.config(shape.H, shape.G, shape.d, shape.d_idx, top_k=shape.top_k,
+                              block=shape.block, scale=shape.scale)
+        self.inp = synth.make_prefill_inputs(shape, device=dev, seed=shape.seed + rank)
+        full_ws = msa.msa_workspace_size(self.cfg, msa.OP_PREFILL, N)
+        cap = int(args.ws_gb * (1 << 30))
+        self.ws = torch.empty(max(min(full_ws, cap), msa.msa_prefill_min_workspace(self.cfg, N)),
+                              dtype=torch.uint8, device=dev)
+        self.out = torch.empty((N, shape.H, shape.d), dtype=torch.bfloat16, device=dev)
+        self.ids = torch.empty((N, shape.G, shape.top_k), dtype=torch.int32, device=dev)
+        chunk = msa.msa_prefill_chunk_tokens(self.cfg, N, self.ws.numel(), ids_returned=True)
+        self.n_chunks = (N + chunk - 1) // chunk
+        self.quant_ms = None
+        if args.index_fp8:
+            # the quantised Index Branch takes e4m3 index tensors (a model with an
+            # 8-bit indexer emits them from its projections): quantised once here,
+            # the time reported beside the index kernel
+            qz = msa.msa_quantize_index_fp8(self.cfg, self.inp["q_idx"], self.inp["k_idx"])
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            self.q8, self.k8, self.ks = msa.msa_quantize_index_fp8(self.cfg, self.inp["q_idx"],
+                                                                   self.inp["k_idx"])
+            e1.record()
+            torch.cuda.synchronize()
+            self.quant_ms = e0.elapsed_time(e1)
+            del qz
+
+    def once(self):
+        msa, inp = self.msa, self.inp
+        if self.args.index_fp8:
+            msa.msa_prefill_fp8_index(self.cfg, inp["q"], inp["k"], inp["v"], self.q8, self.k8,
+                                      self.ks, out=self.out, ids_out=self.ids, workspace=self.ws)
+        else:
+            msa.msa_prefill(self.cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                            out=self.out, ids_out=self.ids, workspace=self.ws)
+        return msa.msa_last_launch_count()
+
+    def events(self, steps):
+        # 5 events per chunk of the query axis (phase boundaries)
+        return [[torch.cuda.Event(enable_timing=True) for _ in range(5 * self.n_chunks)]
+                for _ in range(steps)]
+
+    def report(self, pev, table: KernelTable, world):
+        """Phase times summed over the chunks of each step -> the prefill object;
+        per-phase rows go into `table`."""
+        shape, args = self.shape, self.args
+        assert self.msa.msa_get_device_error(self.ws) == 0, "device error in timed prefill"
+        nc = self.n_chunks
+        pre_ph = np.array([[sum(e[5 * c + ph].elapsed_time(e[5 * c + ph + 1]) for c in range(nc))
+                            for ph in range(4)] for e in pev])
+        value, pre_ms = replica_rate(shape.N, float(pre_ph.sum(axis=1).mean()), world)
+        pw = prefill_work(self.ids.cpu().numpy(), shape.H, shape.d, shape.block)
+        idx_f = index_flops(shape.N, shape.G, shape.d_idx, shape.block)
+        # e4m3 selection: its own dtype's peak, the measured bf16 one times the
+        # nominal e4m3 / bf16 ratio (2)
+        r = table.add("index_select", pre_ph[:, 0], "tensor", idx_f,
+                      2.0 if args.index_fp8 else 1.0)
+        if args.index_fp8:
+            r["dtype"] = "e4m3"
+            r["quantize_ms"] = self.quant_ms
+        table.add("block_query_lists", pre_ph[:, 1], "hbm", pw["csr_bytes"])
+        # the Main Branch against the tensor peak (its target); the HBM rate of its
+        # algorithmic bytes beside it
+        mb = table.add("main_branch", pre_ph[:, 2], "tensor", pw["main_flops"])
+        mb["hbm_bytes_per_launch"] = pw["main_bytes"]
+        mb["hbm_achieved_gbs"] = pw["main_bytes"] / (mb["ms"] * 1e-3) / 1e9
+        mb["hbm_frac"] = mb["hbm_achieved_gbs"] / table.peaks["hbm_gbs"]
+        table.add("merge", pre_ph[:, 3], "hbm", pw["merge_bytes"])
+        return {"value": value, "unit": "tokens/s", "ms_per_step": pre_ms, "query_chunks": nc,
+                "index_ms": float(pre_ph[:, 0].mean()),
+                "main_ms": float(pre_ph[:, 1:].sum(axis=1).mean()),
+                "index_flops": idx_f, "main_flops": pw["main_flops"],
+                "dense_flops": dense_flops(shape.N, shape.H, shape.d),
+                "msa_flops": idx_f + pw["main_flops"],
+                "selected_keys_per_query": pw["selected_keys"]}
+
+
+def _tc_peak_name(total_ms, step_ms):
+    # the sustained (power-capped) bf16 figure for long steps or regions, the burst one else
+    return "bf16_tflops_sustained" if (total_ms > 5000.0 or step_ms > 200.0) else "bf16_tflops"
+
+
+def measure_extra(msa, name, args, dev, rank, world):
+    """A prefill-only measurement of another workload (its own buffers, freed
+    before return): prefill tokens/s, per-phase kernels and clocks."""
+    shape = synth.PREFILL_CONFIGS[name]
+    run = PrefillRun(msa, shape, dev, rank, args)
+    steps = 20 if shape.N <= 65536 else 8
+    for _ in range(3):
+        run.once()
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_error(run.ws) == 0, f"device error in {name} warm-up"
+    pev = run.events(steps)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        msa.msa_set_phase_events(pev[i])
+        run.once()
+    msa.msa_set_phase_events(None)
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    total = reduce_max(t0.elapsed_time(t1), world)
+    peaks, _ = load_peaks()
+    table = KernelTable(peaks, _tc_peak_name(total, total / steps), total / steps)
+    obj = run.report(pev, table, world)
+    obj.update({"workload": name, "N": shape.N, "steps": steps, "warmup": 3,
+                "kernels": table.rows, "clocks": clocks, "tc_peak": table.tc_name})
+    del run
+    torch.cuda.empty_cache()
+    return obj
+
+
+def measure_decode_fp8(msa, dec, dcfg, dc, cu_dev, max_len, dws, dout, dids, args, world,
+                       peaks):
+    """Decode tokens/s with the e4m3 Index Branch: per-row quantised index query
+    and index-key cache; the attention reads the same bf16 K/V."""
+    q8, _ = msa.msa_quantize_rows_fp8(dec["q_idx"])
+    k8, ks = msa.msa_quantize_rows_fp8(dec["k_idx_cache"])
+
+    def once():
+        msa.msa_decode_fp8_index(dcfg, dec["q"], q8, dec["k_cache"], dec["v_cache"], k8, ks,
+                                 cu_dev, max_len, out=dout, ids_out=dids, workspace=dws)
+
+    for _ in range(3):
+        once()
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_error(dws) == 0, "device error in e4m3 decode warm-up"
+    steps = max(args.steps, 10)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        msa.msa_set_phase_events(evs[i])
+        once()
+    msa.msa_set_phase_events(None)
+    torch.cuda.synchronize()
+    barrier(world)
+    ph = np.array([_phase_ms(e, 2) for e in evs])
+    rate, ms = replica_rate(dc.B, float(ph.sum(axis=1).mean()), world)
+    dw = decode_work(dc.seq_lens, dc.H, dc.G, dc.d, dc.d_idx, dids.cpu().numpy(), dc.block,
+                     fp8_index=True)
+    table = KernelTable(peaks, "bf16_tflops", ms)
+    table.add("decode_index_fp8", ph[:, 0], "hbm", dw["idx_bytes"])
+    table.add("decode_select_attend", ph[:, 1], "hbm", dw["attn_bytes"])
+    del q8, k8, ks
+    return {"value": rate, "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "bytes_per_step": dw["bytes"],
+            "hbm_frac": dw["bytes"] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "hbm_frac_nominal": dw["bytes"] / (ms * 1e-3) / 1e9 / NOMINAL_PEAKS["hbm_gbs"],
+            "kernels": table.rows,
+            "index": "e4m3, one fp32 scale per index-key row"}
+
+
 def run_ours(args, rank, world, local):
     import block_sparse_long_branch_b200 as msa
     dev = torch.device("cuda", local)
     shape = synth.PREFILL_CONFIGS[args.workload]
     do_prefill = not args.no_prefill
     N = shape.N
-    cfg = msa.config(shape.H, shape.G, shape.d, shape.d_idx, top_k=shape.top_k,
-                     block=shape.block, scale=shape.scale)
-    if do_prefill:
-        inp = synth.make_prefill_inputs(shape, device=dev, seed=shape.seed + rank)
-        full_ws = msa.msa_workspace_size(cfg, msa.OP_PREFILL, N)
-        cap = int(args.ws_gb * (1 << 30))
-        ws = torch.empty(max(min(full_ws, cap), msa.msa_prefill_min_workspace(cfg, N)),
-                         dtype=torch.uint8, device=dev)
-        out = torch.empty((N, shape.H, shape.d), dtype=torch.bfloat16, device=dev)
-        ids = torch.empty((N, shape.G, shape.top_k), dtype=torch.int32, device=dev)
-        chunk = msa.msa_prefill_chunk_tokens(cfg, N, ws.numel(), ids_returned=True)
-        n_chunks = (N + chunk - 1) // chunk
+    run = PrefillRun(msa, shape, dev, rank, args) if do_prefill else None
+    cfg = run.cfg if run else None
 
     dc = decode_shape(args)
     dec = None
@@ -343,54 +559,26 @@ def run_ours(args, rank, world, local):
         dids = torch.empty((dc.B, dc.G, dc.top_k), dtype=torch.int32, device=dev)
         max_len = max(dc.seq_lens)
 
-    quant_ms = None
-    if do_prefill and args.index_fp8:
-        # the quantised Index Branch takes e4m3 index tensors (a model with an
-        # 8-bit indexer emits them from its projections): quantised once here,
-        # the time reported beside the index kernel
-        qz = msa.msa_quantize_index_fp8(cfg, inp["q_idx"], inp["k_idx"])
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        q8, k8, ks = msa.msa_quantize_index_fp8(cfg, inp["q_idx"], inp["k_idx"])
-        e1.record()
-        torch.cuda.synchronize()
-        quant_ms = e0.elapsed_time(e1)
-        del qz
-
-    def prefill_once():
-        if args.index_fp8:
-            msa.msa_prefill_fp8_index(cfg, inp["q"], inp["k"], inp["v"], q8, k8, ks, out=out,
-                                      ids_out=ids, workspace=ws)
-        else:
-            msa.msa_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
-                            out=out, ids_out=ids, workspace=ws)
-        return msa.msa_last_launch_count()
-
     def decode_once():
         msa.msa_decode(dcfg, dec["q"], dec["q_idx"], dec["k_cache"], dec["v_cache"],
                        dec["k_idx_cache"], cu_dev, max_len, out=dout, ids_out=dids,
                        workspace=dws)
         return msa.msa_last_launch_count()
 
-    def mk_events(n):
-        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-
     # ---- warm-up ----
     for _ in range(args.warmup):
-        if do_prefill:
-            prefill_once()
+        if run:
+            run.once()
         if dec is not None:
             decode_once()
     torch.cuda.synchronize()
-    if do_prefill:
-        assert msa.msa_get_device_error(ws) == 0, "device error after prefill warm-up"
+    if run:
+        assert msa.msa_get_device_error(run.ws) == 0, "device error after prefill warm-up"
     if dec is not None:
         assert msa.msa_get_device_error(dws) == 0, "device error after decode warm-up"
 
-    # prefill chunks: 5 events per chunk of the query axis
-    pev = [mk_events(5 * n_chunks) for _ in range(args.steps)] if do_prefill else []
-    dev_ev = [mk_events(3) for _ in range(args.steps)]
+    pev = run.events(args.steps) if run else []
+    dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     launches = 0
     barrier(world)
     torch.cuda.synchronize()
@@ -400,9 +588,9 @@ def run_ours(args, rank, world, local):
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record()
     for i in range(args.steps):
-        if do_prefill:
+        if run:
             msa.msa_set_phase_events(pev[i])
-            launches += prefill_once()
+            launches += run.once()
         if dec is not None:
             msa.msa_set_phase_events(dev_ev[i])
             launches += decode_once()
@@ -414,79 +602,47 @@ def run_ours(args, rank, world, local):
     total_ms = reduce_max(t_start.elapsed_time(t_end), world)
     step_ms = total_ms / args.steps
     peaks, peak_src = load_peaks()
-    # the sustained (power-capped) bf16 figure for long steps or regions, the burst one else
-    long_region = total_ms > 5000.0 or step_ms > 200.0
-    tc_name = "bf16_tflops_sustained" if long_region else "bf16_tflops"
-    tc_peak = peaks[tc_name]
-    kernels = {}
+    table = KernelTable(peaks, _tc_peak_name(total_ms, step_ms), step_ms)
+    kernels = table.rows
 
-    def add(name, ms_arr, bound, work, unit_is_bytes, peak_scale=1.0):
-        ms = float(np.mean(ms_arr))
-        if unit_is_bytes:
-            ach = work / (ms * 1e-3) / 1e9
-            peak, unit = peaks["hbm_gbs"], "GB/s"
-        else:
-            ach = work / (ms * 1e-3) / 1e12
-            peak, unit = tc_peak * peak_scale, "TFLOP/s"
-        kernels[name] = {"ms": ms, "ms_median": float(np.median(ms_arr)),
-                         "ms_min": float(np.min(ms_arr)), "bound": bound, "achieved": ach,
-                         "peak": peak, "unit": unit, "frac": ach / peak,
-                         "work_per_launch": work, "share": ms / step_ms}
-
-    prefill_obj, value, pre_ms = None, None, None
-    if do_prefill:
-        assert msa.msa_get_device_error(ws) == 0, "device error in timed prefill"
-        chunks_run = n_chunks
-        # per step, per phase: summed over the chunks of the query axis
-        pre_ph = np.array([[sum(e[5 * c + ph].elapsed_time(e[5 * c + ph + 1])
-                                for c in range(chunks_run)) for ph in range(4)] for e in pev])
-        value, pre_ms = replica_rate(N, float(pre_ph.sum(axis=1).mean()), world)
-        ids_np = ids.cpu().numpy()
-        pw = prefill_work(ids_np, shape.H, shape.d, shape.block)
-        idx_f = index_flops(N, shape.G, shape.d_idx, shape.block)
-        # e4m3 selection: its own dtype's peak, the measured bf16 one times the
-        # nominal e4m3 / bf16 ratio (2)
-        add("index_select", pre_ph[:, 0], "tensor", idx_f, False,
-            2.0 if args.index_fp8 else 1.0)
-        if args.index_fp8:
-            kernels["index_select"]["dtype"] = "e4m3"
-            kernels["index_select"]["quantize_ms"] = quant_ms
-        add("block_query_lists", pre_ph[:, 1], "hbm", pw["csr_bytes"], True)
-        add("main_branch", pre_ph[:, 2], "hbm", pw["main_bytes"], True)
-        kernels["main_branch"]["tensor_tflops"] = (pw["main_flops"] /
-                                                   (kernels["main_branch"]["ms"] * 1e-3) / 1e12)
-        kernels["main_branch"]["tensor_frac"] = kernels["main_branch"]["tensor_tflops"] / tc_peak
-        add("merge", pre_ph[:, 3], "hbm", pw["merge_bytes"], True)
-        prefill_obj = {"value": value, "unit": "tokens/s", "ms_per_step": pre_ms,
-                       "query_chunks": chunks_run, "dense_flops": dense_flops(N, shape.H, shape.d),
-                       "msa_flops": idx_f + pw["main_flops"],
-                       "selected_keys_per_query": pw["selected_keys"]}
+    prefill_obj, value = None, None
+    if run:
+        prefill_obj = run.report(pev, table, world)
+        value = prefill_obj["value"]
     decode_obj = None
     if dec is not None:
         dec_ph = np.array([_phase_ms(e, 2) for e in dev_ev])
         dec_rate, dec_ms = replica_rate(dc.B, float(dec_ph.sum(axis=1).mean()), world)
         dw = decode_work(dc.seq_lens, dc.H, dc.G, dc.d, dc.d_idx, dids.cpu().numpy(), dc.block)
-        add("decode_index", dec_ph[:, 0], "hbm", dw["idx_bytes"], True)
-        add("decode_select_attend", dec_ph[:, 1], "hbm", dw["attn_bytes"], True)
+        table.add("decode_index", dec_ph[:, 0], "hbm", dw["idx_bytes"])
+        table.add("decode_select_attend", dec_ph[:, 1], "hbm", dw["attn_bytes"])
         dstep_bytes = dw["bytes"]
         decode_obj = {"value": dec_rate, "unit": "tokens/s",
                       "ms_per_step": dec_ms,
                       "hbm_frac": dstep_bytes / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                      "hbm_frac_nominal": dstep_bytes / (dec_ms * 1e-3) / 1e9 /
+                      NOMINAL_PEAKS["hbm_gbs"],
                       "bytes_per_step": dstep_bytes}
         if value is None:
             value = decode_obj["value"]
+        # the same step with the e4m3 Index Branch over an e4m3 index-key cache
+        # (quantised once, before timing, as a model's projections would emit it)
+        decode_obj["fp8_index"] = measure_decode_fp8(msa, dec, dcfg, dc, cu_dev, max_len, dws,
+                                                     dout, dids, args, world, peaks)
     dominant = max(kernels, key=lambda k: kernels[k]["ms"])
     dk = kernels[dominant]
     roofline = {"kernel": dominant, "bound": dk["bound"], "achieved": dk["achieved"],
                 "peak": dk["peak"], "unit": dk["unit"], "frac": dk["frac"],
-                "traffic": traffic_for(dominant, shape.name if do_prefill else None),
+                "frac_nominal": dk["frac_nominal"],
+                "traffic": traffic_for(dominant, shape.name if run else None),
                 "peak_source": f"{peak_src} "
-                f"({'hbm_gbs' if dk['unit'] == 'GB/s' else tc_name})"}
+                f"({'hbm_gbs' if dk['unit'] == 'GB/s' else table.tc_name})"}
 
     # ---- end to end through the public API with host buffers ----
     e2e = None if (args.no_e2e or args.index_fp8) else run_e2e(
-        args, msa, cfg, shape, inp if do_prefill else None, ws if do_prefill else None, dev, dec,
-        dcfg if dec is not None else None, dws if dec is not None else None, world)
+        args, msa, cfg, shape, run.inp if run else None, run.ws if run else None,
+        run.out if run else None, dev, dec, dcfg if dec is not None else None,
+        dws if dec is not None else None, world)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -496,14 +652,21 @@ def run_ours(args, rank, world, local):
         "prefill": prefill_obj, "decode": decode_obj, "roofline": roofline, "kernels": kernels,
         "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
     }
-    if world == 1 and rank == 0 and do_prefill and not args.no_cpu_baseline:
+    if world == 1 and rank == 0 and run and not args.no_cpu_baseline:
         os.environ.setdefault("OMP_NUM_THREADS", str(cpu_cores()))
-        hinp = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
-        rate, rows, el = oracle_prefill_rate(hinp, shape, args.cpu_budget)
+        rate, rows, el = oracle_prefill_rate(run.inp, shape, args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s",
                                 "cores": int(os.environ["OMP_NUM_THREADS"]), "kind": "oracle",
                                 "sample": f"{rows} query rows uniform over the {shape.name} "
                                           f"positions, {el:.1f} s of oracle time"}
+    extras = [x for x in (args.extra or "").split(",") if x and x != "none" and x != shape.name]
+    if extras and world == 1:
+        # the other prefill workloads, measured after this one's buffers are freed
+        del run
+        if dec is not None:
+            del dec, dws, dout, dids
+        torch.cuda.empty_cache()
+        line["extra"] = {x: measure_extra(msa, x, args, dev, rank, world) for x in extras}
     return line
 
 
@@ -529,23 +692,61 @@ def traffic_for(kernel: str, workload):
     return ent.get("bytes_per_launch") if h == ent.get("source_sha") else None
 
 
-def run_e2e(args, msa, cfg, shape, inp, ws, dev, dec, dcfg, dws, world):
+def run_e2e(args, msa, cfg, shape, inp, ws, out, dev, dec, dcfg, dws, world):
     """Host (pinned) inputs -> device -> msa_prefill -> host output, every step.
 
-    Three streams overlap consecutive steps: step i's kernels run while step
-    i+1's inputs are copied in and step i-1's output is copied out.  Inputs and
-    outputs are double-buffered on both sides; each step still moves its full
-    inputs host->device and its full output device->host inside the timed
-    region.
+    Up to 256K tokens, three streams overlap consecutive steps: step i's
+    kernels run while step i+1's inputs are copied in and step i-1's output is
+    copied out; inputs and outputs are double-buffered on both sides.  Beyond
+    that (the 1M workload: 22 GB in and 16 GB out per step) the steps run one
+    after another on one stream into the bench's own device buffers: copy in,
+    prefill, copy out.  Either way each step moves its full inputs
+    host->device and its full output device->host inside the timed region.
     """
     res = {}
     if inp is not None:
-        res = _e2e_prefill(args, msa, cfg, shape, inp, ws, dev, world)
+        if shape.N > (1 << 18):
+            res = _e2e_prefill_serial(args, msa, cfg, shape, inp, ws, out, world)
+        else:
+            res = _e2e_prefill(args, msa, cfg, shape, inp, ws, dev, world)
     if dec is not None:
         res["decode"] = _e2e_decode(args, msa, dec, dcfg, dws, dev, world)
         if inp is None:
             res.update({k: v for k, v in res["decode"].items()})
     return res
+
+
+def _e2e_prefill_serial(args, msa, cfg, shape, inp, ws, out, world):
+    keys = ("q", "k", "v", "q_idx", "k_idx")
+    host = {k: torch.empty_like(inp[k], device="cpu").pin_memory() for k in keys}
+    for k in keys:
+        host[k].copy_(inp[k])
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+    d2h = out_h.numel() * out_h.element_size()
+    steps = max(2, min(args.steps, 3))
+
+    def step():
+        for k in keys:
+            inp[k].copy_(host[k], non_blocking=True)
+        msa.msa_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], out=out,
+                        workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = reduce_max(a.elapsed_time(b) / steps, world)
+    del host, out_h
+    return {"value": world * shape.N / (ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms,
+            "steps": steps, "pipelined": "no: copy in, prefill, copy out on one stream"}
 
 
 def _e2e_prefill(args, msa, cfg, shape, inp, ws, dev, world):
@@ -717,10 +918,14 @@ def run_varlen(args, rank, world, local):
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 10 for the 1M workload, 20 otherwise)")
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="prefill_32k", choices=sorted(synth.PREFILL_CONFIGS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.PREFILL_CONFIGS))
+    ap.add_argument("--extra", default=DEFAULT_EXTRA,
+                    help="comma-separated prefill workloads measured after the main one "
+                         "(prefill only, own buffers, one GPU); 'none' to skip")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
                     help="time only the decode step (profiling)")
@@ -741,6 +946,8 @@ def parse_args(argv=None):
                          "groups, d 128): one msa_prefill_varlen pass vs one msa_prefill "
                          "per sequence")
     args = ap.parse_args(argv)
+    if args.steps is None:
+        args.steps = 10 if synth.PREFILL_CONFIGS[args.workload].N > (1 << 18) else 20
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
     return args

@@ -44,8 +44,8 @@ def test_prefill_work_matches_a_per_slot_count():
                     keys += sum(1 for s in range(128 * j, 128 * j + 128) if s <= t)
     assert w["slots"] == slots and w["pairs"] == slots * HG
     assert w["main_flops"] == 4.0 * d * HG * keys          # QK^T and PV per visible key
-    assert w["main_bytes"] == slots * HG * (2 * d + 2 * d + 4)
-    assert w["merge_bytes"] == slots * HG * (2 * d + 4) + N * H * 2 * d + N * G * k * 4
+    assert w["main_bytes"] == slots * HG * (2 * d + 2 * d + 8)
+    assert w["merge_bytes"] == slots * HG * (2 * d + 8) + N * H * 2 * d + N * G * k * 4
     assert w["selected_keys"] == keys / (N * G)
 
 
@@ -68,3 +68,18 @@ def test_decode_work_counts_scan_and_selected_keys():
                 keys += sum(1 for s in range(128 * j, 128 * j + 128) if s < L)
     assert w["attn_bytes"] == keys * d * 2 * 2
     assert w["attn_flops"] == 4.0 * d * (H // G) * keys
+
+
+def test_decode_work_e4m3_index_bytes():
+    """e4m3 index cache: one byte per index value plus the row's 4-byte scale per
+    scanned key, one byte per index-query value; the attention bytes unchanged."""
+    lens = [300, 129, 1000]
+    G, H, d, di, k = 2, 8, 64, 128, 4
+    ids = np.full((len(lens), G, k), -1, np.int32)
+    ids[:, :, 0] = 0
+    w8 = bench.decode_work(lens, H, G, d, di, ids, fp8_index=True)
+    w16 = bench.decode_work(lens, H, G, d, di, ids)
+    scan = sum(128 * ((L + 127) // 128 - 1) for L in lens)
+    assert w8["idx_bytes"] == scan * (di + 4) + len(lens) * G * di
+    assert w8["attn_bytes"] == w16["attn_bytes"]
+    assert w8["bytes"] == w8["idx_bytes"] + w8["attn_bytes"]
