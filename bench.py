@@ -915,6 +915,59 @@ def run_varlen(args, rank, world, local):
             "per_sequence_ms": ms_seq, "speedup_vs_per_sequence": ms_seq / ms_one}
 
 
+def run_phase(args, rank, world, local):
+    """Only one phase of the prefill, on the workload's tensors: the Index Branch
+    selection (msa_select_topk) or the query-list build (msa_build_block_query_lists
+    on that selection).  For profiling one kernel on a small device footprint."""
+    import block_sparse_long_branch_b200 as msa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    shape = synth.PREFILL_CONFIGS[args.workload]
+    inp = synth.make_prefill_inputs(shape, device=dev, seed=shape.seed + rank)
+    for k in ("q", "k", "v"):
+        del inp[k]
+    torch.cuda.empty_cache()
+    cfg = msa.config(shape.H, shape.G, shape.d, shape.d_idx, top_k=shape.top_k,
+                     block=shape.block, scale=shape.scale)
+    N = shape.N
+    ids = torch.empty((N, shape.G, shape.top_k), dtype=torch.int32, device=dev)
+    sws = torch.empty(msa.msa_workspace_size(cfg, msa.OP_SELECT_TOPK, N), dtype=torch.uint8,
+                      device=dev)
+    lws = torch.empty(msa.msa_workspace_size(cfg, msa.OP_BLOCK_QUERY_LISTS, N), dtype=torch.uint8,
+                      device=dev)
+    msa.msa_select_topk(cfg, inp["q_idx"], inp["k_idx"], ids=ids, workspace=sws)
+
+    def once():
+        if args.phase == "select":
+            msa.msa_select_topk(cfg, inp["q_idx"], inp["k_idx"], ids=ids, workspace=sws)
+        else:
+            msa.msa_build_block_query_lists(cfg, ids, workspace=lws)
+
+    for _ in range(args.warmup):
+        once()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        once()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = reduce_max(e0.elapsed_time(e1), world) / args.steps
+    peaks, _ = load_peaks()
+    if args.phase == "select":
+        work, unit, peak = index_flops(N, shape.G, shape.d_idx, shape.block) / (ms * 1e-3) / 1e12, \
+            "TFLOP/s", peaks["bf16_tflops"]
+    else:
+        work, unit, peak = 3.0 * N * shape.G * shape.top_k * 4.0 / (ms * 1e-3) / 1e9, "GB/s", \
+            peaks["hbm_gbs"]
+    return {"metric": f"MSA {args.phase} phase alone", "value": world * N / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": {"workload": shape.name},
+            "achieved": work, "achieved_unit": unit, "frac": work / peak}
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -941,6 +994,9 @@ def parse_args(argv=None):
                     help="cap on the prefill workspace; above it the query axis is chunked")
     ap.add_argument("--ref-rows", type=int, default=32,
                     help="query rows per step in the reference arm")
+    ap.add_argument("--phase", choices=("select", "lists"),
+                    help="time only the Index Branch selection or only the query-list build "
+                         "on the workload's index tensors (profiling)")
     ap.add_argument("--varlen", metavar="BxL",
                     help="time only a packed batch of B sequences of L tokens (64 heads, 8 "
                          "groups, d 128): one msa_prefill_varlen pass vs one msa_prefill "
@@ -963,6 +1019,8 @@ def main(argv=None):
             line = run_reference(args, rank, world)
         elif args.varlen:
             line = run_varlen(args, rank, world, local)
+        elif args.phase:
+            line = run_phase(args, rank, world, local)
         else:
             line = run_ours(args, rank, world, local)
         if rank == 0 and line is not None:

@@ -10,11 +10,11 @@
 //   2. scan    : exclusive prefix over that table (flattened g, j, tile), so
 //                the entry gives where tile `tile`'s hits on (g, j) start
 //   3. row_ptr : row_ptr[g*nb+j] = scanned[(g*nb+j)*ntiles]
-//   4. scatter : one warp per (tile, group) copies its tile's keys and its
-//                start offsets into shared memory, then walks its hits in
-//                (t, slot) order; equal keys inside a 32-hit batch are ranked
-//                with match.any, and the shared-memory offset of a key
-//                advances by its batch count
+//   4. scatter : one warp per (tile, set of groups) copies its tile's keys and
+//                their start offsets into shared memory, then walks the rows
+//                in t order, one row of every group of the set per step; the
+//                hits of one step never share a key, so each advances its
+//                key's offset by one
 //   5. units   : one CTA: per list, the number of Main Branch work units, their
 //                exclusive prefix and the unit table
 // HBM-bound integer work: each id is read twice, each entry written once.
@@ -155,50 +155,58 @@ __global__ void csr_rowptr_kernel(const int32_t* __restrict__ scanned, int64_t n
   if (x == n_lists) row_ptr[x] = scanned[n_lists * ntiles - 1] + *last_count;
 }
 
-// One warp per (tile, group).  The tile's list keys are first copied to
-// shared memory with independent, coalesced loads, so the ranking loop below
-// only waits on shared memory.
+// One warp per (tile, group set): the set is GPW = 32 / top_k groups (one when
+// top_k > 16).  A row's ids are distinct within a group and different groups
+// key different lists, so the GPW * top_k hits of one row never share a key:
+// each lane reads its key's next free entry, writes there and advances it,
+// with no ranking among the lanes; rows are walked in order, so every list
+// stays in t order.  The tile's keys are first copied to shared memory with
+// independent loads, and so are the start offsets of every key of the set's
+// groups (the slice of nb keys given by s0).
 __global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restrict__ ids,
                                                          int64_t row_begin, int64_t rows,
                                                          int32_t G, int32_t top_k, int64_t nb,
                                                          int32_t ntiles, int32_t bins,
+                                                         int32_t gpw,
                                                          const int32_t* __restrict__ scanned,
                                                          const int32_t* __restrict__ row_base,
                                                          int32_t* __restrict__ entries) {
   extern __shared__ int32_t sm[];
-  int32_t* run = sm;          // [bins]: next free entry of each key of the slice
-  int32_t* keys = sm + bins;  // [kTileTok * top_k]: the tile's keys of group g
-  const int tile = blockIdx.x, g = blockIdx.y;
+  int32_t* run = sm;                 // [gpw][bins]: next free entry of each key of the slice
+  int32_t* keys = sm + gpw * bins;   // [kTileTok][gpw * top_k]: the tile's keys, by row
+  const int tile = blockIdx.x, g0 = blockIdx.y * gpw;
   const int lane = threadIdx.x;
   const int64_t r0 = (int64_t)tile * kTileTok;
   const int64_t r1 = min(rows, r0 + kTileTok);
-  const int n_el = (int)((r1 - r0) * top_k);
-  for (int e = lane; e < n_el; e += 32) {
-    const int64_t row = r0 + e / top_k;
-    keys[e] = list_key(row_base, row, __ldg(ids + (row * G + g) * top_k + e % top_k));
+  const int nrows = (int)(r1 - r0);
+  const int per_row = gpw * top_k;  // hits of one row handled by one lane each (<= 32)
+  const int ngrp = min(gpw, G - g0);
+  for (int e = lane; e < nrows * per_row; e += 32) {
+    const int rr = e / per_row, c = e - rr * per_row;
+    const int gi = c / top_k, r = c - gi * top_k;
+    const int64_t row = r0 + rr;
+    keys[e] = gi < ngrp ? list_key(row_base, row, __ldg(ids + (row * G + g0 + gi) * top_k + r))
+                        : -1;
   }
-  const unsigned lt_mask = (1u << lane) - 1u;
+  const bool active = lane < per_row;
+  const int gi = active ? lane / top_k : 0;
+  const int r = active ? lane - gi * top_k : 0;
   for (int64_t s0 = 0; s0 < nb; s0 += kBinSlice) {
     const int width = (int)min64(kBinSlice, nb - s0);
-    // where this tile's hits on each key of the slice start
-    for (int i = lane; i < width; i += 32)
-      run[i] = __ldg(scanned + ((int64_t)g * nb + s0 + i) * ntiles + tile);
+    // where this tile's hits on each key of the slice start, per group of the set
+    for (int i = lane; i < ngrp * width; i += 32) {
+      const int gg = i / width, x = i - gg * width;
+      run[gg * bins + x] = __ldg(scanned + ((int64_t)(g0 + gg) * nb + s0 + x) * ntiles + tile);
+    }
     __syncwarp();
-    for (int e0 = 0; e0 < n_el; e0 += 32) {
-      const int e = e0 + lane;
-      const int32_t j = e < n_el ? keys[e] : -1;
-      const bool mine = j >= s0 && j < s0 + width;
-      const int key = mine ? (int)(j - s0) : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, key);
-      int32_t base = 0;
-      if (mine) {
-        base = run[key];
-        const int rank = __popc(peers & lt_mask);
-        const int64_t row = r0 + e / top_k;
-        entries[(int64_t)base + rank] = (int32_t)(((row_begin + row) << 5) | (e % top_k));
+    for (int rr = 0; rr < nrows; ++rr) {
+      const int32_t j = active ? keys[rr * per_row + lane] : -1;
+      if (j >= s0 && j < s0 + width) {
+        int32_t* slot = run + gi * bins + (int)(j - s0);
+        const int32_t pos = *slot;
+        entries[pos] = (int32_t)(((row_begin + r0 + rr) << 5) | r);
+        *slot = pos + 1;
       }
-      __syncwarp();
-      if (mine && (peers & lt_mask) == 0) run[key] = base + __popc(peers);
       __syncwarp();
     }
   }
@@ -350,7 +358,14 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
 
   dim3 grid((unsigned)ntiles, (unsigned)p.G);
   const size_t bin_bytes = (size_t)bins * sizeof(int32_t);
-  const size_t scatter_bytes = bin_bytes + (size_t)kTileTok * p.top_k * sizeof(int32_t);
+  // groups per scatter warp: one row's hits of gpw groups fill at most 32 lanes,
+  // and their offsets and keys fit 200 KiB of shared memory
+  int gpw = p.top_k <= 16 ? (int)min64(32 / p.top_k, p.G) : 1;
+  auto scatter_smem = [&](int w) {
+    return (size_t)w * bin_bytes + (size_t)kTileTok * w * p.top_k * sizeof(int32_t);
+  };
+  while (gpw > 1 && scatter_smem(gpw) > 200 * 1024) --gpw;
+  const size_t scatter_bytes = scatter_smem(gpw);
   if (bin_bytes > 48 * 1024 &&
       (e = cudaFuncSetAttribute(csr_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)bin_bytes)) != cudaSuccess)
@@ -369,9 +384,10 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
   csr_rowptr_kernel<<<(unsigned)((n_lists + 1 + 255) / 256), 256, 0, s>>>(
       cnt, n_lists, (int32_t)ntiles, last, p.row_ptr);
   ++*launches;
-  csr_scatter_kernel<<<grid, 32, scatter_bytes, s>>>(p.ids, p.row_begin, p.rows, p.G, p.top_k,
-                                                     p.nb, (int32_t)ntiles, bins, cnt,
-                                                     p.row_base, p.entries);
+  dim3 sgrid((unsigned)ntiles, (unsigned)((p.G + gpw - 1) / gpw));
+  csr_scatter_kernel<<<sgrid, 32, scatter_bytes, s>>>(p.ids, p.row_begin, p.rows, p.G,
+                                                      p.top_k, p.nb, (int32_t)ntiles, bins, gpw,
+                                                      cnt, p.row_base, p.entries);
   ++*launches;
   if (p.unit_ptr) {
     units_kernel<<<1, kUnitThreads, 0, s>>>(p.row_ptr, n_lists, p.nb,
