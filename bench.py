@@ -671,8 +671,8 @@ def run_ours(args, rank, world, local):
 
 
 def traffic_for(kernel: str, workload):
-    """DRAM bytes per launch from a committed ncu summary, if it is current and
-    was taken on this workload (null otherwise)."""
+    """DRAM bytes of one phase from a committed ncu summary, if it was captured on
+    this workload and the kernel source is unchanged since (null otherwise)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -680,7 +680,7 @@ def traffic_for(kernel: str, workload):
     except (OSError, ValueError):
         return None
     ent = table.get(kernel)
-    if not ent or table.get("workload") != workload:
+    if not ent or ent.get("workload") != workload:
         return None
     src = os.path.join(ROOT, "block_sparse_long_branch_b200", "csrc", ent.get("source", ""))
     try:
@@ -689,7 +689,7 @@ def traffic_for(kernel: str, workload):
             h = hashlib.sha256(f.read()).hexdigest()[:16]
     except OSError:
         return None
-    return ent.get("bytes_per_launch") if h == ent.get("source_sha") else None
+    return ent.get("bytes_per_phase") if h == ent.get("source_sha") else None
 
 
 def run_e2e(args, msa, cfg, shape, inp, ws, out, dev, dec, dcfg, dws, world):

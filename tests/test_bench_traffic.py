@@ -16,12 +16,14 @@ def _table():
 
 def test_traffic_only_for_the_captured_workload():
     t = _table()
-    ent = t["main_branch"]
-    src = os.path.join(ROOT, "block_sparse_long_branch_b200", "csrc", ent["source"])
-    with open(src, "rb") as f:
-        current = hashlib.sha256(f.read()).hexdigest()[:16] == ent["source_sha"]
-    got = bench.traffic_for("main_branch", t["workload"])
-    assert got == (ent["bytes_per_launch"] if current else None)
-    assert bench.traffic_for("main_branch", "prefill_1m") is None
-    assert bench.traffic_for("main_branch", None) is None
-    assert bench.traffic_for("decode_index", t["workload"]) is None
+    for kernel in ("index_select", "main_branch"):
+        ent = t[kernel]
+        src = os.path.join(ROOT, "block_sparse_long_branch_b200", "csrc", ent["source"])
+        with open(src, "rb") as f:
+            current = hashlib.sha256(f.read()).hexdigest()[:16] == ent["source_sha"]
+        assert ent["bytes_per_phase"] == ent["read"] + ent["write"]
+        got = bench.traffic_for(kernel, ent["workload"])
+        assert got == (ent["bytes_per_phase"] if current else None)
+        assert bench.traffic_for(kernel, "prefill_tiny_other") is None
+        assert bench.traffic_for(kernel, None) is None
+    assert bench.traffic_for("decode_index", t["index_select"]["workload"]) is None
