@@ -4,19 +4,19 @@
 // queries that hit a block are gathered; CSDN M3 write-up, section "MiniMax
 // Sparse Attention（MSA）").
 //
-// Deterministic stable counting sort on the key (g, j), in t order:
-//   1. hist    : per tile of kTileTok query rows and per group, a shared-memory
-//                histogram over the key blocks -> cnt[(g*nb + j)*ntiles + tile]
-//   2. scan    : exclusive prefix over that table (flattened g, j, tile), so
-//                the entry gives where tile `tile`'s hits on (g, j) start
-//   3. row_ptr : row_ptr[g*nb+j] = scanned[(g*nb+j)*ntiles]
-//   4. scatter : one warp per (tile, set of groups) copies its tile's keys and
-//                their start offsets into shared memory, then walks the rows
-//                in t order, one row of every group of the set per step; the
-//                hits of one step never share a key, so each advances its
-//                key's offset by one
-//   5. units   : one CTA: per list, the number of Main Branch work units, their
-//                exclusive prefix and the unit table
+// Deterministic stable counting sort on the key (g, j), in t order, over
+// parts of R query rows (R grows with nb so that the (part, list) count table
+// stays at most half the size of the ids):
+//   1. count   : per part and group, a shared-memory histogram over the key
+//                blocks -> cnt[part][g*nb + j] (coalesced) and the list totals
+//                (atomics); the last CTA scans the totals into row_ptr and
+//                cuts the lists into Main Branch work units
+//   2. colscan : the table scanned in (list, part) order, in place, from
+//                row_ptr: where each part's hits on each list start
+//   3. scatter : one warp per (part, set of groups) loads its part's start
+//                offsets, then walks the rows in t order, one row of every
+//                group of the set per step; the hits of one step never share
+//                a key, so each advances its key's offset by one
 // HBM-bound integer work: each id is read twice, each entry written once.
 //
 // For a batch of packed sequences the ids are local to each sequence; the key
@@ -30,11 +30,10 @@
 namespace msa {
 namespace {
 
-constexpr int kTileTok = 256;      // query rows per histogram tile
-constexpr int kBinSlice = 16384;   // shared-memory bins per pass (64 KiB)
-constexpr int kScanThreads = 1024;
-constexpr int kScanPer = 4;
-constexpr int kScanChunk = kScanThreads * kScanPer;
+constexpr int kBinSlice = 16384;  // shared-memory bins per pass (64 KiB)
+constexpr int kCountThreads = 512;
+constexpr int kScanWarps = 32;    // column scan: 32 warps over the parts of 32 lists
+constexpr int kKeyRows = 64;      // rows of keys a scatter warp stages at a time
 
 // Packed sequences: ids are local to each sequence and row_base[row] (the
 // global number of the row's sequence's first block) turns them into the list
@@ -43,38 +42,6 @@ __device__ __forceinline__ int32_t list_key(const int32_t* row_base, int64_t row
   return (row_base && j >= 0) ? __ldg(row_base + row) + j : j;
 }
 
-__global__ void __launch_bounds__(256) csr_hist_kernel(const int32_t* __restrict__ ids, int64_t rows,
-                                                       int32_t G, int32_t top_k, int64_t nb,
-                                                       int32_t ntiles, int32_t* __restrict__ cnt,
-                                                       const int32_t* __restrict__ row_base,
-                                                       uint32_t* err) {
-  extern __shared__ int32_t bins[];
-  const int tile = blockIdx.x, g = blockIdx.y;
-  const int64_t r0 = (int64_t)tile * kTileTok;
-  const int64_t r1 = min(rows, r0 + kTileTok);
-  const int64_t n_el = (r1 - r0) * top_k;
-  for (int64_t s0 = 0; s0 < nb; s0 += kBinSlice) {
-    const int width = (int)min64(kBinSlice, nb - s0);
-    for (int i = threadIdx.x; i < width; i += blockDim.x) bins[i] = 0;
-    __syncthreads();
-    for (int64_t e = threadIdx.x; e < n_el; e += blockDim.x) {
-      const int64_t row = r0 + e / top_k;
-      const int r = (int)(e % top_k);
-      const int32_t j = list_key(row_base, row, ids[(row * G + g) * top_k + r]);
-      if (j < -1 || j >= nb) {
-        if (s0 == 0) record_error(err, kDevBadIndex);
-        continue;
-      }
-      if (j >= s0 && j < s0 + width) atomicAdd(&bins[j - s0], 1);
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < width; i += blockDim.x)
-      cnt[((int64_t)g * nb + s0 + i) * ntiles + tile] = bins[i];
-    __syncthreads();
-  }
-}
-
-// ---- exclusive scan (int32), chunk of 4096 per CTA --------------------------
 __device__ __forceinline__ int32_t warp_incl_scan(int32_t x) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -84,167 +51,190 @@ __device__ __forceinline__ int32_t warp_incl_scan(int32_t x) {
   return x;
 }
 
-__global__ void __launch_bounds__(kScanThreads) scan_chunks_kernel(int32_t* __restrict__ data,
-                                                                   int64_t n,
-                                                                   int32_t* __restrict__ sums) {
-  __shared__ int32_t warp_tot[32];
-  const int64_t base = (int64_t)blockIdx.x * kScanChunk + (int64_t)threadIdx.x * kScanPer;
-  int32_t v[kScanPer];
-  int32_t local = 0;
-#pragma unroll
-  for (int i = 0; i < kScanPer; ++i) {
-    v[i] = (base + i < n) ? data[base + i] : 0;
-    local += v[i];
+struct ListTail {
+  int32_t* row_ptr;    // [n_lists + 1]
+  int32_t per_unit;    // entries per Main Branch work unit
+  int32_t* unit_ptr;   // optional: [n_lists + 1] exclusive prefix of the unit counts
+  int4* unit_desc;     // {g, j, first entry, end entry} of every unit
+};
+
+// row_ptr = the exclusive prefix of the per-list totals and, optionally, the
+// Main Branch work units (each list cut into runs of at most per_unit
+// entries).  One CTA: each thread takes a contiguous range of lists, the CTA
+// scans the per-thread sums, and each thread fills its range.
+__device__ void list_prefix(const int32_t* tot, int64_t n_lists, int64_t nb, const ListTail& t) {
+  __shared__ int32_t wt_e[32], wt_u[32];
+  const int nt = blockDim.x, tid = threadIdx.x, w = tid >> 5, l = tid & 31, nw = nt >> 5;
+  const int64_t per = (n_lists + nt - 1) / nt;
+  const int64_t x0 = min64((int64_t)tid * per, n_lists), x1 = min64(x0 + per, n_lists);
+  const int32_t pu = t.per_unit;
+  int32_t se = 0, su = 0;
+  for (int64_t x = x0; x < x1; ++x) {
+    const int32_t c = __ldcg(tot + x);
+    se += c;
+    su += (c + pu - 1) / pu;
   }
-  const int32_t incl = warp_incl_scan(local);
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  if (l == 31) warp_tot[w] = incl;
+  const int32_t ie = warp_incl_scan(se), iu = warp_incl_scan(su);
+  if (l == 31) wt_e[w] = ie, wt_u[w] = iu;
   __syncthreads();
   if (w == 0) {
-    const int32_t t = warp_tot[l];
-    const int32_t ti = warp_incl_scan(t);
-    warp_tot[l] = ti - t;
-    if (l == 31 && sums) sums[blockIdx.x] = ti;
+    const int32_t te = l < nw ? wt_e[l] : 0, tu = l < nw ? wt_u[l] : 0;
+    const int32_t je = warp_incl_scan(te), ju = warp_incl_scan(tu);
+    if (l < nw) wt_e[l] = je - te, wt_u[l] = ju - tu;
   }
   __syncthreads();
-  int32_t run = warp_tot[w] + incl - local;
-#pragma unroll
-  for (int i = 0; i < kScanPer; ++i) {
-    if (base + i < n) data[base + i] = run;
-    run += v[i];
+  int32_t e = wt_e[w] + ie - se, u = wt_u[w] + iu - su;
+  for (int64_t x = x0; x < x1; ++x) {
+    const int32_t c = __ldcg(tot + x);
+    t.row_ptr[x] = e;
+    if (t.unit_ptr) {
+      t.unit_ptr[x] = u;
+      const int g = (int)(x / nb), j = (int)(x - (int64_t)g * nb);
+      for (int32_t e0 = e; e0 < e + c; e0 += pu, ++u)
+        t.unit_desc[u] = make_int4(g, j, e0, min(e + c, e0 + pu));
+    }
+    e += c;
+  }
+  if (tid == nt - 1) {  // its range is the last (possibly empty): e and u are the totals
+    t.row_ptr[n_lists] = e;
+    if (t.unit_ptr) t.unit_ptr[n_lists] = u;
   }
 }
 
-__global__ void add_offsets_kernel(int32_t* __restrict__ data, int64_t n,
-                                   const int32_t* __restrict__ offs) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) data[i] += offs[i / kScanChunk];
-}
-
-size_t scan_scratch_elems(int64_t n) {
-  size_t s = 0;
-  while (n > kScanChunk) {
-    n = (n + kScanChunk - 1) / kScanChunk;
-    s += (size_t)n;
+// 1. Per part of R query rows and per group: a shared-memory histogram of the
+// part's hits over the key blocks, written as cnt[part][g*nb + j] (contiguous
+// per part) and added to the list totals tot[g*nb + j].  The last CTA to
+// finish (a ticket) computes row_ptr and the work units from the totals.
+__global__ void __launch_bounds__(kCountThreads)
+    csr_count_kernel(const int32_t* __restrict__ ids, int64_t rows, int32_t G, int32_t top_k,
+                     int64_t nb, int32_t R, int32_t* __restrict__ cnt, int32_t* __restrict__ tot,
+                     int32_t* __restrict__ ticket, const int32_t* __restrict__ row_base,
+                     uint32_t* err, ListTail tail) {
+  extern __shared__ int32_t bins[];
+  __shared__ int last;
+  const int part = blockIdx.x, g = blockIdx.y;
+  const int64_t K = (int64_t)G * nb;
+  const int64_t r0 = (int64_t)part * R;
+  const int64_t r1 = min64(rows, r0 + R);
+  const int64_t n_el = (r1 - r0) * top_k;
+  int32_t* crow = cnt + (int64_t)part * K + (int64_t)g * nb;
+  for (int64_t s0 = 0; s0 < nb; s0 += kBinSlice) {
+    const int width = (int)min64(kBinSlice, nb - s0);
+    for (int i = threadIdx.x; i < width; i += blockDim.x) bins[i] = 0;
+    __syncthreads();
+    for (int64_t e = threadIdx.x; e < n_el; e += blockDim.x) {
+      const int64_t row = r0 + e / top_k;
+      const int r = (int)(e % top_k);
+      const int32_t j = list_key(row_base, row, __ldg(ids + (row * G + g) * top_k + r));
+      if (j < -1 || j >= nb) {
+        if (s0 == 0) record_error(err, kDevBadIndex);
+        continue;
+      }
+      if (j >= s0 && j < s0 + width) atomicAdd(&bins[j - s0], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < width; i += blockDim.x) {
+      const int32_t c = bins[i];
+      crow[s0 + i] = c;
+      if (c) atomicAdd(tot + (int64_t)g * nb + s0 + i, c);
+    }
+    __syncthreads();
   }
-  return s + 1;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(ticket, 1) == (int)(gridDim.x * gridDim.y) - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  list_prefix(tot, K, nb, tail);
 }
 
-// In-place exclusive scan of data[0..n); `tmp` holds scan_scratch_elems(n).
-cudaError_t exclusive_scan(int32_t* data, int64_t n, int32_t* tmp, cudaStream_t s, int* launches) {
-  if (n <= 0) return cudaSuccess;
-  const int64_t nch = (n + kScanChunk - 1) / kScanChunk;
-  scan_chunks_kernel<<<(unsigned)nch, kScanThreads, 0, s>>>(data, n, nch > 1 ? tmp : nullptr);
-  ++*launches;
-  if (nch > 1) {
-    cudaError_t e = exclusive_scan(tmp, nch, tmp + nch, s, launches);
-    if (e != cudaSuccess) return e;
-    add_offsets_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(data, n, tmp);
-    ++*launches;
+// 2. The count table in (list, part) order, scanned in place: cnt[part][x]
+// becomes row_ptr[x] + the hits of list x in earlier parts, where this part's
+// hits on x start.  One CTA per 32 lists: lane = list (coalesced rows of the
+// table), warp w walks a contiguous run of parts.
+__global__ void __launch_bounds__(kScanWarps * 32)
+    csr_colscan_kernel(int32_t* __restrict__ cnt, int64_t K, int64_t nparts,
+                       const int32_t* __restrict__ row_ptr) {
+  __shared__ int32_t part_sum[kScanWarps][33];
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int64_t x = (int64_t)blockIdx.x * 32 + l;
+  const int64_t per = (nparts + kScanWarps - 1) / kScanWarps;
+  const int64_t p0 = min64((int64_t)w * per, nparts), p1 = min64(p0 + per, nparts);
+  int32_t s = 0;
+  if (x < K) {
+#pragma unroll 4
+    for (int64_t p = p0; p < p1; ++p) s += cnt[p * K + x];
   }
-  return cudaGetLastError();
+  part_sum[w][l] = s;
+  __syncthreads();
+  if (x >= K) return;
+  int32_t base = __ldg(row_ptr + x);
+  for (int v = 0; v < w; ++v) base += part_sum[v][l];
+  for (int64_t p = p0; p < p1; ++p) {
+    const int32_t c = cnt[p * K + x];
+    cnt[p * K + x] = base;
+    base += c;
+  }
 }
 
-// row_ptr[x] = scanned[x * ntiles]; the end, row_ptr[n_lists], is the last
-// exclusive value plus the last count (saved before the in-place scan)
-__global__ void csr_rowptr_kernel(const int32_t* __restrict__ scanned, int64_t n_lists,
-                                  int32_t ntiles, const int32_t* __restrict__ last_count,
-                                  int32_t* __restrict__ row_ptr) {
-  const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (x < n_lists) row_ptr[x] = scanned[x * ntiles];
-  if (x == n_lists) row_ptr[x] = scanned[n_lists * ntiles - 1] + *last_count;
-}
-
-// One warp per (tile, group set): the set is GPW = 32 / top_k groups (one when
-// top_k > 16).  A row's ids are distinct within a group and different groups
-// key different lists, so the GPW * top_k hits of one row never share a key:
-// each lane reads its key's next free entry, writes there and advances it,
-// with no ranking among the lanes; rows are walked in order, so every list
-// stays in t order.  The tile's keys are first copied to shared memory with
-// independent loads, and so are the start offsets of every key of the set's
-// groups (the slice of nb keys given by s0).
-__global__ void __launch_bounds__(32) csr_scatter_kernel(const int32_t* __restrict__ ids,
-                                                         int64_t row_begin, int64_t rows,
-                                                         int32_t G, int32_t top_k, int64_t nb,
-                                                         int32_t ntiles, int32_t bins,
-                                                         int32_t gpw,
-                                                         const int32_t* __restrict__ scanned,
-                                                         const int32_t* __restrict__ row_base,
-                                                         int32_t* __restrict__ entries) {
+// 3. One warp per (part, group set): the set is gpw = 32 / top_k groups (one
+// when top_k > 16).  A row's ids are distinct within a group and different
+// groups key different lists, so the gpw * top_k hits of one row never share
+// a key: each lane reads its key's next free entry, writes there and advances
+// it, with no ranking among the lanes; rows are walked in order, so every
+// list stays in t order.  The part's start offsets of every key of the set's
+// groups (the slice of nb keys given by s0) are loaded once, contiguously;
+// keys are staged kKeyRows rows at a time with independent loads.
+__global__ void __launch_bounds__(32)
+    csr_scatter_kernel(const int32_t* __restrict__ ids, int64_t row_begin, int64_t rows,
+                       int32_t G, int32_t top_k, int64_t nb, int32_t R, int32_t bins, int32_t gpw,
+                       const int32_t* __restrict__ start, const int32_t* __restrict__ row_base,
+                       int32_t* __restrict__ entries) {
   extern __shared__ int32_t sm[];
-  int32_t* run = sm;                 // [gpw][bins]: next free entry of each key of the slice
-  int32_t* keys = sm + gpw * bins;   // [kTileTok][gpw * top_k]: the tile's keys, by row
-  const int tile = blockIdx.x, g0 = blockIdx.y * gpw;
+  int32_t* run = sm;                // [gpw][bins]: next free entry of each key of the slice
+  int32_t* keys = sm + gpw * bins;  // [kKeyRows][gpw * top_k]: keys of the staged rows
+  const int part = blockIdx.x, g0 = blockIdx.y * gpw;
   const int lane = threadIdx.x;
-  const int64_t r0 = (int64_t)tile * kTileTok;
-  const int64_t r1 = min(rows, r0 + kTileTok);
-  const int nrows = (int)(r1 - r0);
+  const int64_t K = (int64_t)G * nb;
+  const int64_t r0 = (int64_t)part * R;
+  const int nrows = (int)(min64(rows, r0 + R) - r0);
   const int per_row = gpw * top_k;  // hits of one row handled by one lane each (<= 32)
   const int ngrp = min(gpw, G - g0);
-  for (int e = lane; e < nrows * per_row; e += 32) {
-    const int rr = e / per_row, c = e - rr * per_row;
-    const int gi = c / top_k, r = c - gi * top_k;
-    const int64_t row = r0 + rr;
-    keys[e] = gi < ngrp ? list_key(row_base, row, __ldg(ids + (row * G + g0 + gi) * top_k + r))
-                        : -1;
-  }
   const bool active = lane < per_row;
   const int gi = active ? lane / top_k : 0;
   const int r = active ? lane - gi * top_k : 0;
+  const int32_t* srow = start + (int64_t)part * K + (int64_t)g0 * nb;
   for (int64_t s0 = 0; s0 < nb; s0 += kBinSlice) {
     const int width = (int)min64(kBinSlice, nb - s0);
-    // where this tile's hits on each key of the slice start, per group of the set
     for (int i = lane; i < ngrp * width; i += 32) {
       const int gg = i / width, x = i - gg * width;
-      run[gg * bins + x] = __ldg(scanned + ((int64_t)(g0 + gg) * nb + s0 + x) * ntiles + tile);
+      run[gg * bins + x] = __ldg(srow + (int64_t)gg * nb + s0 + x);
     }
-    __syncwarp();
-    for (int rr = 0; rr < nrows; ++rr) {
-      const int32_t j = active ? keys[rr * per_row + lane] : -1;
-      if (j >= s0 && j < s0 + width) {
-        int32_t* slot = run + gi * bins + (int)(j - s0);
-        const int32_t pos = *slot;
-        entries[pos] = (int32_t)(((row_begin + r0 + rr) << 5) | r);
-        *slot = pos + 1;
+    for (int rb = 0; rb < nrows; rb += kKeyRows) {
+      const int nr = min(kKeyRows, nrows - rb);
+      __syncwarp();
+      for (int e = lane; e < nr * per_row; e += 32) {
+        const int rr = e / per_row, c = e - rr * per_row;
+        const int gk = c / top_k, rk = c - gk * top_k;
+        const int64_t row = r0 + rb + rr;
+        keys[e] = gk < ngrp
+                      ? list_key(row_base, row, __ldg(ids + (row * G + g0 + gk) * top_k + rk))
+                      : -1;
       }
       __syncwarp();
+      for (int rr = 0; rr < nr; ++rr) {
+        const int32_t j = active ? keys[rr * per_row + lane] : -1;
+        if (j >= s0 && j < s0 + width) {
+          int32_t* slot = run + gi * bins + (int)(j - s0);
+          const int32_t pos = *slot;
+          entries[pos] = (int32_t)(((row_begin + r0 + rb + rr) << 5) | r);
+          *slot = pos + 1;
+        }
+        __syncwarp();
+      }
     }
   }
-}
-
-// Work units of the Main Branch: list x = g*nb + j is cut into runs of at
-// most `per_unit` entries; unit_ptr[x] is the exclusive prefix of the unit
-// counts (unit_ptr[n_lists] the total) and unit u gets {g, j, first entry,
-// end entry}.  One CTA: each thread counts a contiguous range of lists, the
-// CTA scans the per-thread sums, and each thread fills its range.
-constexpr int kUnitThreads = 1024;
-__global__ void __launch_bounds__(kUnitThreads)
-    units_kernel(const int32_t* __restrict__ row_ptr, int64_t n_lists, int64_t nb,
-                 int32_t per_unit, int32_t* __restrict__ unit_ptr, int4* __restrict__ unit_desc) {
-  __shared__ int32_t warp_tot[32];
-  const int64_t per = (n_lists + kUnitThreads - 1) / kUnitThreads;
-  const int64_t x0 = min64((int64_t)threadIdx.x * per, n_lists);
-  const int64_t x1 = min64(x0 + per, n_lists);
-  int32_t mine = 0;
-  for (int64_t x = x0; x < x1; ++x) mine += (row_ptr[x + 1] - row_ptr[x] + per_unit - 1) / per_unit;
-  const int32_t incl = warp_incl_scan(mine);
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  if (l == 31) warp_tot[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    const int32_t t = warp_tot[l];
-    warp_tot[l] = warp_incl_scan(t) - t;
-  }
-  __syncthreads();
-  int32_t u = warp_tot[w] + incl - mine;
-  for (int64_t x = x0; x < x1; ++x) {
-    unit_ptr[x] = u;
-    const int32_t beg = row_ptr[x], end = row_ptr[x + 1];
-    const int g = (int)(x / nb), j = (int)(x - (int64_t)g * nb);
-    for (int32_t e0 = beg; e0 < end; e0 += per_unit, ++u)
-      unit_desc[u] = make_int4(g, j, e0, min(end, e0 + per_unit));
-  }
-  if (threadIdx.x == kUnitThreads - 1) unit_ptr[n_lists] = u;
 }
 
 // ---- schedule of a batch of packed sequences --------------------------------
@@ -337,64 +327,73 @@ __global__ void __launch_bounds__(256) varlen_tables_kernel(const VarlenOffsets 
 
 }  // namespace
 
+// Query rows per part: the (part, list) count table stays at most half the
+// size of the ids (nb / R <= top_k / 2 for top_k = 16), and parts stay short
+// enough for many scatter warps.
+static int64_t part_rows(int64_t nb) {
+  int64_t R = 64;
+  while (R < 2048 && nb > 8 * R) R *= 2;
+  return R;
+}
+
 size_t csr_scratch_bytes(int64_t rows, int32_t G, int32_t top_k, int64_t nb) {
   (void)top_k;
-  const int64_t ntiles = (rows + kTileTok - 1) / kTileTok;
-  const int64_t table = (int64_t)G * nb * ntiles;
-  const int64_t lists = (int64_t)G * nb + 1;
-  size_t elems = (size_t)table + scan_scratch_elems(table) + 2 + scan_scratch_elems(lists) + 2;
+  const int64_t nparts = (rows + part_rows(nb) - 1) / part_rows(nb);
+  const int64_t K = (int64_t)G * nb;
+  const size_t elems = (size_t)(nparts * K) + (size_t)K + 1;  // table, totals, ticket
   return (elems * sizeof(int32_t) + 255) & ~(size_t)255;
 }
 
 cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
-  const int64_t ntiles = (p.rows + kTileTok - 1) / kTileTok;
-  const int64_t n_lists = (int64_t)p.G * p.nb;
-  const int64_t table = n_lists * ntiles;
+  const int64_t R = part_rows(p.nb);
+  const int64_t nparts = (p.rows + R - 1) / R;
+  const int64_t K = (int64_t)p.G * p.nb;
   int32_t* cnt = static_cast<int32_t*>(p.scratch);
-  int32_t* scan_tmp = cnt + table;
-  int32_t* last = scan_tmp + scan_scratch_elems(table) + 1;  // the table's last count
-  const int bins = (int)(p.nb < kBinSlice ? p.nb : kBinSlice);
+  int32_t* tot = cnt + nparts * K;
+  int32_t* ticket = tot + K;
   cudaError_t e;
-
-  dim3 grid((unsigned)ntiles, (unsigned)p.G);
+  if (nparts == 0) {
+    if ((e = cudaMemsetAsync(p.row_ptr, 0, (size_t)(K + 1) * sizeof(int32_t), s)) != cudaSuccess)
+      return e;
+    if (p.unit_ptr)
+      return cudaMemsetAsync(p.unit_ptr, 0, (size_t)(K + 1) * sizeof(int32_t), s);
+    return cudaSuccess;
+  }
+  if ((e = cudaMemsetAsync(tot, 0, (size_t)(K + 1) * sizeof(int32_t), s)) != cudaSuccess) return e;
+  const int bins = (int)(p.nb < kBinSlice ? p.nb : kBinSlice);
   const size_t bin_bytes = (size_t)bins * sizeof(int32_t);
   // groups per scatter warp: one row's hits of gpw groups fill at most 32 lanes,
-  // and their offsets and keys fit 200 KiB of shared memory
+  // and their offsets and staged keys fit 200 KiB of shared memory
   int gpw = p.top_k <= 16 ? (int)min64(32 / p.top_k, p.G) : 1;
   auto scatter_smem = [&](int w) {
-    return (size_t)w * bin_bytes + (size_t)kTileTok * w * p.top_k * sizeof(int32_t);
+    return (size_t)w * bin_bytes + (size_t)kKeyRows * w * p.top_k * sizeof(int32_t);
   };
   while (gpw > 1 && scatter_smem(gpw) > 200 * 1024) --gpw;
   const size_t scatter_bytes = scatter_smem(gpw);
   if (bin_bytes > 48 * 1024 &&
-      (e = cudaFuncSetAttribute(csr_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      (e = cudaFuncSetAttribute(csr_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)bin_bytes)) != cudaSuccess)
     return e;
   if (scatter_bytes > 48 * 1024 &&
       (e = cudaFuncSetAttribute(csr_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)scatter_bytes)) != cudaSuccess)
     return e;
-  csr_hist_kernel<<<grid, 256, bin_bytes, s>>>(p.ids, p.rows, p.G, p.top_k, p.nb,
-                                               (int32_t)ntiles, cnt, p.row_base, p.err);
+  ListTail tail;
+  tail.row_ptr = p.row_ptr;
+  tail.per_unit = p.unit_ptr ? p.tile_tokens * p.unit_tiles : 1;
+  tail.unit_ptr = p.unit_ptr;
+  tail.unit_desc = p.unit_desc;
+  csr_count_kernel<<<dim3((unsigned)nparts, (unsigned)p.G), kCountThreads, bin_bytes, s>>>(
+      p.ids, p.rows, p.G, p.top_k, p.nb, (int32_t)R, cnt, tot, ticket, p.row_base, p.err, tail);
   ++*launches;
-  if ((e = cudaMemcpyAsync(last, cnt + table - 1, sizeof(int32_t), cudaMemcpyDeviceToDevice, s)) !=
-      cudaSuccess)
-    return e;
-  if ((e = exclusive_scan(cnt, table, scan_tmp, s, launches)) != cudaSuccess) return e;
-  csr_rowptr_kernel<<<(unsigned)((n_lists + 1 + 255) / 256), 256, 0, s>>>(
-      cnt, n_lists, (int32_t)ntiles, last, p.row_ptr);
+  csr_colscan_kernel<<<(unsigned)((K + 31) / 32), kScanWarps * 32, 0, s>>>(cnt, K, nparts,
+                                                                            p.row_ptr);
   ++*launches;
-  dim3 sgrid((unsigned)ntiles, (unsigned)((p.G + gpw - 1) / gpw));
-  csr_scatter_kernel<<<sgrid, 32, scatter_bytes, s>>>(p.ids, p.row_begin, p.rows, p.G,
-                                                      p.top_k, p.nb, (int32_t)ntiles, bins, gpw,
-                                                      cnt, p.row_base, p.entries);
+  dim3 sgrid((unsigned)nparts, (unsigned)((p.G + gpw - 1) / gpw));
+  csr_scatter_kernel<<<sgrid, 32, scatter_bytes, s>>>(p.ids, p.row_begin, p.rows, p.G, p.top_k,
+                                                      p.nb, (int32_t)R, bins, gpw, cnt,
+                                                      p.row_base, p.entries);
   ++*launches;
-  if (p.unit_ptr) {
-    units_kernel<<<1, kUnitThreads, 0, s>>>(p.row_ptr, n_lists, p.nb,
-                                            p.tile_tokens * p.unit_tiles, p.unit_ptr,
-                                            p.unit_desc);
-    ++*launches;
-  }
   return cudaGetLastError();
 }
 

@@ -153,9 +153,9 @@ def test_decode_all_scores_tied(msa):
 
 
 def test_decode_clustered_high_scores(msa):
-    """The high-scoring blocks all fall on the candidates of one warp of the
-    selection (block ids j with j mod 256 < 32), so the threshold taken from
-    per-warp bests is weak and the exhaustive per-thread-list path decides."""
+    """The high-scoring blocks are clustered (block ids j with j mod 32 == 7, in
+    every range of 1,024 blocks), so a threshold taken from per-thread or
+    per-lane bests is weak and many candidates pass it."""
     s = synth.DecodeShape("dclu", seq_lens=(128 * 2048, 128 * 300), H=16, G=2, d=64, d_idx=128,
                           top_k=16, seed=15)
     inp = synth.make_decode_inputs(s, device="cuda")
@@ -165,9 +165,35 @@ def test_decode_clustered_high_scores(msa):
         u = inp["q_idx"][b, 0].double() + inp["q_idx"][b, 1].double()
         nb = (s.seq_lens[b] + s.block - 1) // s.block
         for j in range(nb - 1):
-            if j % 256 < 32:
+            if j % 32 == 7:
                 r0 = cu[b] + j * s.block
                 kic[r0:r0 + s.block] = (u * (1.0 + 1e-3 * j)).to(torch.bfloat16)
+    _check(msa, s, inp)
+
+
+def test_decode_selection_across_slices(msa):
+    """Selection over sequences of 2,000 to 3,000 blocks.
+    Sequence 0: the best blocks all lie in its last third (ids >= 2048).
+    Sequence 1: every score ties, so the lowest ids win.  Sequence 2: 2,050
+    blocks, one more than a multiple of 1,024 non-local candidates."""
+    s = synth.DecodeShape("dsli", seq_lens=(128 * 3000 + 9, 128 * 2601, 128 * 2050), H=16, G=2,
+                          d=64, d_idx=128, top_k=16, seed=16)
+    inp = synth.make_decode_inputs(s, device="cuda")
+    kic = inp["k_idx_cache"]
+    cu = inp["cu_seqlens"].tolist()
+    u = inp["q_idx"][0, 0].double() + inp["q_idx"][0, 1].double()
+    for j in range(2048, 3000):
+        if j % 61 == 3:
+            r0 = cu[0] + j * s.block
+            kic[r0:r0 + s.block] = (u * (1.0 + 1e-3 * j)).to(torch.bfloat16)
+    kic[cu[1]:cu[2]].zero_()
+    g_out, g_ids = _run(msa, s, inp)
+    nb1 = 2601
+    want = list(range(s.top_k - 1)) + [nb1 - 1]
+    for g in range(s.G):
+        assert g_ids[1, g].tolist() == want, g
+    sel0 = {int(j) for j in g_ids[0].ravel() if j >= 0}
+    assert all(j >= 2048 for j in sel0), sorted(sel0)
     _check(msa, s, inp)
 
 
