@@ -101,51 +101,77 @@ __device__ void list_prefix(const int32_t* tot, int64_t n_lists, int64_t nb, con
   }
 }
 
-// 1. Per part of R query rows and per group: a shared-memory histogram of the
-// part's hits over the key blocks, written as cnt[part][g*nb + j] (contiguous
-// per part) and added to the list totals tot[g*nb + j].  The last CTA to
-// finish (a ticket) computes row_ptr and the work units from the totals.
+// 1. Per part of R query rows and per set of gpc groups (all of them when
+// their gpc * nb bins fit kBinSlice): a shared-memory histogram of the part's
+// hits over the set's keys, written as cnt[part][g*nb + j] (contiguous per
+// part) and added to the list totals tot[g*nb + j].  Thread t owns column
+// t % (gpc * top_k) of every row it visits (one row's ids of the set are
+// contiguous).  The last CTA to finish (a ticket) computes row_ptr and the
+// work units from the totals.
 __global__ void __launch_bounds__(kCountThreads)
     csr_count_kernel(const int32_t* __restrict__ ids, int64_t rows, int32_t G, int32_t top_k,
-                     int64_t nb, int32_t R, int32_t* __restrict__ cnt, int32_t* __restrict__ tot,
-                     int32_t* __restrict__ ticket, const int32_t* __restrict__ row_base,
-                     uint32_t* err, ListTail tail) {
-  extern __shared__ int32_t bins[];
+                     int64_t nb, int32_t R, int32_t gpc, int32_t* __restrict__ cnt,
+                     int32_t* __restrict__ tot, int32_t* __restrict__ ticket,
+                     const int32_t* __restrict__ row_base, uint32_t* err, ListTail tail) {
+  extern __shared__ int32_t bins[];  // [gpc][width]
   __shared__ int last;
-  const int part = blockIdx.x, g = blockIdx.y;
+  const int part = blockIdx.x, g0 = blockIdx.y * gpc;
+  const int ng = min(gpc, G - g0);
   const int64_t K = (int64_t)G * nb;
   const int64_t r0 = (int64_t)part * R;
-  const int64_t r1 = min64(rows, r0 + R);
-  const int64_t n_el = (r1 - r0) * top_k;
-  int32_t* crow = cnt + (int64_t)part * K + (int64_t)g * nb;
-  for (int64_t s0 = 0; s0 < nb; s0 += kBinSlice) {
-    const int width = (int)min64(kBinSlice, nb - s0);
-    for (int i = threadIdx.x; i < width; i += blockDim.x) bins[i] = 0;
+  const int nrows = (int)(min64(rows, r0 + R) - r0);
+  const int per_row = ng * top_k;
+  const int col = threadIdx.x % per_row, rstep = blockDim.x / per_row;
+  const int rsub = threadIdx.x / per_row;
+  const int gk = col / top_k;  // group of this column within the set
+  const bool on = rsub < rstep;
+  int32_t* crow = cnt + (int64_t)part * K + (int64_t)g0 * nb;
+  const int32_t* idrow = ids + (r0 * G + g0) * top_k + col;
+  const int64_t id_pitch = (int64_t)G * top_k;
+  const int slice_w = kBinSlice / ng;  // one pass whenever ng > 1 (gpc * nb <= kBinSlice)
+  for (int64_t s0 = 0; s0 < nb; s0 += slice_w) {
+    const int width = (int)min64(slice_w, nb - s0);
+    for (int i = threadIdx.x; i < ng * width; i += blockDim.x) bins[i] = 0;
     __syncthreads();
-    for (int64_t e = threadIdx.x; e < n_el; e += blockDim.x) {
-      const int64_t row = r0 + e / top_k;
-      const int r = (int)(e % top_k);
-      const int32_t j = list_key(row_base, row, __ldg(ids + (row * G + g) * top_k + r));
-      if (j < -1 || j >= nb) {
-        if (s0 == 0) record_error(err, kDevBadIndex);
-        continue;
+    if (on) {
+      constexpr int kB = 16;
+      for (int rr0 = rsub; rr0 < nrows; rr0 += rstep * kB) {
+        int32_t v[kB];
+#pragma unroll
+        for (int q = 0; q < kB; ++q) {
+          const int rr = rr0 + q * rstep;
+          v[q] = rr < nrows ? __ldg(idrow + rr * id_pitch) : -1;
+        }
+#pragma unroll
+        for (int q = 0; q < kB; ++q) {
+          const int rr = rr0 + q * rstep;
+          if (rr >= nrows) continue;
+          const int32_t j = list_key(row_base, r0 + rr, v[q]);
+          if (j < -1 || j >= nb) {
+            if (s0 == 0) record_error(err, kDevBadIndex);
+            continue;
+          }
+          if (j >= s0 && j < s0 + width) atomicAdd(&bins[gk * width + (int)(j - s0)], 1);
+        }
       }
-      if (j >= s0 && j < s0 + width) atomicAdd(&bins[j - s0], 1);
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < width; i += blockDim.x) {
+    for (int i = threadIdx.x; i < ng * width; i += blockDim.x) {
+      const int gg = i / width, x = i - gg * width;
       const int32_t c = bins[i];
-      crow[s0 + i] = c;
-      if (c) atomicAdd(tot + (int64_t)g * nb + s0 + i, c);
+      crow[(int64_t)gg * nb + s0 + x] = c;
+      if (c) atomicAdd(tot + (int64_t)(g0 + gg) * nb + s0 + x, c);
     }
     __syncthreads();
   }
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(ticket, 1) == (int)(gridDim.x * gridDim.y) - 1;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last = atomicAdd(ticket, 1) == (int)(gridDim.x * gridDim.y) - 1;
+    __threadfence();
+  }
   __syncthreads();
   if (!last) return;
-  __threadfence();
   list_prefix(tot, K, nb, tail);
 }
 
@@ -161,20 +187,32 @@ __global__ void __launch_bounds__(kScanWarps * 32)
   const int64_t x = (int64_t)blockIdx.x * 32 + l;
   const int64_t per = (nparts + kScanWarps - 1) / kScanWarps;
   const int64_t p0 = min64((int64_t)w * per, nparts), p1 = min64(p0 + per, nparts);
+  constexpr int kB = 8;  // parts loaded at once
   int32_t s = 0;
   if (x < K) {
-#pragma unroll 4
-    for (int64_t p = p0; p < p1; ++p) s += cnt[p * K + x];
+    for (int64_t pb = p0; pb < p1; pb += kB) {
+      int32_t c[kB];
+#pragma unroll
+      for (int q = 0; q < kB; ++q) c[q] = pb + q < p1 ? cnt[(pb + q) * K + x] : 0;
+#pragma unroll
+      for (int q = 0; q < kB; ++q) s += c[q];
+    }
   }
   part_sum[w][l] = s;
   __syncthreads();
   if (x >= K) return;
   int32_t base = __ldg(row_ptr + x);
   for (int v = 0; v < w; ++v) base += part_sum[v][l];
-  for (int64_t p = p0; p < p1; ++p) {
-    const int32_t c = cnt[p * K + x];
-    cnt[p * K + x] = base;
-    base += c;
+  for (int64_t pb = p0; pb < p1; pb += kB) {
+    int32_t c[kB];
+#pragma unroll
+    for (int q = 0; q < kB; ++q) c[q] = pb + q < p1 ? cnt[(pb + q) * K + x] : 0;
+#pragma unroll
+    for (int q = 0; q < kB; ++q)
+      if (pb + q < p1) {
+        cnt[(pb + q) * K + x] = base;
+        base += c[q];
+      }
   }
 }
 
@@ -205,22 +243,36 @@ __global__ void __launch_bounds__(32)
   const int gi = active ? lane / top_k : 0;
   const int r = active ? lane - gi * top_k : 0;
   const int32_t* srow = start + (int64_t)part * K + (int64_t)g0 * nb;
+  const int32_t* idcol = ids + (r0 * G + g0) * top_k + lane;  // this lane's column
+  const int64_t id_pitch = (int64_t)G * top_k;
+  const bool col_on = lane < ngrp * top_k;
+  constexpr int kB = 8;  // loads in flight per lane
   for (int64_t s0 = 0; s0 < nb; s0 += kBinSlice) {
     const int width = (int)min64(kBinSlice, nb - s0);
-    for (int i = lane; i < ngrp * width; i += 32) {
-      const int gg = i / width, x = i - gg * width;
-      run[gg * bins + x] = __ldg(srow + (int64_t)gg * nb + s0 + x);
-    }
+    for (int gg = 0; gg < ngrp; ++gg)
+      for (int x0 = lane; x0 < width; x0 += 32 * kB) {
+        int32_t v[kB];
+#pragma unroll
+        for (int q = 0; q < kB; ++q)
+          v[q] = x0 + 32 * q < width ? __ldg(srow + (int64_t)gg * nb + s0 + x0 + 32 * q) : 0;
+#pragma unroll
+        for (int q = 0; q < kB; ++q)
+          if (x0 + 32 * q < width) run[gg * bins + x0 + 32 * q] = v[q];
+      }
     for (int rb = 0; rb < nrows; rb += kKeyRows) {
       const int nr = min(kKeyRows, nrows - rb);
       __syncwarp();
-      for (int e = lane; e < nr * per_row; e += 32) {
-        const int rr = e / per_row, c = e - rr * per_row;
-        const int gk = c / top_k, rk = c - gk * top_k;
-        const int64_t row = r0 + rb + rr;
-        keys[e] = gk < ngrp
-                      ? list_key(row_base, row, __ldg(ids + (row * G + g0 + gk) * top_k + rk))
-                      : -1;
+      if (active) {
+        for (int rr0 = 0; rr0 < nr; rr0 += kB) {
+          int32_t v[kB];
+#pragma unroll
+          for (int q = 0; q < kB; ++q)
+            v[q] = (col_on && rr0 + q < nr) ? __ldg(idcol + (int64_t)(rb + rr0 + q) * id_pitch) : -1;
+#pragma unroll
+          for (int q = 0; q < kB; ++q)
+            if (rr0 + q < nr)
+              keys[(rr0 + q) * per_row + lane] = list_key(row_base, r0 + rb + rr0 + q, v[q]);
+        }
       }
       __syncwarp();
       for (int rr = 0; rr < nr; ++rr) {
@@ -362,6 +414,11 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
   if ((e = cudaMemsetAsync(tot, 0, (size_t)(K + 1) * sizeof(int32_t), s)) != cudaSuccess) return e;
   const int bins = (int)(p.nb < kBinSlice ? p.nb : kBinSlice);
   const size_t bin_bytes = (size_t)bins * sizeof(int32_t);
+  // groups per count CTA: all whose bins fit one pass of kBinSlice, and whose
+  // ids of one row fit the CTA's threads
+  const int gpc = (int)min64(min64(p.G, p.nb <= kBinSlice ? kBinSlice / p.nb : 1),
+                             kCountThreads / p.top_k);
+  const size_t count_bytes = (size_t)min64((int64_t)gpc * p.nb, kBinSlice) * sizeof(int32_t);
   // groups per scatter warp: one row's hits of gpw groups fill at most 32 lanes,
   // and their offsets and staged keys fit 200 KiB of shared memory
   int gpw = p.top_k <= 16 ? (int)min64(32 / p.top_k, p.G) : 1;
@@ -370,9 +427,9 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
   };
   while (gpw > 1 && scatter_smem(gpw) > 200 * 1024) --gpw;
   const size_t scatter_bytes = scatter_smem(gpw);
-  if (bin_bytes > 48 * 1024 &&
+  if (count_bytes > 48 * 1024 &&
       (e = cudaFuncSetAttribute(csr_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)bin_bytes)) != cudaSuccess)
+                                (int)count_bytes)) != cudaSuccess)
     return e;
   if (scatter_bytes > 48 * 1024 &&
       (e = cudaFuncSetAttribute(csr_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -383,8 +440,9 @@ cudaError_t launch_csr(const CsrLaunch& p, cudaStream_t s, int* launches) {
   tail.per_unit = p.unit_ptr ? p.tile_tokens * p.unit_tiles : 1;
   tail.unit_ptr = p.unit_ptr;
   tail.unit_desc = p.unit_desc;
-  csr_count_kernel<<<dim3((unsigned)nparts, (unsigned)p.G), kCountThreads, bin_bytes, s>>>(
-      p.ids, p.rows, p.G, p.top_k, p.nb, (int32_t)R, cnt, tot, ticket, p.row_base, p.err, tail);
+  csr_count_kernel<<<dim3((unsigned)nparts, (unsigned)((p.G + gpc - 1) / gpc)), kCountThreads,
+                     count_bytes, s>>>(p.ids, p.rows, p.G, p.top_k, p.nb, (int32_t)R, gpc, cnt,
+                                       tot, ticket, p.row_base, p.err, tail);
   ++*launches;
   csr_colscan_kernel<<<(unsigned)((K + 31) / 32), kScanWarps * 32, 0, s>>>(cnt, K, nparts,
                                                                             p.row_ptr);
