@@ -380,3 +380,99 @@ def pooled_scores_fp8_rows(q8_rows, pos, k8, k_row_scale, block: int, nb_out: in
     lib.msa_oracle_pooled_scores_f64(_ptr(qv), _ptr(pos), n, _ptr(kv), G, di, block, nb_out,
                                      _ptr(out))
     return out
+
+
+# ---------------------------------------------------------------------------
+# Quantised Main Branch ("Q8KV4"; dot-ai "MiniMax M3.1 Flashとは？428BのMoEモデル
+# がウェイト公開", the passage on the ModelScope model card's quantisation: the
+# sparse attention moving from Q8KV8 to Q8KV4).  The pages name no number
+# format.  The reading used: the OCP Microscaling (MX) formats, version 1.0 --
+# every 32 consecutive values along d share one power-of-two scale 2^X, kept
+# as an 8-bit biased exponent (E8M0, X + 127); X = floor(log2(max|x|)) -
+# emax_elem (emax_elem = 8 for e4m3, 2 for e2m1), -127 for an all-zero block,
+# clamped to [-127, 127]; each element is the nearest value of its format to
+# x / 2^X (ties to even), saturating at the format's largest magnitude.  Q is
+# MXFP8 (e4m3 elements), K and V are MXFP4 (e2m1 elements).
+# ---------------------------------------------------------------------------
+
+MX_BLOCK = 32
+MX_E4M3, MX_E2M1 = 0, 1
+MX_EMAX = {MX_E4M3: 8, MX_E2M1: 2}
+# e2m1: 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit; code & 7 indexes
+# the magnitude (0 and 1 are the zero and the subnormal 0.5)
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    """e2m1 codes (0..15, one per byte) -> fp64."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    return np.where(c & 8, -1.0, 1.0) * E2M1_VALUES[c & 7]
+
+
+def e2m1_encode(y: np.ndarray) -> np.ndarray:
+    """Values -> nearest e2m1 code, ties to the even code, saturating at 6;
+    the sign bit is the value's own (so -0 gives code 8)."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.minimum(np.abs(y), 6.0)
+    lo = np.clip(np.searchsorted(E2M1_VALUES, a, side="right") - 1, 0, 7)
+    hi = np.minimum(lo + 1, 7)
+    vlo, vhi = E2M1_VALUES[lo], E2M1_VALUES[hi]
+    mid = (vlo + vhi) / 2.0
+    pick = np.where(a < mid, lo, np.where(a > mid, hi, np.where(lo % 2 == 0, lo, hi)))
+    pick = np.where(hi == lo, lo, pick)
+    return (pick | np.where(np.signbit(y), 8, 0)).astype(np.uint8)
+
+
+def mx_block_exponent(amax: np.ndarray, fmt: int) -> np.ndarray:
+    """X of each block from its largest magnitude (exact: frexp)."""
+    amax = np.asarray(amax, dtype=np.float64)
+    _, e = np.frexp(np.where(amax > 0, amax, 1.0))  # amax = m 2^e, m in [0.5, 1)
+    x = np.where(amax > 0, e - 1 - MX_EMAX[fmt], -127)
+    return np.clip(x, -127, 127).astype(np.int64)
+
+
+def mx_quantize(x, fmt: int):
+    """x [..., d] bf16 (d a multiple of 32) -> (codes [..., d] uint8: e4m3
+    bytes or e2m1 codes, one per byte; scales [..., d/32] uint8, X + 127)."""
+    xf = bf16_bits_to_f64(as_bf16_bits(x))
+    d = xf.shape[-1]
+    assert d % MX_BLOCK == 0
+    blocks = xf.reshape(xf.shape[:-1] + (d // MX_BLOCK, MX_BLOCK))
+    X = mx_block_exponent(np.abs(blocks).max(axis=-1), fmt)
+    y = blocks / np.exp2(X.astype(np.float64))[..., None]  # exact: a power of two
+    codes = e4m3_encode(y.astype(np.float32)) if fmt == MX_E4M3 else e2m1_encode(y)
+    return codes.reshape(xf.shape).astype(np.uint8), (X + 127).astype(np.uint8)
+
+
+def mx_dequantize(codes, scales, fmt: int) -> np.ndarray:
+    """(codes [..., d], scales [..., d/32]) -> fp64 values code * 2^(scale - 127)."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    d = codes.shape[-1]
+    v = e4m3_decode(codes) if fmt == MX_E4M3 else e2m1_decode(codes)
+    X = np.asarray(scales, dtype=np.uint8).astype(np.int64) - 127
+    v = v.reshape(codes.shape[:-1] + (d // MX_BLOCK, MX_BLOCK))
+    return (v * np.exp2(X.astype(np.float64))[..., None]).reshape(codes.shape)
+
+
+def pack_e2m1(codes: np.ndarray) -> np.ndarray:
+    """[..., d] codes -> [..., d/2] bytes, element 2i in the low nibble."""
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)
+
+
+def unpack_e2m1(packed: np.ndarray) -> np.ndarray:
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp64 values that bf16 represents exactly -> their bf16 bit patterns."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    assert np.array_equal(f.astype(np.float64), np.asarray(x, dtype=np.float64),
+                          equal_nan=True), "value not exact in fp32"
+    bits = f.view(np.uint32)
+    assert not np.any(bits & 0xFFFF), "value not exact in bf16"
+    return (bits >> 16).astype(np.uint16)

@@ -153,9 +153,9 @@ def test_decode_all_scores_tied(msa):
 
 
 def test_decode_clustered_high_scores(msa):
-    """The high-scoring blocks are clustered (block ids j with j mod 32 == 7, in
-    every range of 1,024 blocks), so a threshold taken from per-thread or
-    per-lane bests is weak and many candidates pass it."""
+    """The high-scoring blocks all fall on the candidates of one warp of the
+    selection (block ids j with j mod 256 < 32), so the threshold taken from
+    per-warp bests is weak and the exhaustive per-thread-list path decides."""
     s = synth.DecodeShape("dclu", seq_lens=(128 * 2048, 128 * 300), H=16, G=2, d=64, d_idx=128,
                           top_k=16, seed=15)
     inp = synth.make_decode_inputs(s, device="cuda")
@@ -165,13 +165,13 @@ def test_decode_clustered_high_scores(msa):
         u = inp["q_idx"][b, 0].double() + inp["q_idx"][b, 1].double()
         nb = (s.seq_lens[b] + s.block - 1) // s.block
         for j in range(nb - 1):
-            if j % 32 == 7:
+            if j % 256 < 32:
                 r0 = cu[b] + j * s.block
                 kic[r0:r0 + s.block] = (u * (1.0 + 1e-3 * j)).to(torch.bfloat16)
     _check(msa, s, inp)
 
 
-def test_decode_selection_across_slices(msa):
+def test_decode_selection_long_sequences(msa):
     """Selection over sequences of 2,000 to 3,000 blocks.
     Sequence 0: the best blocks all lie in its last third (ids >= 2048).
     Sequence 1: every score ties, so the lowest ids win.  Sequence 2: 2,050
