@@ -333,6 +333,8 @@ def workload_config(args, shape):
            "block": shape.block, "top_k": shape.top_k, "needles": shape.n_needles,
            "l2": "inputs larger than L2 (no flush)", "parallelism": "replicas",
            "index": "e4m3" if getattr(args, "index_fp8", False) else "bf16"}
+    if getattr(args, "q8kv4", False):
+        cfg["main_inputs"] = "MX: e4m3 q, e2m1 k/v, one E8M0 scale per 32 values"
     if not args.no_decode:
         dc = decode_shape(args)
         lens = sorted(set(dc.seq_lens))
@@ -381,13 +383,15 @@ class PrefillRun:
         self.cfg = msa.config(shape.H, shape.G, shape.d, shape.d_idx, top_k=shape.top_k,
                               block=shape.block, scale=shape.scale)
         self.inp = synth.make_prefill_inputs(shape, device=dev, seed=shape.seed + rank)
+        q8kv4 = getattr(args, "q8kv4", False)
         full_ws = msa.msa_workspace_size(self.cfg, msa.OP_PREFILL, N)
+        dq = (msa.msa_workspace_size(self.cfg, msa.OP_PREFILL_Q8KV4, N) - full_ws) if q8kv4 else 0
         cap = int(args.ws_gb * (1 << 30))
-        self.ws = torch.empty(max(min(full_ws, cap), msa.msa_prefill_min_workspace(self.cfg, N)),
-                              dtype=torch.uint8, device=dev)
+        self.ws = torch.empty(max(min(full_ws, cap), msa.msa_prefill_min_workspace(self.cfg, N))
+                              + dq, dtype=torch.uint8, device=dev)
         self.out = torch.empty((N, shape.H, shape.d), dtype=torch.bfloat16, device=dev)
         self.ids = torch.empty((N, shape.G, shape.top_k), dtype=torch.int32, device=dev)
-        chunk = msa.msa_prefill_chunk_tokens(self.cfg, N, self.ws.numel(), ids_returned=True)
+        chunk = msa.msa_prefill_chunk_tokens(self.cfg, N, self.ws.numel() - dq, ids_returned=True)
         self.n_chunks = (N + chunk - 1) // chunk
         self.quant_ms = None
         if args.index_fp8:
@@ -404,10 +408,29 @@ class PrefillRun:
             torch.cuda.synchronize()
             self.quant_ms = e0.elapsed_time(e1)
             del qz
+        self.dq_start = []  # q8kv4: an event before each call (the dequantisation)
+        if q8kv4:
+            # MX inputs (a model serving a Q8KV4 cache holds them): quantised once
+            # here, the quantiser's time reported beside the dequantisation
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            self.mx = (*msa.msa_quantize_mx(self.inp["q"], msa.MX_E4M3),
+                       *msa.msa_quantize_mx(self.inp["k"], msa.MX_E2M1),
+                       *msa.msa_quantize_mx(self.inp["v"], msa.MX_E2M1))
+            e1.record()
+            torch.cuda.synchronize()
+            self.quant_ms = e0.elapsed_time(e1)
 
     def once(self):
         msa, inp = self.msa, self.inp
-        if self.args.index_fp8:
+        if getattr(self.args, "q8kv4", False):
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record()
+            self.dq_start.append(ev)
+            q8, qs, k4, ks, v4, vs = self.mx
+            msa.msa_prefill_q8kv4(self.cfg, q8, qs, k4, ks, v4, vs, inp["q_idx"], inp["k_idx"],
+                                  out=self.out, ids_out=self.ids, workspace=self.ws)
+        elif self.args.index_fp8:
             msa.msa_prefill_fp8_index(self.cfg, inp["q"], inp["k"], inp["v"], self.q8, self.k8,
                                       self.ks, out=self.out, ids_out=self.ids, workspace=self.ws)
         else:
@@ -428,7 +451,19 @@ class PrefillRun:
         nc = self.n_chunks
         pre_ph = np.array([[sum(e[5 * c + ph].elapsed_time(e[5 * c + ph + 1]) for c in range(nc))
                             for ph in range(4)] for e in pev])
+        q8kv4 = getattr(args, "q8kv4", False)
+        if q8kv4:  # the dequantisation runs before the library's first phase event
+            starts = self.dq_start[-len(pev):]
+            dq_ph = np.array([st.elapsed_time(e[0]) for st, e in zip(starts, pev)])
+            pre_ph = np.concatenate([dq_ph[:, None], pre_ph], axis=1)
         value, pre_ms = replica_rate(shape.N, float(pre_ph.sum(axis=1).mean()), world)
+        if q8kv4:
+            N, H, G, d = shape.N, shape.H, shape.G, shape.d
+            mx_bytes = (N * H * d * (1 + 2) + N * 2 * G * d * (0.5 + 2)
+                        + (N * H + 2 * N * G) * d / 32)  # codes + scales in, bf16 out
+            r = table.add("mx_dequantize", pre_ph[:, 0], "hbm", mx_bytes)
+            r["quantize_ms"] = self.quant_ms
+            pre_ph = pre_ph[:, 1:]
         pw = prefill_work(self.ids.cpu().numpy(), shape.H, shape.d, shape.block)
         idx_f = index_flops(shape.N, shape.G, shape.d_idx, shape.block)
         # e4m3 selection: its own dtype's peak, the measured bf16 one times the
@@ -639,7 +674,7 @@ def run_ours(args, rank, world, local):
                 f"({'hbm_gbs' if dk['unit'] == 'GB/s' else table.tc_name})"}
 
     # ---- end to end through the public API with host buffers ----
-    e2e = None if (args.no_e2e or args.index_fp8) else run_e2e(
+    e2e = None if (args.no_e2e or args.index_fp8 or args.q8kv4) else run_e2e(
         args, msa, cfg, shape, run.inp if run else None, run.ws if run else None,
         run.out if run else None, dev, dec, dcfg if dec is not None else None,
         dws if dec is not None else None, world)
@@ -986,6 +1021,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--index-fp8", action="store_true",
                     help="prefill with the quantised (e4m3) Index Branch; e2e is not run")
+    ap.add_argument("--q8kv4", action="store_true",
+                    help="prefill on MX inputs (e4m3 q, e2m1 k/v): msa_prefill_q8kv4; e2e is "
+                         "not run")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (large workloads)")
     ap.add_argument("--cpu-budget", type=float, default=15.0,

@@ -27,7 +27,8 @@ __all__ = [
     "msa_status_string", "msa_last_launch_count", "msa_set_phase_events", "msa_decode_static",
     "msa_selftest_wait_timeout", "msa_prefill_varlen", "msa_prefill_block_alignment",
     "msa_prefill_fp8_index", "msa_prefill_varlen_workspace_size", "msa_decode_fp8_index",
-    "msa_quantize_rows_fp8",
+    "msa_quantize_rows_fp8", "OP_PREFILL_Q8KV4", "MX_E4M3", "MX_E2M1", "msa_quantize_mx",
+    "msa_prefill_q8kv4",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,6 +38,8 @@ OP_SELECT_TOPK = 0
 OP_BLOCK_QUERY_LISTS = 1
 OP_PREFILL = 2
 OP_DECODE = 3
+OP_PREFILL_Q8KV4 = 4
+MX_E4M3, MX_E2M1 = 0, 1
 
 STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
                 3: "MSA_ERR_WORKSPACE", 4: "MSA_ERR_CUDA", 5: "MSA_ERR_DEVICE_TIMEOUT",
@@ -107,6 +110,8 @@ def load_library():
     lib.msa_decode_static.argtypes = [C, P, P, P, P, P, P, I32, I64, I64, P, P, I32, P]
     lib.msa_decode_fp8_index.argtypes = [C, P, P, P, P, P, P, P, I32, I64, P, P, P, SZ, P]
     lib.msa_quantize_rows_fp8.argtypes = [P, I64, P, P, P]
+    lib.msa_quantize_mx.argtypes = [P, I64, I32, I32, P, P, P]
+    lib.msa_prefill_q8kv4.argtypes = [C, P, P, P, P, P, P, P, P, I64, P, P, P, SZ, P]
     lib.msa_get_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
     lib.msa_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
     lib.msa_status_string.argtypes = [ctypes.c_int]
@@ -121,6 +126,7 @@ def load_library():
                  "msa_build_block_query_lists", "msa_prefill",
                  "msa_prefill_varlen", "msa_prefill_varlen_workspace_size",
                  "msa_prefill_block_alignment", "msa_prefill_fp8_index",
+                 "msa_quantize_mx", "msa_prefill_q8kv4",
                  "msa_decode",
                  "msa_decode_static", "msa_get_device_error", "msa_selftest_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
@@ -466,6 +472,52 @@ def msa_quantize_rows_fp8(x: torch.Tensor, stream=None):
                                    _stream(stream))
     _check(st, "msa_quantize_rows_fp8")
     return x8, sc
+
+
+def msa_quantize_mx(x: torch.Tensor, fmt: int, stream=None):
+    """x [..., d] bf16 (d a multiple of 32) -> (codes uint8, scales uint8 [..., d/32]):
+    MX_E4M3 codes [..., d], MX_E2M1 codes [..., d/2] (two per byte)."""
+    lib = load_library()
+    d = x.shape[-1]
+    if d % 32 != 0:
+        raise MsaError("msa_quantize_mx: rows of a multiple of 32 values expected")
+    rows = x.numel() // d
+    cw = d if fmt == MX_E4M3 else d // 2
+    codes = torch.empty(x.shape[:-1] + (cw,), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(x.shape[:-1] + (d // 32,), dtype=torch.uint8, device=x.device)
+    st = lib.msa_quantize_mx(_dev(x, torch.bfloat16, "x"), rows, d, fmt,
+                             _dev(codes, torch.uint8, "codes"), _dev(scales, torch.uint8, "scales"),
+                             _stream(stream))
+    _check(st, "msa_quantize_mx")
+    return codes, scales
+
+
+def msa_prefill_q8kv4(cfg: MsaConfig, q8, q_scale, k4, k_scale, v4, v_scale, q_idx, k_idx,
+                      out: Optional[torch.Tensor] = None, ids_out=None,
+                      workspace: Optional[torch.Tensor] = None, stream=None):
+    """msa_prefill on MX inputs (see include/msa.h): q8 [N,H,d] e4m3 with q_scale
+    [N,H,d/32]; k4, v4 [N,G,d/2] packed e2m1 with k_scale, v_scale [N,G,d/32]."""
+    lib = load_library()
+    N = q8.shape[0]
+    H, G, d, di, kk = cfg.num_heads, cfg.num_groups, cfg.head_dim, cfg.index_dim, cfg.top_k
+    if out is None:
+        out = torch.empty((N, H, d), dtype=torch.bfloat16, device=q8.device)
+    if ids_out is True:
+        ids_out = torch.empty((N, G, kk), dtype=torch.int32, device=q8.device)
+    ws = _workspace(workspace, msa_workspace_size(cfg, OP_PREFILL_Q8KV4, N), q8.device)
+    ids_ptr = None if ids_out is None else _dev(ids_out, torch.int32, "ids_out", (N, G, kk))
+    st = lib.msa_prefill_q8kv4(
+        ctypes.byref(cfg), _dev(q8, torch.uint8, "q8", (N, H, d)),
+        _dev(q_scale, torch.uint8, "q_scale", (N, H, d // 32)),
+        _dev(k4, torch.uint8, "k4", (N, G, d // 2)),
+        _dev(k_scale, torch.uint8, "k_scale", (N, G, d // 32)),
+        _dev(v4, torch.uint8, "v4", (N, G, d // 2)),
+        _dev(v_scale, torch.uint8, "v_scale", (N, G, d // 32)),
+        _dev(q_idx, torch.bfloat16, "q_idx", (N, G, di)), _dev(k_idx, torch.bfloat16, "k_idx", (N, di)),
+        N, _dev(out, torch.bfloat16, "out", (N, H, d)), ids_ptr, _dev(ws, torch.uint8, "ws"),
+        ws.numel(), _stream(stream))
+    _check(st, "msa_prefill_q8kv4")
+    return out if ids_out is None else (out, ids_out)
 
 
 def msa_decode_fp8_index(cfg: MsaConfig, q, q_idx8, k_cache, v_cache, k_idx8_cache, k_idx_scale,

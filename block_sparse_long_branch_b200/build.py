@@ -19,7 +19,7 @@ LIB = os.path.join(HERE, "libmsa_b200.so")
 HEADER = os.path.join(ROOT, "include", "msa.h")
 
 SOURCES = ["api.cu", "index_kernel.cu", "csr_kernel.cu", "main_kernel.cu", "merge_kernel.cu",
-           "align_kernel.cu", "quant_kernel.cu",
+           "align_kernel.cu", "quant_kernel.cu", "mx_kernel.cu",
            "decode_kernel.cu", "decode_static.cu", "selftest.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",

@@ -60,6 +60,12 @@ constexpr int kDecodeMaxHeadsPerGroup = 16;
 
 int64_t n_blocks(int64_t n) { return (n + kBlock - 1) / kBlock; }
 
+// the dequantised q, k, v (bf16) of msa_prefill_q8kv4
+size_t mx_dequant_bytes(const msa_config_t* c, int64_t N) {
+  return align256((size_t)N * c->num_heads * c->head_dim * 2) +
+         2 * align256((size_t)N * c->num_groups * c->head_dim * 2);
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -219,6 +225,10 @@ msa_status_t msa_workspace_size(const msa_config_t* cfg, msa_op_t op, int64_t n_
       return MSA_OK;
     case MSA_OP_PREFILL:
       *bytes = prefill_layout(cfg, n_tokens, n_tokens, nb, true).total;
+      return MSA_OK;
+    case MSA_OP_PREFILL_Q8KV4:
+      *bytes = prefill_layout(cfg, n_tokens, n_tokens, nb, true).total +
+               mx_dequant_bytes(cfg, n_tokens);
       return MSA_OK;
     case MSA_OP_DECODE:
       break;
@@ -746,6 +756,53 @@ msa_status_t msa_prefill_fp8_index(const msa_config_t* cfg, const void* q, const
   int launches = 0;
   st = prefill_run(cfg, q, k, v, q_idx8, k_idx8, N, out, ids_out, ws, ws_bytes, s, true,
                    &launches, nullptr, nullptr, nullptr, k_scale);
+  g_launches = launches;
+  return st;
+}
+
+msa_status_t msa_quantize_mx(const void* x, int64_t rows, int32_t d, int32_t fmt, void* codes,
+                             uint8_t* scales, msa_stream_t stream) {
+  g_launches = 0;
+  if (rows < 0 || d <= 0 || d % 32 != 0 || (fmt != MSA_MX_E4M3 && fmt != MSA_MX_E2M1))
+    return MSA_ERR_INVALID_ARG;
+  if (rows == 0) return MSA_OK;
+  if (!x || !codes || !scales || !aligned16(x) || !aligned16(codes)) return MSA_ERR_INVALID_ARG;
+  const msa_status_t st =
+      cuda_status(launch_mx_quantize(x, rows * (d / 32), fmt == MSA_MX_E4M3 ? kMxE4m3 : kMxE2m1,
+                                     codes, scales, sm_count(),
+                                     reinterpret_cast<cudaStream_t>(stream)));
+  if (st == MSA_OK) g_launches = 1;
+  return st;
+}
+
+msa_status_t msa_prefill_q8kv4(const msa_config_t* cfg, const void* q8, const uint8_t* q_scale,
+                               const void* k4, const uint8_t* k_scale, const void* v4,
+                               const uint8_t* v_scale, const void* q_idx, const void* k_idx,
+                               int64_t N, void* out, int32_t* ids_out, void* ws, size_t ws_bytes,
+                               msa_stream_t stream) {
+  g_launches = 0;
+  msa_status_t st = check_cfg(cfg);
+  if (st != MSA_OK) return st;
+  if ((st = check_tokens(cfg, N)) != MSA_OK) return st;
+  if ((st = check_prefill_ptrs(q8, k4, v4, q_idx, k_idx, out, ids_out, ws)) != MSA_OK) return st;
+  if (!q_scale || !k_scale || !v_scale) return MSA_ERR_INVALID_ARG;
+  const size_t dq = mx_dequant_bytes(cfg, N);
+  if (ws_bytes < dq) return MSA_ERR_WORKSPACE;
+  const size_t pws = (ws_bytes - dq) & ~(size_t)255;  // the prefill's part, at the front
+  if (prefill_chunk(cfg, N, pws, ids_out == nullptr) == 0) return MSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  const int64_t H = cfg->num_heads, G = cfg->num_groups, d = cfg->head_dim;
+  uint8_t* qd = static_cast<uint8_t*>(ws) + pws;
+  uint8_t* kd = qd + align256((size_t)N * H * d * 2);
+  uint8_t* vd = kd + align256((size_t)N * G * d * 2);
+  const int sms = sm_count();
+  cudaError_t e = launch_mx_dequantize(q8, q_scale, N * H * d / 32, kMxE4m3, qd, sms, s);
+  if (e == cudaSuccess) e = launch_mx_dequantize(k4, k_scale, N * G * d / 32, kMxE2m1, kd, sms, s);
+  if (e == cudaSuccess) e = launch_mx_dequantize(v4, v_scale, N * G * d / 32, kMxE2m1, vd, sms, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  int launches = 3;
+  st = prefill_run(cfg, qd, kd, vd, q_idx, k_idx, N, out, ids_out, ws, pws, s, true, &launches);
   g_launches = launches;
   return st;
 }

@@ -182,6 +182,15 @@ struct DecodeLaunch {
   int n_events;
 };
 size_t decode_pooled_rows(int64_t total_len, int32_t B);
+
+// ---- MX block formats of the quantised Main Branch (mx_kernel.cu) ----------
+// x [n_blocks * 32] bf16 <-> codes (e4m3: one byte per value; e2m1: two values
+// per byte, element 2i in the low nibble) and one E8M0 scale byte per block.
+constexpr int kMxE4m3 = 0, kMxE2m1 = 1;
+cudaError_t launch_mx_quantize(const void* x, int64_t n_blocks, int fmt, void* codes,
+                               uint8_t* scales, int sms, cudaStream_t s);
+cudaError_t launch_mx_dequantize(const void* codes, const uint8_t* scales, int64_t n_blocks,
+                                 int fmt, void* out, int sms, cudaStream_t s);
 // floats of one split partial of the decode attention: [heads][d] + max + sum
 size_t decode_partial_floats(int32_t H, int32_t G, int32_t d);
 constexpr int kDecodeMaxSplit = 4;

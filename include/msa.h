@@ -86,7 +86,8 @@ typedef enum {
   MSA_OP_SELECT_TOPK = 0,
   MSA_OP_BLOCK_QUERY_LISTS = 1,
   MSA_OP_PREFILL = 2,
-  MSA_OP_DECODE = 3
+  MSA_OP_DECODE = 3,
+  MSA_OP_PREFILL_Q8KV4 = 4
 } msa_op_t;
 
 /*
@@ -96,6 +97,8 @@ typedef enum {
  *     msa_prefill also accepts less (down to msa_prefill_min_workspace) and
  *     then walks the query axis in chunks (msa_prefill_chunk_tokens).
  *   DECODE: n_tokens = total cache rows (sum of sequence lengths), batch = B.
+ *   PREFILL_Q8KV4: n_tokens = N; the PREFILL size plus the dequantised
+ *     q, k, v (bf16) that msa_prefill_q8kv4 keeps at the end of its workspace.
  * Host-only; returns MSA_ERR_INVALID_ARG / MSA_ERR_UNSUPPORTED like the op.
  */
 MSA_API msa_status_t msa_workspace_size(const msa_config_t* cfg, msa_op_t op, int64_t n_tokens,
@@ -228,6 +231,46 @@ MSA_API msa_status_t msa_prefill_fp8_index(const msa_config_t* cfg, const void* 
                                            const float* k_scale, int64_t N, void* out,
                                            int32_t* ids_out, void* ws, size_t ws_bytes,
                                            msa_stream_t stream);
+
+/*
+ * Quantised Main Branch inputs ("Q8KV4"; same passage as above: the sparse
+ * attention moving from Q8KV8 to Q8KV4).  The pages name no format; the
+ * reading used is the OCP Microscaling (MX) formats, version 1.0: every 32
+ * consecutive values along a row share one power-of-two scale 2^X stored as
+ * an E8M0 byte (X + 127), X = floor(log2(max|x|)) - emax (emax 8 for e4m3, 2
+ * for e2m1; -127 for an all-zero block; clamped to [-127, 127]), and each
+ * element is the nearest value of its format to x / 2^X, ties to even,
+ * saturating at 448 (e4m3) or 6 (e2m1).  Q is MXFP8 (e4m3), K and V MXFP4
+ * (e2m1, two per byte, element 2i in the low nibble).
+ *
+ * msa_quantize_mx: x [rows][d] bf16 (d a multiple of 32) -> codes and scales.
+ *   fmt 0 (MSA_MX_E4M3): codes [rows][d] bytes; fmt 1 (MSA_MX_E2M1): codes
+ *   [rows][d/2] bytes.  scales [rows][d/32] bytes.  x and codes 16-byte
+ *   aligned; device pointers; rows = 0 is a no-op.  Inputs must be finite.
+ */
+#define MSA_MX_E4M3 0
+#define MSA_MX_E2M1 1
+MSA_API msa_status_t msa_quantize_mx(const void* x, int64_t rows, int32_t d, int32_t fmt,
+                                     void* codes, uint8_t* scales, msa_stream_t stream);
+
+/*
+ * msa_prefill on MX inputs: q8 [N][H][d] e4m3 with q_scale [N][H][d/32];
+ * k4, v4 [N][G][d/2] packed e2m1 with k_scale, v_scale [N][G][d/32] (as
+ * msa_quantize_mx writes them); q_idx, k_idx bf16 as for msa_prefill.  The
+ * three are dequantised exactly to bf16 (at most 4 significant bits times a
+ * power of two) in the last msa_workspace_size(PREFILL_Q8KV4) -
+ * msa_workspace_size(PREFILL) bytes of the workspace, and msa_prefill runs
+ * on them with the rest: the output is the bf16 prefill of the dequantised
+ * tensors.  ws: at least msa_prefill_min_workspace() plus those bytes (the
+ * query axis is then chunked as in msa_prefill).  Phase events
+ * (msa_set_phase_events) start at the index kernel, after the dequantisation.
+ */
+MSA_API msa_status_t msa_prefill_q8kv4(const msa_config_t* cfg, const void* q8,
+                                       const uint8_t* q_scale, const void* k4,
+                                       const uint8_t* k_scale, const void* v4,
+                                       const uint8_t* v_scale, const void* q_idx,
+                                       const void* k_idx, int64_t N, void* out, int32_t* ids_out,
+                                       void* ws, size_t ws_bytes, msa_stream_t stream);
 
 /*
  * msa_prefill plus the data of the Index Branch's KL alignment, forward only:

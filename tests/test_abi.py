@@ -167,6 +167,30 @@ def test_fp8_entry_points_checked_before_any_launch():
                                      1 << 30, None) == 1
 
 
+def test_mx_entry_points_checked_before_any_launch():
+    lib = msa.load_library()
+    p = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 21)
+    cfg = msa.config(8, 2, 128, 128, top_k=16)
+    # rows of a multiple of 32 values, a known element format, aligned pointers
+    assert lib.msa_quantize_mx(p, 4, 48, msa.MX_E4M3, p, p, None) == 1
+    assert lib.msa_quantize_mx(p, 4, 64, 7, p, p, None) == 1
+    assert lib.msa_quantize_mx(p, -1, 64, msa.MX_E2M1, p, p, None) == 1
+    assert lib.msa_quantize_mx(ctypes.c_void_p((1 << 20) + 8), 4, 64, msa.MX_E2M1, p, p,
+                               None) == 1
+    assert lib.msa_quantize_mx(p, 4, 64, msa.MX_E2M1, p, None, None) == 1
+    assert lib.msa_quantize_mx(None, 0, 64, msa.MX_E2M1, None, None, None) == 0  # no rows
+    # the three scale arrays are required
+    assert lib.msa_prefill_q8kv4(ctypes.byref(cfg), p, p, p, None, p, p, p, p, 256, p, None, ws,
+                                 1 << 30, None) == 1
+    # the dequantised q, k, v must fit behind the prefill's own workspace
+    need = msa.msa_workspace_size(cfg, msa.OP_PREFILL_Q8KV4, 256)
+    full = msa.msa_workspace_size(cfg, msa.OP_PREFILL, 256)
+    assert need - full == 256 * 8 * 128 * 2 + 2 * 256 * 2 * 128 * 2
+    assert lib.msa_prefill_q8kv4(ctypes.byref(cfg), p, p, p, p, p, p, p, p, 256, p, None, ws,
+                                 need - full, None) == 3  # MSA_ERR_WORKSPACE
+
+
 def test_decode_heads_per_group_limit():
     """Decode tiles a group's heads in 8s, at most 16; prefill takes up to 2048/d."""
     lib = msa.load_library()
