@@ -265,17 +265,27 @@ constexpr int kAttnThreads = 256;
 constexpr int kAttnWarps = kAttnThreads / 32;
 constexpr int kCandCap = 256;  // candidates kept for the exact ranking step
 
+template <int KSEL>
+struct SelScratch {
+  float wl_s[kAttnWarps][KSEL];  // each warp's best candidates, best first
+  int32_t wl_i[kAttnWarps][KSEL];
+  float tm_s[kAttnThreads];      // each warp's best thread bests
+  int32_t tm_i[kAttnThreads];
+  float cand_s[kCandCap];        // candidates not worse than the threshold
+  int32_t cand_i[kCandCap];
+};
+
 template <int D, int NT, int KSEL>
 struct AttnSmem {
+  // the sequence's pooled scores staged for the selection, in what is left
+  // of the V tiles' space next to the selection scratch
+  static constexpr int kStageCap =
+      (int)((sizeof(__nv_bfloat16) * 2 * kBlock * D - sizeof(SelScratch<KSEL>)) / sizeof(float));
   union {
     __nv_bfloat16 v[2][kBlock * D];  // attention: V tiles, 16-byte chunks swizzled by key
-    struct {                         // selection scratch (done before the first V copy)
-      float wl_s[kAttnWarps][KSEL];  // each warp's best candidates, best first
-      int32_t wl_i[kAttnWarps][KSEL];
-      float tm_s[kAttnThreads];      // each warp's best thread bests
-      int32_t tm_i[kAttnThreads];
-      float cand_s[kCandCap];        // candidates not worse than the threshold
-      int32_t cand_i[kCandCap];
+    struct {                         // selection (done before the first V copy)
+      SelScratch<KSEL> sel_scr;
+      float stage[kStageCap];
     };
   };
   __nv_bfloat16 p[NT * 8][kBlock + 8];     // P (heads x keys), padded rows: bf16(p)
@@ -352,6 +362,28 @@ __global__ void __launch_bounds__(kAttnThreads)
     const int64_t n_cand = (pooled_offset(cu, b) + nb > pooled_cap) ? 0 : nb - 1;
     const float* ps = pooled + pooled_offset(cu, b) * G + (int64_t)g * nb;  // [G][nb] per sequence
     const int want = (int)min64(top_k - 1, n_cand);
+    // the scores are staged in shared memory when they fit (8,191 candidates of
+    // a 1M-token sequence do at d = 128): their loads then go out 16 a thread at
+    // a time, once, instead of once per pass below
+    const bool staged = n_cand <= AttnSmem<D, NT, KSEL>::kStageCap;
+    if (staged) {
+      constexpr int kSB = 16;
+      for (int64_t j0 = tid; j0 < n_cand; j0 += kSB * kAttnThreads) {
+        float v[kSB];
+#pragma unroll
+        for (int c = 0; c < kSB; ++c) {
+          const int64_t j = j0 + (int64_t)c * kAttnThreads;
+          v[c] = j < n_cand ? __ldg(ps + j) : 0.f;
+        }
+#pragma unroll
+        for (int c = 0; c < kSB; ++c) {
+          const int64_t j = j0 + (int64_t)c * kAttnThreads;
+          if (j < n_cand) sm.stage[j] = v[c];
+        }
+      }
+      __syncthreads();
+    }
+    auto cand = [&](int64_t j) { return staged ? sm.stage[j] : __ldg(ps + j); };
     constexpr int kBatch = 8;
     float best_s = -INFINITY;
     int32_t best_i = 0x7FFFFFFF;
@@ -360,7 +392,7 @@ __global__ void __launch_bounds__(kAttnThreads)
 #pragma unroll
       for (int c = 0; c < kBatch; ++c) {
         const int64_t j = j0 + (int64_t)c * kAttnThreads;
-        v[c] = j < n_cand ? __ldg(ps + j) : -INFINITY;
+        v[c] = j < n_cand ? cand(j) : -INFINITY;
       }
 #pragma unroll
       for (int c = 0; c < kBatch; ++c) {
@@ -383,7 +415,7 @@ __global__ void __launch_bounds__(kAttnThreads)
           if (better(s2, i2, sc, id)) sc = s2, id = i2;
         }
         if (mi == id) ms = -INFINITY, mi = 0x7FFFFFFF;  // the owner drops it
-        if (lane == 0) sm.tm_s[warp * R + round] = sc, sm.tm_i[warp * R + round] = id;
+        if (lane == 0) sm.sel_scr.tm_s[warp * R + round] = sc, sm.sel_scr.tm_i[warp * R + round] = id;
       }
     }
     if (tid == 0) {
@@ -397,10 +429,10 @@ __global__ void __launch_bounds__(kAttnThreads)
     if (warp == 0 && want > 0) {
       // thr = the want-th best of the 8R collected (lane x ranks entry x)
       for (int x = lane; x < kAttnWarps * R; x += 32) {
-        const float sx = sm.tm_s[x];
-        const int32_t ix = sm.tm_i[x];
+        const float sx = sm.sel_scr.tm_s[x];
+        const int32_t ix = sm.sel_scr.tm_i[x];
         int rank = 0;
-        for (int y = 0; y < kAttnWarps * R; ++y) rank += better(sm.tm_s[y], sm.tm_i[y], sx, ix);
+        for (int y = 0; y < kAttnWarps * R; ++y) rank += better(sm.sel_scr.tm_s[y], sm.sel_scr.tm_i[y], sx, ix);
         if (rank == want - 1) sm.thr_s = sx, sm.thr_i = ix;
       }
     }
@@ -414,14 +446,14 @@ __global__ void __launch_bounds__(kAttnThreads)
 #pragma unroll
         for (int c = 0; c < kBatch; ++c) {
           const int64_t j = j0 + (int64_t)c * kAttnThreads;
-          v[c] = j < n_cand ? __ldg(ps + j) : -INFINITY;
+          v[c] = j < n_cand ? cand(j) : -INFINITY;
         }
 #pragma unroll
         for (int c = 0; c < kBatch; ++c) {
           const int64_t j = j0 + (int64_t)c * kAttnThreads;
           if (j < n_cand && !better(ts, ti, v[c], (int32_t)j)) {
             const int x = atomicAdd(&sm.ncand, 1);
-            if (x < kCandCap) sm.cand_s[x] = v[c], sm.cand_i[x] = (int32_t)j;
+            if (x < kCandCap) sm.sel_scr.cand_s[x] = v[c], sm.sel_scr.cand_i[x] = (int32_t)j;
           }
         }
       }
@@ -431,17 +463,17 @@ __global__ void __launch_bounds__(kAttnThreads)
     if (nc <= kCandCap) {
       // exact ranks among the collected: the best `want` go to pick[0..want)
       for (int x = tid; x < nc; x += kAttnThreads) {
-        const float s_x = sm.cand_s[x];
-        const int32_t i_x = sm.cand_i[x];
+        const float s_x = sm.sel_scr.cand_s[x];
+        const int32_t i_x = sm.sel_scr.cand_i[x];
         int rank = 0;
-        for (int y = 0; y < nc; ++y) rank += better(sm.cand_s[y], sm.cand_i[y], s_x, i_x);
+        for (int y = 0; y < nc; ++y) rank += better(sm.sel_scr.cand_s[y], sm.sel_scr.cand_i[y], s_x, i_x);
         if (rank < want) sm.pick[rank] = i_x;
       }
     } else {
       // fallback: per-thread lists, then warp tournaments
       TopList<KSEL> list;
       list.init();
-      for (int64_t j = tid; j < n_cand; j += kAttnThreads) list.insert(__ldg(ps + j), (int32_t)j);
+      for (int64_t j = tid; j < n_cand; j += kAttnThreads) list.insert(cand(j), (int32_t)j);
       for (int round = 0; round < want; ++round) {
         float sc = list.sc[0];
         int32_t id = list.id[0];
@@ -452,7 +484,7 @@ __global__ void __launch_bounds__(kAttnThreads)
           if (better(s2, i2, sc, id)) sc = s2, id = i2;
         }
         if (list.id[0] == id) list.pop();  // real ids are unique; empty heads pop harmlessly
-        if (lane == 0) sm.wl_s[warp][round] = sc, sm.wl_i[warp][round] = id;
+        if (lane == 0) sm.sel_scr.wl_s[warp][round] = sc, sm.sel_scr.wl_i[warp][round] = id;
       }
       __syncthreads();
       if (warp == 0) {
@@ -460,7 +492,7 @@ __global__ void __launch_bounds__(kAttnThreads)
         wl.init();
 #pragma unroll
         for (int i = 0; i < KSEL; ++i)
-          if (lane < kAttnWarps && i < want) wl.sc[i] = sm.wl_s[lane][i], wl.id[i] = sm.wl_i[lane][i];
+          if (lane < kAttnWarps && i < want) wl.sc[i] = sm.sel_scr.wl_s[lane][i], wl.id[i] = sm.sel_scr.wl_i[lane][i];
         for (int round = 0; round < want; ++round) {
           float sc = wl.sc[0];
           int32_t id = wl.id[0];

@@ -117,39 +117,51 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const __nv_bfloat16* __re
 }
 
 // codes and scales -> bf16, exactly (see the file header).  Thread t handles
-// elements 8t .. 8t+7.
+// block t: 32 (e4m3) or 16 (e2m1) bytes of codes in, 64 bytes of bf16 out, so
+// that enough bytes are in flight to stream at HBM rate.
 template <int FMT>
 __global__ void __launch_bounds__(256) mx_dequant_kernel(const uint8_t* __restrict__ codes,
                                                          const uint8_t* __restrict__ scales,
                                                          int64_t n_blocks,
                                                          __nv_bfloat16* __restrict__ out) {
-  const int64_t n_threads = n_blocks * (kMxBlock / kPer);
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_threads; t += stride) {
-    const int X = (int)__ldg(scales + (t >> 2)) - 127;
-    float v[kPer];
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n_blocks; b += stride) {
+    const int X = (int)__ldg(scales + b) - 127;
+    uint32_t w[8];  // the block's codes: 8 words of 4 e4m3 bytes, or 4 words of 8 nibbles
     if (FMT == kMxE4m3) {
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(codes) + t);
+      const uint4 c0 = __ldg(reinterpret_cast<const uint4*>(codes) + 2 * b);
+      const uint4 c1 = __ldg(reinterpret_cast<const uint4*>(codes) + 2 * b + 1);
+      w[0] = c0.x, w[1] = c0.y, w[2] = c0.z, w[3] = c0.w;
+      w[4] = c1.x, w[5] = c1.y, w[6] = c1.z, w[7] = c1.w;
+    } else {
+      const uint4 c = __ldg(reinterpret_cast<const uint4*>(codes) + b);
+      w[0] = c.x, w[1] = c.y, w[2] = c.z, w[3] = c.w;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out) + 4 * b;
+    // v * 2^X by one multiply, exact while 2^X and the product stay normal
+    // (elements are at least 2^-9 in magnitude, or zero); ldexpf otherwise
+    const bool mul = X >= -110 && X <= 120;
+    const float p2 = __uint_as_float((uint32_t)(mul ? X + 127 : 127) << 23);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // elements 8q .. 8q+7
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (FMT == kMxE4m3)
+          v[i] = from_e4m3((w[2 * q + i / 4] >> (8 * (i % 4))) & 0xFF);
+        else
+          v[i] = from_e2m1((w[q] >> (4 * i)) & 0xF);
+        v[i] = mul ? v[i] * p2 : ldexpf(v[i], X);
+      }
+      uint4 o;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        v[i] = from_e4m3((w.x >> (8 * i)) & 0xFF);
-        v[4 + i] = from_e4m3((w.y >> (8 * i)) & 0xFF);
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        ow[i] = *reinterpret_cast<const uint32_t*>(&h2);
       }
-    } else {
-      const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(codes) + t);
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) v[i] = from_e2m1((w >> (4 * i)) & 0xF);
+      dst[q] = o;
     }
-    uint4 o;
-    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-    for (int i = 0; i < kPer / 2; ++i) {
-      // ldexpf is exact; the bf16 rounding is then exact for representable values
-      const __nv_bfloat16 a = __float2bfloat16_rn(ldexpf(v[2 * i], X));
-      const __nv_bfloat16 b = __float2bfloat16_rn(ldexpf(v[2 * i + 1], X));
-      ow[i] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
-    }
-    reinterpret_cast<uint4*>(out)[t] = o;
   }
 }
 
@@ -177,7 +189,7 @@ cudaError_t launch_mx_quantize(const void* x, int64_t n_blocks, int fmt, void* c
 cudaError_t launch_mx_dequantize(const void* codes, const uint8_t* scales, int64_t n_blocks,
                                  int fmt, void* out, int sms, cudaStream_t s) {
   if (n_blocks <= 0) return cudaSuccess;
-  const unsigned g = grid_for(n_blocks * 4, sms);
+  const unsigned g = grid_for(n_blocks, sms);
   const auto* c = static_cast<const uint8_t*>(codes);
   auto* o = static_cast<__nv_bfloat16*>(out);
   if (fmt == kMxE4m3)
