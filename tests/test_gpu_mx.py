@@ -100,6 +100,42 @@ def _check(msa, s, inp, rows):
     return out
 
 
+@pytest.mark.parametrize("rows,d", [(1, 32), (3, 64), (1000, 96)])
+def test_quantize_mx_small_shapes(msa, rows, d):
+    g = torch.Generator().manual_seed(rows + d)
+    x = (torch.randn((rows, d), generator=g) * 5.0).to(torch.bfloat16).cuda()
+    for fmt in (msa.MX_E4M3, msa.MX_E2M1):
+        codes, scales = msa.msa_quantize_mx(x, fmt)
+        want_c, want_s = oracle.mx_quantize(x.cpu(), fmt)
+        if fmt == msa.MX_E2M1:
+            want_c = oracle.pack_e2m1(want_c)
+        assert np.array_equal(scales.cpu().numpy(), want_s)
+        assert np.array_equal(codes.cpu().numpy(), want_c)
+
+
+def test_prefill_q8kv4_chunked_equals_one_shot(msa):
+    """A workspace that holds only part of the query axis: the prefill runs in
+    query chunks behind the dequantised tensors and gives the same bytes."""
+    s = synth.PrefillShape("mxc", N=2000, H=16, G=2, d=128, d_idx=128, top_k=8, n_needles=2,
+                           seed=77)
+    inp = synth.make_prefill_inputs(s, device="cuda")
+    cfg = msa.config(s.H, s.G, s.d, s.d_idx, top_k=s.top_k, block=s.block, scale=s.scale)
+    q8, qs, k4, ks, v4, vs = _quantised_inputs(msa, inp)
+    full = msa.msa_workspace_size(cfg, msa.OP_PREFILL_Q8KV4, s.N)
+    dq = full - msa.msa_workspace_size(cfg, msa.OP_PREFILL, s.N)
+    small = msa.msa_prefill_min_workspace(cfg, s.N) + dq + 4096
+    outs = []
+    for size in (full, small):
+        ws = torch.empty(size, dtype=torch.uint8, device="cuda")
+        out, ids = msa.msa_prefill_q8kv4(cfg, q8, qs, k4, ks, v4, vs, inp["q_idx"], inp["k_idx"],
+                                         ids_out=True, workspace=ws)
+        torch.cuda.synchronize()
+        assert msa.msa_get_device_error(ws) == 0
+        outs.append((out.clone(), ids.clone()))
+    assert msa.msa_prefill_chunk_tokens(cfg, s.N, small - dq, ids_returned=True) < s.N
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
 def test_prefill_q8kv4_tiny_all_rows(msa):
     s = synth.PREFILL_CONFIGS["tiny"]
     inp = synth.make_prefill_inputs(s, device="cuda")
