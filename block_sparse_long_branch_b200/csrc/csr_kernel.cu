@@ -7,17 +7,20 @@
 // Deterministic stable counting sort on the key (g, j), in t order, over
 // parts of R query rows (R grows with nb so that the (part, list) count table
 // stays at most half the size of the ids):
-//   1. count   : per part and group, a shared-memory histogram over the key
-//                blocks -> cnt[part][g*nb + j] (coalesced) and the list totals
-//                (atomics); the last CTA scans the totals into row_ptr and
-//                cuts the lists into Main Branch work units
+//   1. count   : per part and set of groups (all whose bins fit shared
+//                memory), a histogram over the key blocks -> cnt[part][g*nb +
+//                j] (coalesced) and the list totals (atomics); the last CTA
+//                scans the totals into row_ptr and cuts the lists into Main
+//                Branch work units
 //   2. colscan : the table scanned in (list, part) order, in place, from
 //                row_ptr: where each part's hits on each list start
 //   3. scatter : one warp per (part, set of groups) loads its part's start
 //                offsets, then walks the rows in t order, one row of every
 //                group of the set per step; the hits of one step never share
 //                a key, so each advances its key's offset by one
-// HBM-bound integer work: each id is read twice, each entry written once.
+// Integer work: each id is read twice and each entry written once.  At the
+// sizes measured it is bound by latency and by the scatter's stores (one
+// row step writes 32 entries of 32 different lists), not by HBM bandwidth.
 //
 // For a batch of packed sequences the ids are local to each sequence; the key
 // is row_base[row] + id, a global block number.  The plan kernels at the end
