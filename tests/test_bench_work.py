@@ -11,7 +11,7 @@ def test_index_flops_counts_every_non_local_visible_key():
     for N, G, di in [(700, 2, 64), (129, 1, 128), (128, 4, 64), (1, 8, 128)]:
         keys = sum(128 * (t // 128) for t in range(N))  # whole blocks before the local one
         assert bench.index_flops(N, G, di) == 2.0 * di * G * keys
-    # the 32K workload: 1.095e12, as derived independently for the survey of the path
+    # the 32K workload: 1.095e12, derived independently by hand
     assert abs(bench.index_flops(32768, 8, 128) - 1.095e12) / 1.095e12 < 1e-3
 
 
