@@ -117,40 +117,52 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const __nv_bfloat16* __re
 }
 
 // codes and scales -> bf16, exactly (see the file header).  Thread t handles
-// block t: 32 (e4m3) or 16 (e2m1) bytes of codes in, 64 bytes of bf16 out, so
-// that enough bytes are in flight to stream at HBM rate.
+// chunk t: elements 8t .. 8t+7 of block t/4, that is 8 (e4m3) or 4 (e2m1)
+// bytes of codes in and 16 bytes of bf16 out, so a warp's loads and stores
+// each cover one contiguous run.  A thread issues the loads of kDqDepth chunks
+// (one grid stride apart) before it converts any of them.  The grid is one
+// resident wave (kDqCtasPerSm CTAs per SM), so no CTA waits for a second wave.
+constexpr int kDqDepth = 8;
+constexpr int kDqCtasPerSm = 6;
+
 template <int FMT>
-__global__ void __launch_bounds__(256) mx_dequant_kernel(const uint8_t* __restrict__ codes,
-                                                         const uint8_t* __restrict__ scales,
-                                                         int64_t n_blocks,
-                                                         __nv_bfloat16* __restrict__ out) {
+__global__ void __launch_bounds__(256, kDqCtasPerSm)
+    mx_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                      int64_t n_blocks, __nv_bfloat16* __restrict__ out) {
+  const int64_t n_chunks = n_blocks * (kMxBlock / kPer);
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n_blocks; b += stride) {
-    const int X = (int)__ldg(scales + b) - 127;
-    uint32_t w[8];  // the block's codes: 8 words of 4 e4m3 bytes, or 4 words of 8 nibbles
-    if (FMT == kMxE4m3) {
-      const uint4 c0 = __ldg(reinterpret_cast<const uint4*>(codes) + 2 * b);
-      const uint4 c1 = __ldg(reinterpret_cast<const uint4*>(codes) + 2 * b + 1);
-      w[0] = c0.x, w[1] = c0.y, w[2] = c0.z, w[3] = c0.w;
-      w[4] = c1.x, w[5] = c1.y, w[6] = c1.z, w[7] = c1.w;
-    } else {
-      const uint4 c = __ldg(reinterpret_cast<const uint4*>(codes) + b);
-      w[0] = c.x, w[1] = c.y, w[2] = c.z, w[3] = c.w;
-    }
-    uint4* dst = reinterpret_cast<uint4*>(out) + 4 * b;
-    // v * 2^X by one multiply, exact while 2^X and the product stay normal
-    // (elements are at least 2^-9 in magnitude, or zero); ldexpf otherwise
-    const bool mul = X >= -110 && X <= 120;
-    const float p2 = __uint_as_float((uint32_t)(mul ? X + 127 : 127) << 23);
+  for (int64_t c0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c0 < n_chunks;
+       c0 += kDqDepth * stride) {
+    uint2 w[kDqDepth];  // e4m3: 8 codes in x and y; e2m1: 8 nibbles in x
+    uint32_t sx[kDqDepth / 4] = {};  // the chunks' scale bytes, four to a word
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {  // elements 8q .. 8q+7
-      float v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
+    for (int u = 0; u < kDqDepth; ++u) {
+      const int64_t c = c0 + u * stride;
+      w[u] = make_uint2(0, 0);
+      if (c < n_chunks) {
         if (FMT == kMxE4m3)
-          v[i] = from_e4m3((w[2 * q + i / 4] >> (8 * (i % 4))) & 0xFF);
+          w[u] = __ldg(reinterpret_cast<const uint2*>(codes) + c);
         else
-          v[i] = from_e2m1((w[q] >> (4 * i)) & 0xF);
+          w[u].x = __ldg(reinterpret_cast<const uint32_t*>(codes) + c);
+        sx[u / 4] |= (uint32_t)__ldg(scales + (c >> 2)) << (8 * (u % 4));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kDqDepth; ++u) {
+      const int64_t c = c0 + u * stride;
+      if (c >= n_chunks) break;
+      const int X = (int)((sx[u / 4] >> (8 * (u % 4))) & 0xFF) - 127;
+      // v * 2^X by one multiply, exact while 2^X and the product stay normal
+      // (elements are at least 2^-9 in magnitude, or zero); ldexpf otherwise
+      const bool mul = X >= -110 && X <= 120;
+      const float p2 = __uint_as_float((uint32_t)(mul ? X + 127 : 127) << 23);
+      float v[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        if (FMT == kMxE4m3)
+          v[i] = from_e4m3(((i < 4 ? w[u].x : w[u].y) >> (8 * (i % 4))) & 0xFF);
+        else
+          v[i] = from_e2m1((w[u].x >> (4 * i)) & 0xF);
         v[i] = mul ? v[i] * p2 : ldexpf(v[i], X);
       }
       uint4 o;
@@ -160,14 +172,14 @@ __global__ void __launch_bounds__(256) mx_dequant_kernel(const uint8_t* __restri
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
         ow[i] = *reinterpret_cast<const uint32_t*>(&h2);
       }
-      dst[q] = o;
+      reinterpret_cast<uint4*>(out)[c] = o;
     }
   }
 }
 
-unsigned grid_for(int64_t n_threads, int sms) {
+unsigned grid_for(int64_t n_threads, int sms, int ctas_per_sm = 16) {
   const int64_t want = (n_threads + 255) / 256;
-  const int64_t cap = (int64_t)sms * 16;
+  const int64_t cap = (int64_t)sms * ctas_per_sm;
   return (unsigned)(want < 1 ? 1 : (want > cap ? cap : want));
 }
 
@@ -189,7 +201,7 @@ cudaError_t launch_mx_quantize(const void* x, int64_t n_blocks, int fmt, void* c
 cudaError_t launch_mx_dequantize(const void* codes, const uint8_t* scales, int64_t n_blocks,
                                  int fmt, void* out, int sms, cudaStream_t s) {
   if (n_blocks <= 0) return cudaSuccess;
-  const unsigned g = grid_for(n_blocks, sms);
+  const unsigned g = grid_for((n_blocks * 4 + kDqDepth - 1) / kDqDepth, sms, kDqCtasPerSm);
   const auto* c = static_cast<const uint8_t*>(codes);
   auto* o = static_cast<__nv_bfloat16*>(out);
   if (fmt == kMxE4m3)
