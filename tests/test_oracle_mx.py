@@ -111,12 +111,18 @@ def test_quantisation_error_is_within_half_a_step(fmt):
 
 
 def test_dequantised_values_are_exact_in_bf16():
+    # an element has at most 4 significant bits and the scale is a power of two,
+    # so the product is a bf16 value (8 significant bits) while it stays normal;
+    # rows span block magnitudes from 2^-100 to 2^100
     rng = np.random.default_rng(17)
-    x = _bf16(rng.standard_normal((16, 128)) * 3.0)
+    mag = np.exp2(np.linspace(-100, 100, 16))[:, None]
+    x = _bf16(rng.standard_normal((16, 128)) * 3.0 * mag)
     for fmt in (oracle.MX_E4M3, oracle.MX_E2M1):
         codes, scales = oracle.mx_quantize(x, fmt)
-        bits = oracle.f64_to_bf16_bits(oracle.mx_dequantize(codes, scales, fmt))
-        assert bits.shape == (16, 128)
+        deq = oracle.mx_dequantize(codes, scales, fmt)
+        back = oracle.bf16_bits_to_f64(oracle.f64_to_bf16_bits(deq))
+        assert np.array_equal(back, deq)
+        assert np.count_nonzero(deq) > deq.size // 2
 
 
 def test_e2m1_packing_puts_even_elements_in_the_low_nibble():
